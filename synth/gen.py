@@ -1,0 +1,181 @@
+"""Host (numpy) half of the counter-based input generator; see the package
+docstring for the definition.  Also holds the workload presets and the input
+recipe of each one."""
+
+from __future__ import annotations
+
+import math
+from dataclasses import dataclass
+
+import numpy as np
+
+_M64 = (1 << 64) - 1
+_GOLDEN = 0x9E3779B97F4A7C15
+_TENSOR_MUL = 0xD1B54A32D192ED03
+_C1 = 0xBF58476D1CE4E5B9
+_C2 = 0x94D049BB133111EB
+IRWIN_HALL_MEAN = 12 * 65535 // 2  # 393210: the sum of twelve U{0..65535} has mean 393210
+
+TENSOR_X, TENSOR_WG, TENSOR_W1, TENSOR_W3, TENSOR_W2 = 1, 2, 3, 4, 5
+
+# Skewed-routing recipe: channel d-1 of x is the constant 1 and the router's
+# weight for that channel is a Zipf-shaped log prior b_e = -beta * s * ln(e+1)
+# (s = 1.2).  beta was calibrated on seed 0 at T = 16384 so that expert 0
+# receives 35% of the T*k assignments (the script that finds it is
+# tests/golden/calibrate_skew.py; a CPU test checks the share).
+SKEW_ZIPF_S = 1.2
+SKEW_BETA = 0.791126
+
+
+def _mix_int(z: int) -> int:
+    z &= _M64
+    z ^= z >> 30
+    z = (z * _C1) & _M64
+    z ^= z >> 27
+    z = (z * _C2) & _M64
+    return z ^ (z >> 31)
+
+
+def _mix_arr(z: np.ndarray) -> np.ndarray:
+    with np.errstate(over="ignore"):
+        z = z ^ (z >> np.uint64(30))
+        z = z * np.uint64(_C1)
+        z = z ^ (z >> np.uint64(27))
+        z = z * np.uint64(_C2)
+        return z ^ (z >> np.uint64(31))
+
+
+def tensor_id(kind: int, layer: int = 0) -> int:
+    """Tensor id of tensor `kind` (TENSOR_*) of layer `layer`."""
+    return layer * 8 + kind
+
+
+def _key(seed: int, tid: int) -> int:
+    return _mix_int(seed * _GOLDEN + tid * _TENSOR_MUL)
+
+
+def normal_u16bits_f32(seed: int, tid: int, start: int, count: int) -> np.ndarray:
+    """z values (fp32, exact) for element indices [start, start+count)."""
+    key = np.uint64(_key(seed, tid))
+    i = np.arange(start, start + count, dtype=np.uint64)
+    s = np.zeros(count, dtype=np.int64)
+    with np.errstate(over="ignore"):
+        base = i * np.uint64(3)
+        for j in range(3):
+            w = _mix_arr(key + (base + np.uint64(j + 1)) * np.uint64(_GOLDEN))
+            for q in range(4):
+                s += ((w >> np.uint64(16 * q)) & np.uint64(0xFFFF)).astype(np.int64)
+    return (s - IRWIN_HALL_MEAN).astype(np.float32) * np.float32(1.0 / 65536.0)
+
+
+def bf16_round_bits(v: np.ndarray) -> np.ndarray:
+    """fp32 -> bf16 bit pattern, round to nearest even (finite inputs)."""
+    u = np.ascontiguousarray(v, dtype=np.float32).view(np.uint32).astype(np.uint64)
+    u = u + np.uint64(0x7FFF) + ((u >> np.uint64(16)) & np.uint64(1))
+    return (u >> np.uint64(16)).astype(np.uint16)
+
+
+def bf16_bits_to_f32(b: np.ndarray) -> np.ndarray:
+    return (np.asarray(b, dtype=np.uint16).astype(np.uint32) << np.uint32(16)).view(np.float32)
+
+
+def bf16_bits_to_f64(b: np.ndarray) -> np.ndarray:
+    return bf16_bits_to_f32(b).astype(np.float64)
+
+
+def normal_values(seed: int, tid: int, count: int, sigma: float, dtype: str,
+                  start: int = 0, chunk: int = 1 << 22) -> np.ndarray:
+    """count values N(0, sigma^2): uint16 bf16 bits for dtype 'bf16', fp32 for 'f32'."""
+    out = np.empty(count, dtype=np.uint16 if dtype == "bf16" else np.float32)
+    sig = np.float32(sigma)
+    for c0 in range(0, count, chunk):
+        n = min(chunk, count - c0)
+        v = normal_u16bits_f32(seed, tid, start + c0, n) * sig
+        out[c0:c0 + n] = bf16_round_bits(v) if dtype == "bf16" else v
+    return out
+
+
+def sigma_of(kind: int, d: int, f: int) -> float:
+    """Scale of each tensor: x ~ N(0,1); Wg, W1, W3 ~ N(0, 1/d); W2 ~ N(0, 1/f)."""
+    if kind == TENSOR_X:
+        return 1.0
+    if kind in (TENSOR_WG, TENSOR_W1, TENSOR_W3):
+        return float(np.float32(1.0 / math.sqrt(d)))
+    if kind == TENSOR_W2:
+        return float(np.float32(1.0 / math.sqrt(f)))
+    raise ValueError(kind)
+
+
+def skew_biases(E: int, beta: float, dtype: str) -> np.ndarray:
+    """Router weights of the constant channel: b_e = -beta * s * ln(e + 1)."""
+    b = np.array([-beta * SKEW_ZIPF_S * math.log(e + 1) for e in range(E)], dtype=np.float32)
+    return bf16_round_bits(b) if dtype == "bf16" else b
+
+
+@dataclass(frozen=True)
+class MoEShape:
+    name: str
+    T: int
+    d: int
+    f: int
+    E: int
+    k: int
+    dtype: str          # "bf16" or "f32"
+    skew: bool = False  # constant channel + Zipf log-prior in Wg
+    layers: int = 1
+
+    @property
+    def flops(self) -> float:
+        """Algorithmic flops of one layer: router 2dE per token, and per
+        assignment 4df (W1, W3) + 2df (W2)."""
+        return float(self.T) * (2 * self.d * self.E + self.k * 6 * self.d * self.f) * self.layers
+
+    @property
+    def weight_bytes(self) -> int:
+        esz = 2 if self.dtype == "bf16" else 4
+        return (3 * self.E * self.d * self.f + self.E * self.d) * esz * self.layers
+
+
+CONFIGS = {
+    "tiny": MoEShape("tiny", 16, 64, 128, 8, 2, "f32"),
+    "decode": MoEShape("decode", 32, 4096, 14336, 8, 2, "bf16"),
+    "prefill": MoEShape("prefill", 4096, 4096, 14336, 8, 2, "bf16"),
+    "skewed": MoEShape("skewed", 16384, 4096, 14336, 8, 2, "bf16", skew=True),
+    "stack": MoEShape("stack", 8192, 4096, 14336, 8, 2, "bf16", layers=32),
+}
+
+
+def host_inputs(shape: MoEShape, seed: int = 0, layer: int = 0, with_x: bool = True,
+                skew_beta: float | None = None, with_experts: bool = True) -> dict:
+    """All inputs of one layer as numpy arrays (bf16 as uint16 bit patterns).
+
+    Layouts: x [T, d]; Wg [E, d]; W1, W3 [E, f, d]; W2 [E, d, f]; row-major.
+    """
+    T, d, f, E, dt = shape.T, shape.d, shape.f, shape.E, shape.dtype
+    out = {}
+    if with_x:
+        out["x"] = normal_values(seed, tensor_id(TENSOR_X, layer), T * d,
+                                 sigma_of(TENSOR_X, d, f), dt).reshape(T, d)
+    out["Wg"] = normal_values(seed, tensor_id(TENSOR_WG, layer), E * d,
+                              sigma_of(TENSOR_WG, d, f), dt).reshape(E, d)
+    if not with_experts:
+        if shape.skew:
+            apply_skew(out, E, SKEW_BETA if skew_beta is None else skew_beta, dt)
+        return out
+    out["W1"] = normal_values(seed, tensor_id(TENSOR_W1, layer), E * f * d,
+                              sigma_of(TENSOR_W1, d, f), dt).reshape(E, f, d)
+    out["W3"] = normal_values(seed, tensor_id(TENSOR_W3, layer), E * f * d,
+                              sigma_of(TENSOR_W3, d, f), dt).reshape(E, f, d)
+    out["W2"] = normal_values(seed, tensor_id(TENSOR_W2, layer), E * d * f,
+                              sigma_of(TENSOR_W2, d, f), dt).reshape(E, d, f)
+    if shape.skew:
+        apply_skew(out, E, SKEW_BETA if skew_beta is None else skew_beta, dt)
+    return out
+
+
+def apply_skew(t: dict, E: int, beta: float, dtype: str) -> None:
+    """Make channel d-1 of x the constant 1 and put the Zipf log prior in Wg."""
+    one = bf16_round_bits(np.ones(1, np.float32))[0] if dtype == "bf16" else np.float32(1.0)
+    if "x" in t:
+        t["x"][:, -1] = one
+    t["Wg"][:, -1] = skew_biases(E, beta, dtype)
