@@ -1,0 +1,422 @@
+#!/usr/bin/env python
+"""Throughput of the sparse MoE feed-forward layer (Mixtral 8x7B shapes) on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload prefill|decode|skewed]
+                    [--impl ours|reference] [--no-extras]
+
+A step is one full layer (router, permutation, both grouped GEMMs, combine)
+over the workload's T tokens, through the C ABI (moe_layer_forward_ex), with
+inputs resident in HBM.  Default workload: the prefill layer, T = 4096
+tokens, d = 4096, f = 14336, E = 8, top-2, bf16.  With N > 1 (torchrun, one
+process per GPU) every rank runs its own T tokens on its own replica of the
+weights; the layer needs no exchange between ranks, so there is no
+collective on the data path (weak scaling).  Rank 0 prints one JSON line.
+
+Timing: W untimed warm-up steps, then K steps between a barrier and a device
+synchronisation on both sides; each step is bracketed by CUDA events on the
+launching stream and the L2 is flushed (a 512 MiB write) between steps,
+outside the events.  The elapsed time is the max over ranks.
+
+--impl reference times the fp64 CPU oracle on the host cores (rank 0 only)
+on a bounded sample of the same workload.
+"""
+
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "MoE-layer tokens/sec and TFLOP/s (fraction of bf16 peak / HBM GB/s) on 1 B200"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=300)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--workload", default="prefill", choices=["prefill", "decode", "skewed"])
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-extras", action="store_true", help="skip the decode line and the CPU baseline")
+    ap.add_argument("--cpu-sample", type=int, default=32, help="tokens in the oracle's timed sample")
+    return ap.parse_args()
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return d, "measured"
+    return FALLBACK_PEAKS, "fallback"
+
+
+def workload_desc(s, n):
+    return {"workload": "Mixtral-8x7B MoE FFN layer, %s: T=%d tokens per GPU, d=%d, f=%d, E=%d, top-%d, %s"
+                        % (s.name, s.T, s.d, s.f, s.E, s.k, s.dtype),
+            "T": s.T, "d": s.d, "f": s.f, "E": s.E, "k": s.k, "routing": "skewed (Zipf log prior, hottest expert 35%)"
+            if s.skew else "near-uniform (Wg ~ N(0, 1/d))",
+            "global_batch_tokens": s.T * n, "parallelism": "replicas x%d (token-sharded, no collective)" % n,
+            "l2": "flushed between timed steps (512 MiB write outside the step events); weights 2.82 GB > L2"}
+
+
+class ClockSampler:
+    """nvidia-smi samples every 200 ms while the timed region runs."""
+
+    FIELDS = ("index,pci.bus_id,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, bus_id):
+        self.bus_id = (bus_id or "").lower()
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        try:
+            fd, self.path = tempfile.mkstemp(suffix=".csv")
+            os.close(fd)
+            self.proc = subprocess.Popen(["nvidia-smi", "--query-gpu=" + self.FIELDS, "--format=csv,noheader,nounits",
+                                          "-lms", "200", "-f", self.path], stdout=subprocess.DEVNULL,
+                                         stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        rows = []
+        for line in open(self.path):
+            f = [c.strip() for c in line.split(",")]
+            if len(f) < 10:
+                continue
+            if self.bus_id and self.bus_id[-12:] not in f[1].lower():
+                continue
+            rows.append(f)
+        os.unlink(self.path)
+        if not rows:
+            return None
+        sm = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+        mx = max(float(r[3]) for r in rows if r[3].replace(".", "").isdigit())
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[6 + i].lower().startswith("active")})
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": mx, "reasons": reasons,
+                "samples": len(rows), "power_w_max": max(float(r[4]) for r in rows if r[4].replace(".", "").isdigit())}
+
+
+def gemm_source_hash():
+    p = os.path.join(ROOT, "sparse_mixture_experts_06_b200", "csrc", "gemm_sm100.cu")
+    return hashlib.sha256(open(p, "rb").read()).hexdigest()[:16]
+
+
+def traffic_record(kernel):
+    """DRAM bytes per launch from the committed ncu summary, if it was taken on this kernel source."""
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(p):
+        return None
+    d = json.load(open(p)).get(kernel)
+    if not d or d.get("source_sha256_16") != gemm_source_hash():
+        return None
+    return d
+
+
+# --------------------------------------------------------------------- oracle (CPU) side
+
+def oracle_weights_f64(t, E):
+    """Host fp64 copies of the weights (input marshalling for the oracle)."""
+    import numpy as np
+    import synth
+    from synth.device import to_host_bits
+    out = {}
+    for name in ("W1", "W3", "W2"):
+        bits = to_host_bits(t[name])
+        out[name] = np.stack([synth.bf16_bits_to_f64(bits[e]) for e in range(E)])
+    out["Wg"] = synth.bf16_bits_to_f64(to_host_bits(t["Wg"]))
+    return out
+
+
+def time_oracle(w64, x_bits, k):
+    """Times oracle.moe_forward on the host rows x_bits (as it stands)."""
+    import oracle
+    import synth
+    from threadpoolctl import threadpool_info
+    x64 = synth.bf16_bits_to_f64(x_bits)
+    t0 = time.perf_counter()
+    oracle.moe_forward(x64, w64["Wg"], w64["W1"], w64["W3"], w64["W2"], k)
+    dt = time.perf_counter() - t0
+    threads = max([i.get("num_threads", 1) for i in threadpool_info()] + [1])
+    return dt, threads
+
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    import numpy as np
+    import torch
+    import synth
+    from synth.device import device_inputs, to_host_bits
+    s = synth.CONFIGS[args.workload]
+    t = device_inputs(s, 0)
+    w64 = oracle_weights_f64(t, s.E)
+    x_bits = to_host_bits(t["x"])
+    del t
+    torch.cuda.empty_cache()
+    n = args.cpu_sample
+    rng = np.random.default_rng(0)
+    times = []
+    threads = 1
+    for i in range(args.warmup + args.steps):
+        rows = np.sort(rng.choice(s.T, size=min(n, s.T), replace=False))
+        dt, threads = time_oracle(w64, x_bits[rows], s.k)
+        if i >= args.warmup:
+            times.append(dt)
+    tot = sum(times)
+    value = len(times) * min(n, s.T) / tot
+    line = {"metric": METRIC, "impl": "reference", "value": value, "unit": "tokens/s", "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * tot / len(times),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic", "config": workload_desc(s, 1),
+            "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": threads, "kind": "oracle",
+                             "sample": "%d random tokens of the %s workload per step (router, top-k, both "
+                                       "experts, combine in fp64)" % (min(n, s.T), s.name)},
+            "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# --------------------------------------------------------------------- GPU side
+
+def make_inputs(s, rank, device):
+    import torch
+    import synth
+    from synth.device import device_inputs, normal_tensor
+    t = device_inputs(synth.MoEShape(s.name, s.T, s.d, s.f, s.E, s.k, s.dtype, skew=s.skew), 0,
+                      device=device, with_x=False)
+    t["x"] = normal_tensor((s.T, s.d), 1000 + rank, synth.tensor_id(synth.TENSOR_X), 1.0, s.dtype, device)
+    if s.skew:
+        t["x"][:, -1] = 1.0
+    torch.cuda.synchronize()
+    return t
+
+
+def timed_loop(step, steps, flush, stream):
+    import torch
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+    for a, b in evs:
+        flush.zero_()
+        a.record(stream)
+        step()
+        b.record(stream)
+    return evs
+
+
+def bench_workload(args, s, rank, world, device, dist, extras_for_decode=False):
+    import torch
+    import sparse_mixture_experts_06_b200 as moe
+    t = make_inputs(s, rank, device)
+    stream = torch.cuda.current_stream(device)
+    y = torch.empty_like(t["x"])
+    ws = torch.empty(moe.moe_workspace_size(s.T, s.d, s.f, s.E, s.k, 0), dtype=torch.uint8, device=device)
+    flush = torch.empty(512 << 20, dtype=torch.uint8, device=device)
+
+    def step():
+        moe.moe_layer_forward_ex(t["x"], t["Wg"], t["W1"], t["W3"], t["W2"], s.k, y=y, workspace=ws, stream=stream)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize(device)
+    if dist is not None:
+        dist.barrier()
+    torch.cuda.synchronize(device)
+    moe.moe_profile_enable(True)
+    props = torch.cuda.get_device_properties(device)
+    bus = "%04x:%02x:%02x" % (getattr(props, "pci_domain_id", 0), getattr(props, "pci_bus_id", 0),
+                              getattr(props, "pci_device_id", 0)) if hasattr(props, "pci_bus_id") else ""
+    sampler = ClockSampler(bus) if rank == 0 and not extras_for_decode else None
+    if sampler:
+        sampler.start()
+        time.sleep(0.5)
+    evs = timed_loop(step, args.steps, flush, stream)
+    torch.cuda.synchronize(device)
+    if dist is not None:
+        dist.barrier()
+    torch.cuda.synchronize(device)
+    clocks = sampler.stop() if sampler else None
+    moe.moe_profile_enable(False)
+    prof = moe.moe_profile_read()
+    step_ms = [a.elapsed_time(b) for a, b in evs]
+    total_ms = sum(step_ms)
+    if dist is not None:
+        tt = torch.tensor([total_ms], dtype=torch.float64, device=device)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        total_ms = float(tt.item())
+    deverr = moe.moe_device_errors()
+    res = {"t": t, "y": y, "ws": ws, "total_ms": total_ms, "step_ms": step_ms, "prof": prof, "clocks": clocks,
+           "deverr": deverr, "stream": stream}
+    return res
+
+
+def e2e_leg(args, s, t, device, steps):
+    """Same layer through the public entry point moe_layer_forward (library
+    workspace), with the step's tokens copied in from pinned host memory and
+    the output copied back, all inside the timed region."""
+    import torch
+    import sparse_mixture_experts_06_b200 as moe
+    x_h = t["x"].cpu().pin_memory()
+    y_h = torch.empty_like(x_h).pin_memory()
+    x_d = torch.empty_like(t["x"])
+    y_d = torch.empty_like(t["x"])
+    stream = torch.cuda.current_stream(device)
+
+    def step():
+        x_d.copy_(x_h, non_blocking=True)
+        moe.moe_layer_forward(x_d, t["Wg"], t["W1"], t["W3"], t["W2"], s.k, y=y_d, stream=stream)
+        y_h.copy_(y_d, non_blocking=True)
+
+    for _ in range(3):
+        step()
+    torch.cuda.synchronize(device)
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    for _ in range(steps):
+        step()
+    b.record(stream)
+    torch.cuda.synchronize(device)
+    ms = a.elapsed_time(b) / steps
+    nbytes = x_h.numel() * x_h.element_size()
+    return ms, nbytes, y_h.numel() * y_h.element_size()
+
+
+def main():
+    args = parse()
+    if args.impl == "reference":
+        return run_reference(args)
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    import torch
+    torch.cuda.set_device(local)
+    device = torch.device("cuda", local)
+    dist = None
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=device)
+    import synth
+    s = synth.CONFIGS[args.workload]
+    pk, pk_kind = peaks()
+
+    r = bench_workload(args, s, rank, world, device, dist)
+    K = args.steps
+    total_s = r["total_ms"] * 1e-3
+    value = world * s.T * K / total_s
+    tflops = world * s.flops * K / total_s / 1e12
+
+    prof = r["prof"]
+    up_ms, up_n = prof["up_swiglu_gemm"]
+    dn_ms, dn_n = prof["down_scaled_gemm"]
+    launches = sum(n for _, n in prof.values())
+    rows = s.T * s.k
+    # dominant kernel: the up-projection GEMM (2/3 of the flops; HBM-bound at decode)
+    up_flops = 2.0 * rows * s.d * (2 * s.f)
+    up_avg_s = up_ms / max(up_n, 1) * 1e-3
+    if s.T * s.k >= 1024:
+        tr = traffic_record("up_swiglu_gemm")
+        roofline = {"kernel": "up_swiglu_gemm (tcgen05 grouped GEMM, SwiGLU epilogue)", "bound": "tensor",
+                    "achieved": up_flops / up_avg_s / 1e12, "peak": pk["bf16_tflops"], "unit": "TFLOP/s",
+                    "peak_kind": pk_kind + " bf16 (burst)",
+                    "algorithmic_per_launch": up_flops, "avg_launch_ms": up_avg_s * 1e3,
+                    "traffic": tr["bytes_per_launch"] if tr else None}
+    else:
+        up_bytes = 2.0 * s.E * s.f * s.d * 2 + rows * s.d * 2 + rows * s.f * 2
+        tr = traffic_record("up_swiglu_gemm_decode")
+        roofline = {"kernel": "up_swiglu_gemm (weight streaming)", "bound": "hbm",
+                    "achieved": up_bytes / up_avg_s / 1e9, "peak": pk["hbm_gbs"], "unit": "GB/s",
+                    "peak_kind": pk_kind, "algorithmic_per_launch": up_bytes, "avg_launch_ms": up_avg_s * 1e3,
+                    "traffic": tr["bytes_per_launch"] if tr else None}
+    roofline["frac"] = roofline["achieved"] / roofline["peak"]
+
+    line = {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": K,
+            "warmup": args.warmup, "ms_per_step": r["total_ms"] / K, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic: seeded counter-based N(0,1) tokens, N(0,1/fan_in) random-init Mixtral-8x7B expert "
+                    "and router weights",
+            "config": workload_desc(s, world),
+            "tflops": tflops, "frac_of_bf16_peak": tflops / world / pk["bf16_tflops"], "peak_kind": pk_kind,
+            "roofline": roofline, "gpu_launches": launches,
+            "stages_ms_per_step": {k: round(v[0] / K, 4) for k, v in prof.items() if v[1]},
+            "device_error_flags": r["deverr"]}
+    if r["clocks"]:
+        line["clocks"] = r["clocks"]
+
+    if rank == 0:
+        e_ms, hb, db = e2e_leg(args, s, r["t"], device, max(10, min(K, 100)))
+        line["e2e"] = {"value": world * s.T / (e_ms * 1e-3), "unit": "tokens/s", "h2d_bytes_per_step": hb,
+                       "d2h_bytes_per_step": db, "ms_per_step": e_ms,
+                       "path": "pinned host x -> moe_layer_forward (library workspace) -> pinned host y"}
+    del r
+    torch.cuda.empty_cache()
+
+    if not args.no_extras and args.workload == "prefill":
+        d = synth.CONFIGS["decode"]
+        dargs = argparse.Namespace(**vars(args))
+        dargs.steps = max(20, min(200, K))
+        rd = bench_workload(dargs, d, rank, world, device, dist, extras_for_decode=True)
+        p = rd["prof"]
+        dms = rd["total_ms"] / dargs.steps
+        counts = None
+        wbytes = 3.0 * d.E * d.d * d.f * 2  # all 8 experts are touched at T=32 with near-uniform routing
+        ups, upn = p["up_swiglu_gemm"]
+        dns, dnn = p["down_scaled_gemm"]
+        line["decode"] = {"workload": workload_desc(d, world)["workload"], "ms_per_step": dms,
+                          "tokens_per_s": world * d.T / (dms * 1e-3),
+                          "weight_GBps": wbytes / (dms * 1e-3) / 1e9,
+                          "frac_of_hbm": wbytes / (dms * 1e-3) / 1e9 / pk["hbm_gbs"],
+                          "up_gemm_GBps": (2.0 * d.E * d.f * d.d * 2) / (ups / upn * 1e-3) / 1e9,
+                          "down_gemm_GBps": (1.0 * d.E * d.f * d.d * 2) / (dns / dnn * 1e-3) / 1e9,
+                          "stages_ms_per_step": {k: round(v[0] / dargs.steps, 4) for k, v in p.items() if v[1]},
+                          "device_error_flags": rd["deverr"]}
+        del rd, counts
+        torch.cuda.empty_cache()
+
+    if rank == 0 and world == 1 and not args.no_extras:
+        import numpy as np
+        from synth.device import device_inputs, to_host_bits
+        t = make_inputs(s, 0, device)
+        w64 = oracle_weights_f64(t, s.E)
+        n = min(args.cpu_sample, s.T)
+        rows_sel = np.sort(np.random.default_rng(0).choice(s.T, size=n, replace=False))
+        x_bits = to_host_bits(t["x"])[rows_sel]
+        del t
+        dt, threads = time_oracle(w64, x_bits, s.k)
+        line["cpu_baseline"] = {"value": n / dt, "unit": "tokens/s", "cores": threads, "kind": "oracle",
+                                "sample": "%d random tokens of the %s workload (fp64 router, top-k, both experts "
+                                          "and combine; weights pre-widened to fp64 outside the timing), %.1f s"
+                                          % (n, s.name, dt)}
+    if dist is not None:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

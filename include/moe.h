@@ -1,0 +1,158 @@
+/*
+ * moe.h - C ABI of the sparse mixture-of-experts feed-forward layer for
+ * NVIDIA B200 (sm_100a).
+ *
+ * The layer ("Mixtral of Experts", §2.1, displays 1-3; Method, steps 2-4):
+ *
+ *     y[t] = sum_{j < k} w[t, j] * SwiGLU_{idx[t, j]}(x[t])
+ *     idx[t, :] = TopK(x[t] . Wg^T),  w[t, :] = softmax(kept logits)
+ *     SwiGLU_e(x) = W2_e (SiLU(W1_e x) * (W3_e x))
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ *  - Every tensor pointer is a DEVICE pointer owned by the caller.  The
+ *    library never frees or keeps them; it reads inputs and overwrites
+ *    outputs (never accumulates into them).  Outputs must not alias inputs.
+ *  - Layouts are row-major and contiguous:
+ *        x, y      [T, d]        Wg  [E, d]   (the router weight stored as
+ *        W1, W3    [E, f, d]                   (n_experts, dim), as in the
+ *        W2        [E, d, f]                   Method pseudocode)
+ *        topk_idx  [T, k] int32  topk_w [T, k] float32
+ *        offsets   [E + 1] int32 perm, inv [T * k] int32
+ *  - dtype: MOE_BF16 (bf16 tensors, fp32 accumulation, bf16 y) or MOE_F32
+ *    (fp32 everywhere, true fp32 FMA; no TF32).
+ *  - All calls are asynchronous on `stream` (a cudaStream_t; NULL = legacy
+ *    default stream): they validate arguments on the host, enqueue kernels
+ *    and return.  Nothing is copied back to the host and nothing waits, so
+ *    every call can be captured in a CUDA graph once the workspace exists.
+ *  - Return value: MOE_OK or an error code.  Invalid arguments are detected
+ *    on the host before anything is launched.  Kernel faults surface at the
+ *    caller's next synchronisation, as in CUDA; conditions the kernels
+ *    detect themselves (an expert id out of range, a pipeline wait that
+ *    timed out) set device flags read by moe_device_errors().
+ *  - Limits on the GPU path: 1 <= E <= 64, 1 <= k <= min(E, 8), T >= 0
+ *    (T = 0 is a no-op), d and f >= 8 and multiples of 8 (16-byte rows for
+ *    the tensor-memory-accelerator copies), all pointers 16-byte aligned.
+ *    Non-finite inputs give undefined outputs.
+ *  - Top-k ties go to the lower expert index; slot 0 holds the largest
+ *    logit.  Router logits are accumulated in fp64, so the chosen experts
+ *    are those of the exact logits except within ~1e-13 relative near-ties.
+ *  - Thread safety: calls on different streams may run concurrently when
+ *    each uses its own workspace (moe_layer_forward_ex); moe_layer_forward
+ *    shares one library-owned workspace per device and must not be called
+ *    concurrently on two streams of one device.
+ */
+#ifndef MOE_B200_H
+#define MOE_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st* moe_stream_t; /* identical to cudaStream_t */
+
+typedef enum { MOE_BF16 = 0, MOE_F32 = 1 } moe_dtype;
+
+enum {
+    MOE_OK = 0,
+    MOE_ERR_INVALID_ARG = 1, /* null pointer, size out of range, misalignment      */
+    MOE_ERR_UNSUPPORTED = 2, /* valid for the method but not on this GPU path (k>8) */
+    MOE_ERR_WORKSPACE = 3,   /* workspace null or smaller than moe_workspace_size   */
+    MOE_ERR_CUDA = 4         /* a CUDA call failed; see moe_last_error_string()     */
+};
+
+/* Device-side flags reported by moe_device_errors(). */
+enum {
+    MOE_DEVERR_PIPELINE_TIMEOUT = 1u, /* a GEMM pipeline wait gave up (kernel returned early)  */
+    MOE_DEVERR_BAD_EXPERT = 2u        /* moe_permute met an expert id outside [0, E)           */
+};
+
+/* Bytes of device workspace needed by moe_layer_forward_ex and moe_expert_ffn
+ * for this shape (0 for invalid arguments).  Holds the routing result, the
+ * permutation, the expert-ordered copy of x, the hidden activations h
+ * [T*k, f] and the gate-scaled expert outputs [T*k, d] (fp32). */
+size_t moe_workspace_size(int T, int d, int f, int E, int k, int dtype);
+
+/* Router and top-k gate ("Mixtral of Experts" §2.1 display 2; Method, steps
+ * 2-3; Pitfalls, renormalised top-2 weights).  For every token t:
+ * logits l[t, e] = sum_i x[t, i] * Wg[e, i] (bias-free, fp64 accumulation),
+ * topk_idx[t, :] = the k largest logits, largest first, lower index on ties;
+ * topk_w[t, :] = softmax over those k logits only, computed in fp32 and kept
+ * in fp32 (the weights sum to 1 over the chosen experts). */
+int moe_router_topk(const void* x, const void* Wg, int T, int d, int E, int k, int dtype,
+                    int32_t* topk_idx, float* topk_w, moe_stream_t stream);
+
+/* Expert-grouped order of the T*k assignments q = t*k + j (Method: the batch
+ * is processed "grouped by expert").  offsets[e] .. offsets[e+1] is expert
+ * e's block of permuted rows; perm[r] = the assignment at row r; inv[q] = the
+ * row of assignment q.  Stable: within an expert, assignment ids increase.
+ * Expert ids outside [0, E) are skipped and flagged (MOE_DEVERR_BAD_EXPERT). */
+int moe_permute(const int32_t* topk_idx, int T, int E, int k, int32_t* offsets, int32_t* perm,
+                int32_t* inv, moe_stream_t stream);
+
+/* The experts and the combine ("Mixtral of Experts" §2.1 display 3; Method,
+ * step 4; SwiGLU expert).  For every permuted row r of expert e with
+ * assignment q = perm[r] = t*k + j:  h_r = SiLU(W1_e x_t) * (W3_e x_t)
+ * (rounded to bf16 on the bf16 path), o_r = topk_w[q] * (W2_e h_r) in fp32,
+ * and y[t] = sum_j o_{inv[t*k+j]} in slot order, rounded once to y's dtype.
+ * offsets/perm/inv/topk_w are as produced by moe_permute / moe_router_topk.
+ * workspace: device memory of at least moe_workspace_size() bytes. */
+int moe_expert_ffn(const void* x, const void* W1, const void* W3, const void* W2,
+                   const int32_t* offsets, const int32_t* perm, const int32_t* inv,
+                   const float* topk_w, int T, int d, int f, int E, int k, int dtype,
+                   void* workspace, size_t ws_bytes, void* y, moe_stream_t stream);
+
+/* The whole layer in bf16: router, permutation, experts, combine.  The
+ * workspace comes from a library-owned, stream-ordered allocation per device
+ * (grown with cudaMallocAsync on `stream` when a larger shape arrives and
+ * kept until moe_release_workspace()). */
+int moe_layer_forward(const void* x, const void* Wg, const void* W1, const void* W3,
+                      const void* W2, int T, int d, int f, int E, int k, void* y,
+                      moe_stream_t stream);
+
+/* As moe_layer_forward with an explicit dtype and a caller-owned workspace.
+ * If `residual` is not NULL it must be a [T, d] tensor of the same dtype and
+ * y = residual + MoE(x), added in that order after the slot-ordered sum (the
+ * residual stream of Method, step 5).  residual may equal x. */
+int moe_layer_forward_ex(const void* x, const void* Wg, const void* W1, const void* W3,
+                         const void* W2, const void* residual, int T, int d, int f, int E,
+                         int k, int dtype, void* workspace, size_t ws_bytes, void* y,
+                         moe_stream_t stream);
+
+/* Frees the workspace moe_layer_forward keeps for the current device
+ * (stream-ordered on `stream`). */
+int moe_release_workspace(moe_stream_t stream);
+
+/* Synchronises the current device, returns the device-side flags
+ * (MOE_DEVERR_*) raised since the last call, and clears them. */
+unsigned int moe_device_errors(void);
+
+/* Per-stage device timing, for measurement: while enabled, every kernel the
+ * library launches on the current device is bracketed by a pair of CUDA
+ * events recorded on the launching stream (no synchronisation is added).
+ * Stages: 0 router_topk, 1 permute, 2 gather, 3 up-projection GEMM (SwiGLU
+ * epilogue), 4 down-projection GEMM (gate scaling), 5 combine, 6 fp32 expert
+ * kernels.  moe_profile_enable(1) clears and starts recording (up to 8192
+ * launches), moe_profile_enable(0) stops.  moe_profile_read() waits for the
+ * recorded events, writes per-stage total milliseconds and launch counts
+ * for the first n stages, clears the record, and returns the number of
+ * stages (MOE_PROFILE_STAGES) or -1 on a CUDA error. */
+#define MOE_PROFILE_STAGES 7
+int moe_profile_enable(int on);
+int moe_profile_read(double* total_ms, int* launches, int n);
+const char* moe_profile_stage_name(int stage);
+
+/* Text of the last error returned on this host thread ("" if none). */
+const char* moe_last_error_string(void);
+
+/* Library version string. */
+const char* moe_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MOE_B200_H */

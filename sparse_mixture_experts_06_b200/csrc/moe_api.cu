@@ -1,0 +1,427 @@
+// C ABI of the sparse MoE layer (declared in include/moe.h): argument
+// validation, workspace layout, and the launch sequence
+//   router_topk -> permute -> [gather] -> up GEMM -> down GEMM -> combine
+// on the caller's stream.  Nothing here waits on the device.
+
+#include <cstdarg>
+#include <cstdio>
+#include <mutex>
+#include <string>
+#include <vector>
+
+#include "../../include/moe.h"
+#include "moe_internal.cuh"
+
+namespace {
+
+thread_local std::string g_last_error;
+
+int fail(int code, const char* fmt, ...) {
+    char buf[512];
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(buf, sizeof(buf), fmt, ap);
+    va_end(ap);
+    g_last_error = buf;
+    return code;
+}
+
+int cuda_fail(cudaError_t e, const char* where) {
+    return fail(MOE_ERR_CUDA, "%s: %s", where, cudaGetErrorString(e));
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+size_t align256(size_t v) { return (v + 255) & ~size_t(255); }
+
+int num_sms_current() {
+    static int cache[64] = {0};
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (dev < 64 && cache[dev]) return cache[dev];
+    int sms = 0;
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    if (sms <= 0) sms = 148;
+    if (dev < 64) cache[dev] = sms;
+    return sms;
+}
+
+// Shape checks shared by every entry point.  `need_f` is false for calls
+// that do not involve the expert width.
+int check_shape(int T, int d, int f, int E, int k, int dtype, bool need_f) {
+    if (dtype != MOE_BF16 && dtype != MOE_F32) return fail(MOE_ERR_INVALID_ARG, "dtype %d is not MOE_BF16 or MOE_F32", dtype);
+    if (T < 0) return fail(MOE_ERR_INVALID_ARG, "T = %d < 0", T);
+    if (E < 1 || E > moe::kMaxExperts) return fail(MOE_ERR_INVALID_ARG, "E = %d outside [1, %d]", E, moe::kMaxExperts);
+    if (k < 1 || k > E) return fail(MOE_ERR_INVALID_ARG, "k = %d outside [1, E = %d]", k, E);
+    if (k > moe::kMaxTopK) return fail(MOE_ERR_UNSUPPORTED, "k = %d > %d is not supported on the GPU path", k, moe::kMaxTopK);
+    if (d < 8 || d % 8) return fail(MOE_ERR_INVALID_ARG, "d = %d must be a positive multiple of 8", d);
+    if (need_f && (f < 8 || f % 8)) return fail(MOE_ERR_INVALID_ARG, "f = %d must be a positive multiple of 8", f);
+    if ((long long)T * k > 0x7fffffffLL) return fail(MOE_ERR_INVALID_ARG, "T*k = %lld exceeds 2^31-1", (long long)T * k);
+    if ((long long)E * (need_f ? (f > d ? f : d) : d) > 0x7fffffffLL)
+        return fail(MOE_ERR_INVALID_ARG, "E * max(d, f) exceeds 2^31-1");
+    return MOE_OK;
+}
+
+int check_ptr(const void* p, const char* name) {
+    if (!p) return fail(MOE_ERR_INVALID_ARG, "%s is NULL", name);
+    if (!aligned16(p)) return fail(MOE_ERR_INVALID_ARG, "%s is not 16-byte aligned", name);
+    return MOE_OK;
+}
+
+#define CHECK(expr)                      \
+    do {                                 \
+        int _rc = (expr);                \
+        if (_rc != MOE_OK) return _rc;   \
+    } while (0)
+
+}  // namespace
+
+namespace moe {
+
+Workspace carve_workspace(void* base, int T, int d, int f, int E, int k, bool bf16) {
+    Workspace w{};
+    const size_t n = (size_t)T * k;
+    char* p = static_cast<char*>(base);
+    size_t off = 0;
+    auto take = [&](size_t bytes) {
+        char* q = p ? p + off : nullptr;
+        off += align256(bytes);
+        return q;
+    };
+    w.topk_idx = reinterpret_cast<int32_t*>(take(n * 4));
+    w.topk_w = reinterpret_cast<float*>(take(n * 4));
+    w.offsets = reinterpret_cast<int32_t*>(take((size_t)(E + 1) * 4));
+    w.perm = reinterpret_cast<int32_t*>(take(n * 4));
+    w.inv = reinterpret_cast<int32_t*>(take(n * 4));
+    w.x_perm = bf16 ? take(n * d * 2) : nullptr;
+    w.h = take(n * f * (bf16 ? 2 : 4));
+    w.obuf = reinterpret_cast<float*>(take(n * d * 4));
+    w.bytes = off;
+    return w;
+}
+
+}  // namespace moe
+
+namespace {
+
+// ---- optional per-stage event timing (moe_profile_*) --------------------
+enum Stage { kRouter = 0, kPermute, kGather, kUp, kDown, kCombine, kFfnF32, kNumStages };
+const char* const kStageNames[kNumStages] = {"router_topk", "permute", "gather_rows", "up_swiglu_gemm",
+                                             "down_scaled_gemm", "combine", "ffn_f32"};
+constexpr int kMaxProfiled = 8192;
+struct Prof {
+    std::mutex mu;
+    bool on = false;
+    int device = -1;
+    std::vector<cudaEvent_t> pool;  // 2 per launch
+    std::vector<int> stage;
+    int used = 0;
+} g_prof;
+
+// Brackets one launch with events when profiling is on.
+struct StageTimer {
+    cudaEvent_t b = nullptr;
+    int slot = -1;
+    StageTimer(int st, cudaStream_t s) {
+        std::lock_guard<std::mutex> lock(g_prof.mu);
+        int dev = -1;
+        cudaGetDevice(&dev);
+        if (!g_prof.on || dev != g_prof.device || g_prof.used >= kMaxProfiled) return;
+        slot = g_prof.used++;
+        g_prof.stage[slot] = st;
+        cudaEventRecord(g_prof.pool[2 * slot], s);
+        b = g_prof.pool[2 * slot + 1];
+    }
+    void done(cudaStream_t s) {
+        if (b) cudaEventRecord(b, s);
+    }
+};
+
+// Experts + combine on carved workspace `w` (routing fields supplied by the caller).
+int run_ffn(const void* x, const void* W1, const void* W3, const void* W2, const int32_t* offsets,
+            const int32_t* perm, const int32_t* inv, const float* topk_w, const void* residual,
+            int T, int d, int f, int E, int k, bool bf16, const moe::Workspace& w, void* y,
+            cudaStream_t s) {
+    const int rows = T * k;
+    cudaError_t e;
+    if (bf16) {
+        if (const char* msg = moe::gemm_init_error()) return fail(MOE_ERR_CUDA, "%s", msg);
+        {
+            StageTimer tm(kGather, s);
+            e = moe::launch_gather_rows_bf16(static_cast<const __nv_bfloat16*>(x), perm, rows, d, k,
+                                             static_cast<__nv_bfloat16*>(w.x_perm), s);
+            tm.done(s);
+        }
+        if (e != cudaSuccess) return cuda_fail(e, "gather_rows");
+        unsigned int* err = moe::device_error_word();
+        if (!err) return fail(MOE_ERR_CUDA, "cannot locate the device error word");
+        moe::GroupedGemmArgs a{offsets, E, rows, d, f, num_sms_current(), err};
+        {
+            StageTimer tm(kUp, s);
+            e = moe::launch_up_swiglu(a, static_cast<const __nv_bfloat16*>(w.x_perm),
+                                      static_cast<const __nv_bfloat16*>(W1), static_cast<const __nv_bfloat16*>(W3),
+                                      static_cast<__nv_bfloat16*>(w.h), s);
+            tm.done(s);
+        }
+        if (e != cudaSuccess) return cuda_fail(e, "grouped up-projection GEMM");
+        {
+            StageTimer tm(kDown, s);
+            e = moe::launch_down_scaled(a, static_cast<const __nv_bfloat16*>(w.h),
+                                        static_cast<const __nv_bfloat16*>(W2), perm, topk_w, w.obuf, s);
+            tm.done(s);
+        }
+        if (e != cudaSuccess) return cuda_fail(e, "grouped down-projection GEMM");
+    } else {
+        StageTimer tm(kFfnF32, s);
+        e = moe::launch_ffn_f32(static_cast<const float*>(x), static_cast<const float*>(W1),
+                                static_cast<const float*>(W3), static_cast<const float*>(W2), offsets, perm,
+                                topk_w, T, d, f, E, k, static_cast<float*>(w.h), w.obuf, s);
+        tm.done(s);
+        if (e != cudaSuccess) return cuda_fail(e, "fp32 expert kernels");
+    }
+    {
+        StageTimer tm(kCombine, s);
+        e = moe::launch_combine(w.obuf, inv, residual, T, d, k, bf16, y, s);
+        tm.done(s);
+    }
+    if (e != cudaSuccess) return cuda_fail(e, "combine");
+    return MOE_OK;
+}
+
+struct Pool {
+    void* ptr = nullptr;
+    size_t bytes = 0;
+};
+std::mutex g_pool_mu;
+Pool g_pool[64];
+
+}  // namespace
+
+extern "C" {
+
+size_t moe_workspace_size(int T, int d, int f, int E, int k, int dtype) {
+    if (check_shape(T, d, f, E, k, dtype, true) != MOE_OK) return 0;
+    return moe::carve_workspace(nullptr, T, d, f, E, k, dtype == MOE_BF16).bytes;
+}
+
+int moe_router_topk(const void* x, const void* Wg, int T, int d, int E, int k, int dtype,
+                    int32_t* topk_idx, float* topk_w, moe_stream_t stream) {
+    g_last_error.clear();
+    CHECK(check_shape(T, d, 8, E, k, dtype, false));
+    if (T == 0) return MOE_OK;
+    CHECK(check_ptr(x, "x"));
+    CHECK(check_ptr(Wg, "Wg"));
+    if (!topk_idx) return fail(MOE_ERR_INVALID_ARG, "topk_idx is NULL");
+    if (!topk_w) return fail(MOE_ERR_INVALID_ARG, "topk_w is NULL");
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    StageTimer tm(kRouter, s);
+    cudaError_t e = moe::launch_router_topk(x, Wg, T, d, E, k, dtype == MOE_BF16, topk_idx, topk_w, s);
+    tm.done(s);
+    return e == cudaSuccess ? MOE_OK : cuda_fail(e, "router_topk");
+}
+
+int moe_permute(const int32_t* topk_idx, int T, int E, int k, int32_t* offsets, int32_t* perm,
+                int32_t* inv, moe_stream_t stream) {
+    g_last_error.clear();
+    if (T < 0) return fail(MOE_ERR_INVALID_ARG, "T = %d < 0", T);
+    if (E < 1 || E > moe::kMaxExperts) return fail(MOE_ERR_INVALID_ARG, "E = %d outside [1, %d]", E, moe::kMaxExperts);
+    if (k < 1 || k > E) return fail(MOE_ERR_INVALID_ARG, "k = %d outside [1, E = %d]", k, E);
+    if ((long long)T * k > 0x7fffffffLL) return fail(MOE_ERR_INVALID_ARG, "T*k exceeds 2^31-1");
+    if (!offsets) return fail(MOE_ERR_INVALID_ARG, "offsets is NULL");
+    if (T > 0 && (!topk_idx || !perm || !inv)) return fail(MOE_ERR_INVALID_ARG, "topk_idx, perm and inv must not be NULL");
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    StageTimer tm(kPermute, s);
+    cudaError_t e = moe::launch_permute(topk_idx, T * k, E, offsets, perm, inv, s);
+    tm.done(s);
+    return e == cudaSuccess ? MOE_OK : cuda_fail(e, "permute");
+}
+
+int moe_expert_ffn(const void* x, const void* W1, const void* W3, const void* W2,
+                   const int32_t* offsets, const int32_t* perm, const int32_t* inv,
+                   const float* topk_w, int T, int d, int f, int E, int k, int dtype,
+                   void* workspace, size_t ws_bytes, void* y, moe_stream_t stream) {
+    g_last_error.clear();
+    CHECK(check_shape(T, d, f, E, k, dtype, true));
+    if (T == 0) return MOE_OK;
+    CHECK(check_ptr(x, "x"));
+    CHECK(check_ptr(W1, "W1"));
+    CHECK(check_ptr(W3, "W3"));
+    CHECK(check_ptr(W2, "W2"));
+    CHECK(check_ptr(y, "y"));
+    if (!offsets || !perm || !inv || !topk_w) return fail(MOE_ERR_INVALID_ARG, "routing pointers must not be NULL");
+    const bool bf16 = dtype == MOE_BF16;
+    const size_t need = moe::carve_workspace(nullptr, T, d, f, E, k, bf16).bytes;
+    if (!workspace || ws_bytes < need)
+        return fail(MOE_ERR_WORKSPACE, "workspace of %zu bytes needed, %zu given", need, workspace ? ws_bytes : 0);
+    if (!aligned16(workspace)) return fail(MOE_ERR_INVALID_ARG, "workspace is not 16-byte aligned");
+    moe::Workspace w = moe::carve_workspace(workspace, T, d, f, E, k, bf16);
+    return run_ffn(x, W1, W3, W2, offsets, perm, inv, topk_w, nullptr, T, d, f, E, k, bf16, w, y,
+                   reinterpret_cast<cudaStream_t>(stream));
+}
+
+int moe_layer_forward_ex(const void* x, const void* Wg, const void* W1, const void* W3,
+                         const void* W2, const void* residual, int T, int d, int f, int E,
+                         int k, int dtype, void* workspace, size_t ws_bytes, void* y,
+                         moe_stream_t stream) {
+    g_last_error.clear();
+    CHECK(check_shape(T, d, f, E, k, dtype, true));
+    if (T == 0) return MOE_OK;
+    CHECK(check_ptr(x, "x"));
+    CHECK(check_ptr(Wg, "Wg"));
+    CHECK(check_ptr(W1, "W1"));
+    CHECK(check_ptr(W3, "W3"));
+    CHECK(check_ptr(W2, "W2"));
+    CHECK(check_ptr(y, "y"));
+    if (residual) CHECK(check_ptr(residual, "residual"));
+    if (x == y) return fail(MOE_ERR_INVALID_ARG, "x and y must not alias");
+    const bool bf16 = dtype == MOE_BF16;
+    const size_t need = moe::carve_workspace(nullptr, T, d, f, E, k, bf16).bytes;
+    if (!workspace || ws_bytes < need)
+        return fail(MOE_ERR_WORKSPACE, "workspace of %zu bytes needed, %zu given", need, workspace ? ws_bytes : 0);
+    if (!aligned16(workspace)) return fail(MOE_ERR_INVALID_ARG, "workspace is not 16-byte aligned");
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    moe::Workspace w = moe::carve_workspace(workspace, T, d, f, E, k, bf16);
+    cudaError_t e;
+    {
+        StageTimer tm(kRouter, s);
+        e = moe::launch_router_topk(x, Wg, T, d, E, k, bf16, w.topk_idx, w.topk_w, s);
+        tm.done(s);
+    }
+    if (e != cudaSuccess) return cuda_fail(e, "router_topk");
+    {
+        StageTimer tm(kPermute, s);
+        e = moe::launch_permute(w.topk_idx, T * k, E, w.offsets, w.perm, w.inv, s);
+        tm.done(s);
+    }
+    if (e != cudaSuccess) return cuda_fail(e, "permute");
+    return run_ffn(x, W1, W3, W2, w.offsets, w.perm, w.inv, w.topk_w, residual, T, d, f, E, k, bf16, w,
+                   y, s);
+}
+
+int moe_layer_forward(const void* x, const void* Wg, const void* W1, const void* W3,
+                      const void* W2, int T, int d, int f, int E, int k, void* y,
+                      moe_stream_t stream) {
+    g_last_error.clear();
+    CHECK(check_shape(T, d, f, E, k, MOE_BF16, true));
+    if (T == 0) return MOE_OK;
+    const size_t need = moe_workspace_size(T, d, f, E, k, MOE_BF16);
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+    if (dev >= 64) return fail(MOE_ERR_UNSUPPORTED, "device ordinal %d >= 64", dev);
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    void* ws;
+    {
+        std::lock_guard<std::mutex> lock(g_pool_mu);
+        Pool& p = g_pool[dev];
+        if (p.bytes < need) {
+            if (p.ptr) {
+                e = cudaFreeAsync(p.ptr, s);
+                p.ptr = nullptr;
+                p.bytes = 0;
+                if (e != cudaSuccess) return cuda_fail(e, "cudaFreeAsync(workspace)");
+            }
+            e = cudaMallocAsync(&p.ptr, need, s);
+            if (e != cudaSuccess) {
+                p.ptr = nullptr;
+                return cuda_fail(e, "cudaMallocAsync(workspace)");
+            }
+            p.bytes = need;
+        }
+        ws = p.ptr;
+    }
+    return moe_layer_forward_ex(x, Wg, W1, W3, W2, nullptr, T, d, f, E, k, MOE_BF16, ws, need, y, stream);
+}
+
+int moe_release_workspace(moe_stream_t stream) {
+    g_last_error.clear();
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+    if (dev >= 64) return MOE_OK;
+    std::lock_guard<std::mutex> lock(g_pool_mu);
+    Pool& p = g_pool[dev];
+    if (p.ptr) {
+        e = cudaFreeAsync(p.ptr, reinterpret_cast<cudaStream_t>(stream));
+        p.ptr = nullptr;
+        p.bytes = 0;
+        if (e != cudaSuccess) return cuda_fail(e, "cudaFreeAsync(workspace)");
+    }
+    return MOE_OK;
+}
+
+unsigned int moe_device_errors(void) {
+    cudaError_t e = cudaDeviceSynchronize();
+    if (e != cudaSuccess) {
+        cuda_fail(e, "cudaDeviceSynchronize");
+        return 0x80000000u;
+    }
+    unsigned int v = 0;
+    e = moe::read_clear_device_errors(&v);
+    if (e != cudaSuccess) {
+        cuda_fail(e, "reading the device error flags");
+        return 0x80000000u;
+    }
+    return v;
+}
+
+int moe_profile_enable(int on) {
+    g_last_error.clear();
+    std::lock_guard<std::mutex> lock(g_prof.mu);
+    if (!on) {
+        g_prof.on = false;
+        return MOE_OK;
+    }
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+    if (g_prof.device != dev) {
+        for (cudaEvent_t ev : g_prof.pool) cudaEventDestroy(ev);
+        g_prof.pool.clear();
+        g_prof.device = dev;
+    }
+    while ((int)g_prof.pool.size() < 2 * kMaxProfiled) {
+        cudaEvent_t ev;
+        e = cudaEventCreate(&ev);
+        if (e != cudaSuccess) return cuda_fail(e, "cudaEventCreate");
+        g_prof.pool.push_back(ev);
+    }
+    g_prof.stage.assign(kMaxProfiled, -1);
+    g_prof.used = 0;
+    g_prof.on = true;
+    return MOE_OK;
+}
+
+int moe_profile_read(double* total_ms, int* launches, int n) {
+    g_last_error.clear();
+    std::lock_guard<std::mutex> lock(g_prof.mu);
+    double ms[kNumStages] = {0};
+    int cnt[kNumStages] = {0};
+    for (int i = 0; i < g_prof.used; ++i) {
+        cudaError_t e = cudaEventSynchronize(g_prof.pool[2 * i + 1]);
+        float t = 0.f;
+        if (e == cudaSuccess) e = cudaEventElapsedTime(&t, g_prof.pool[2 * i], g_prof.pool[2 * i + 1]);
+        if (e != cudaSuccess) {
+            cuda_fail(e, "reading profile events");
+            return -1;
+        }
+        ms[g_prof.stage[i]] += t;
+        cnt[g_prof.stage[i]] += 1;
+    }
+    g_prof.used = 0;
+    for (int i = 0; i < n && i < kNumStages; ++i) {
+        if (total_ms) total_ms[i] = ms[i];
+        if (launches) launches[i] = cnt[i];
+    }
+    return kNumStages;
+}
+
+const char* moe_profile_stage_name(int stage) {
+    return (stage >= 0 && stage < kNumStages) ? kStageNames[stage] : "";
+}
+
+const char* moe_last_error_string(void) { return g_last_error.c_str(); }
+
+const char* moe_version(void) { return "moe-b200 0.1.0 (sm_100a)"; }
+
+}  // extern "C"

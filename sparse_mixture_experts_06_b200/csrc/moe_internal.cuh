@@ -1,0 +1,65 @@
+// Internal interface between the kernels and the C ABI layer (moe_api.cu).
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace moe {
+
+// Device-side error flags (MOE_DEVERR_* in moe.h): one word per device,
+// defined in permute.cu.  Kernels in other files receive its device address.
+unsigned int* device_error_word();                 // nullptr if the lookup fails
+cudaError_t read_clear_device_errors(unsigned int* out);
+
+constexpr int kMaxExperts = 64;
+constexpr int kMaxTopK = 8;
+
+// 256-byte aligned carve-up of one workspace blob.
+struct Workspace {
+    int32_t* topk_idx;  // [T*k]
+    float* topk_w;      // [T*k]
+    int32_t* offsets;   // [E+1]
+    int32_t* perm;      // [T*k]
+    int32_t* inv;       // [T*k]
+    void* x_perm;       // [T*k, d]  bf16 path only
+    void* h;            // [T*k, f]  bf16 or f32
+    float* obuf;        // [T*k, d]  gate-scaled expert outputs, fp32
+    size_t bytes;
+};
+
+Workspace carve_workspace(void* base, int T, int d, int f, int E, int k, bool bf16);
+
+// ---- launchers (return cudaError_t of the launch) ------------------------
+cudaError_t launch_router_topk(const void* x, const void* Wg, int T, int d, int E, int k,
+                               bool bf16, int32_t* idx, float* w, cudaStream_t s);
+cudaError_t launch_permute(const int32_t* idx, int n, int E, int32_t* offsets, int32_t* perm,
+                           int32_t* inv, cudaStream_t s);
+cudaError_t launch_gather_rows_bf16(const __nv_bfloat16* x, const int32_t* perm, int rows, int d,
+                                    int k, __nv_bfloat16* x_perm, cudaStream_t s);
+cudaError_t launch_combine(const float* obuf, const int32_t* inv, const void* residual, int T,
+                           int d, int k, bool bf16, void* y, cudaStream_t s);
+
+// tcgen05 grouped GEMMs (gemm_sm100.cu)
+struct GroupedGemmArgs {
+    const int32_t* offsets;  // [E+1] permuted-row blocks per expert
+    int E, rows;             // rows = T*k (permuted rows)
+    int d, f;
+    int num_sms;
+    unsigned int* err;       // device error word
+};
+cudaError_t launch_up_swiglu(const GroupedGemmArgs& a, const __nv_bfloat16* x_perm,
+                             const __nv_bfloat16* W1, const __nv_bfloat16* W3, __nv_bfloat16* h,
+                             cudaStream_t s);
+cudaError_t launch_down_scaled(const GroupedGemmArgs& a, const __nv_bfloat16* h,
+                               const __nv_bfloat16* W2, const int32_t* perm, const float* topk_w,
+                               float* obuf, cudaStream_t s);
+const char* gemm_init_error();  // non-null if the driver entry point is missing
+
+// fp32 SIMT expert path (ffn_f32.cu)
+cudaError_t launch_ffn_f32(const float* x, const float* W1, const float* W3, const float* W2,
+                           const int32_t* offsets, const int32_t* perm, const float* topk_w,
+                           int T, int d, int f, int E, int k, float* h, float* obuf,
+                           cudaStream_t s);
+
+}  // namespace moe

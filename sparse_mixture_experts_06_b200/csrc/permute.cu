@@ -1,0 +1,210 @@
+// Token permutation to expert-contiguous order and back (Method: the batch is
+// processed "grouped by expert"; Pitfalls: results are scattered back to the
+// tokens).
+//
+//  permute_kernel   histogram -> exclusive scan -> stable scatter, one block
+//  gather_rows      x_perm[r] = x[perm[r] / k]            (bf16 path)
+//  combine_kernel   y[t] = (residual[t] +) sum_j obuf[inv[t*k + j]]
+//
+// The scatter is stable and deterministic without global atomics: the
+// assignments are walked in tiles of 1024 in increasing id; inside a warp,
+// __match_any_sync groups lanes with the same expert and a lane's rank is
+// the number of lower lanes in its group; a per-tile exclusive scan over the
+// 32 warps gives each warp's base inside the expert's block.
+
+#include "moe_internal.cuh"
+
+namespace moe {
+
+namespace {
+
+__device__ unsigned int g_dev_err = 0;
+
+constexpr int kPermThreads = 1024;
+
+__global__ void __launch_bounds__(kPermThreads)
+permute_kernel(const int32_t* __restrict__ idx, int n, int E, int32_t* __restrict__ offsets,
+               int32_t* __restrict__ perm, int32_t* __restrict__ inv) {
+    __shared__ int s_cnt[kMaxExperts];
+    __shared__ int s_base[kMaxExperts];
+    __shared__ int s_tile[kMaxExperts];
+    __shared__ int s_warp[32][kMaxExperts];
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+
+    for (int i = tid; i < E; i += kPermThreads) s_cnt[i] = 0;
+    __syncthreads();
+    for (int q = tid; q < n; q += kPermThreads) {
+        const int e = idx[q];
+        if ((unsigned)e < (unsigned)E) atomicAdd(&s_cnt[e], 1);
+        else atomicOr(&g_dev_err, 2u);
+    }
+    __syncthreads();
+    if (tid == 0) {
+        int run = 0;
+        for (int e = 0; e < E; ++e) {
+            offsets[e] = run;
+            s_base[e] = run;
+            run += s_cnt[e];
+        }
+        offsets[E] = run;
+    }
+    __syncthreads();
+
+    const unsigned lt_mask = (1u << lane) - 1u;
+    int e_next = (tid < n) ? idx[tid] : -1;
+    for (int t0 = 0; t0 < n; t0 += kPermThreads) {
+        const int q = t0 + tid;
+        const int e = e_next;
+        // prefetch the next tile's expert id while this tile is ranked
+        e_next = (q + kPermThreads < n) ? idx[q + kPermThreads] : -1;
+        const bool valid = q < n && (unsigned)e < (unsigned)E;
+        const unsigned peers = __match_any_sync(0xffffffffu, valid ? e : -1);
+        const int rank = __popc(peers & lt_mask);
+        for (int i = tid; i < 32 * kMaxExperts; i += kPermThreads) (&s_warp[0][0])[i] = 0;
+        __syncthreads();
+        if (valid && rank == 0) s_warp[warp][e] = __popc(peers);
+        __syncthreads();
+        if (tid < E) {
+            int run = 0;
+            for (int w = 0; w < 32; ++w) {
+                const int c = s_warp[w][tid];
+                s_warp[w][tid] = run;
+                run += c;
+            }
+            s_tile[tid] = run;
+        }
+        __syncthreads();
+        if (q < n) {
+            if (valid) {
+                const int pos = s_base[e] + s_warp[warp][e] + rank;
+                perm[pos] = q;
+                inv[q] = pos;
+            } else {
+                inv[q] = -1;
+            }
+        }
+        __syncthreads();
+        if (tid < E) s_base[tid] += s_tile[tid];
+        __syncthreads();
+    }
+}
+
+constexpr int kRowWarps = 8;
+
+__global__ void __launch_bounds__(kRowWarps * 32)
+gather_rows_kernel(const __nv_bfloat16* __restrict__ x, const int32_t* __restrict__ perm, int rows,
+                   int d, int k, __nv_bfloat16* __restrict__ xp) {
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int nvec = d / 8;
+    for (int r = blockIdx.x * kRowWarps + warp; r < rows; r += gridDim.x * kRowWarps) {
+        const int q = perm[r];
+        uint4* dst = reinterpret_cast<uint4*>(xp + (size_t)r * d);
+        if ((unsigned)q >= (unsigned)rows) {  // not a valid assignment id: zero row
+            for (int v = lane; v < nvec; v += 32) dst[v] = make_uint4(0, 0, 0, 0);
+            continue;
+        }
+        const uint4* src = reinterpret_cast<const uint4*>(x + (size_t)(q / k) * d);
+        for (int v = lane; v < nvec; v += 32) dst[v] = __ldg(src + v);
+    }
+}
+
+template <bool BF16>
+__global__ void __launch_bounds__(kRowWarps * 32)
+combine_kernel(const float* __restrict__ obuf, const int32_t* __restrict__ inv,
+               const void* __restrict__ residual, int T, int d, int k, void* __restrict__ y) {
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int nvec = d / 4;
+    for (int t = blockIdx.x * kRowWarps + warp; t < T; t += gridDim.x * kRowWarps) {
+        int rows[kMaxTopK];
+#pragma unroll
+        for (int j = 0; j < kMaxTopK; ++j) {
+            rows[j] = (j < k) ? inv[(size_t)t * k + j] : -1;
+            if ((unsigned)rows[j] >= (unsigned)(T * k)) rows[j] = -1;  // unrouted slot adds nothing
+        }
+        for (int v = lane; v < nvec; v += 32) {
+            float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+            if (rows[0] >= 0) acc = __ldg(reinterpret_cast<const float4*>(obuf + (size_t)rows[0] * d) + v);
+#pragma unroll
+            for (int j = 1; j < kMaxTopK; ++j) {
+                if (rows[j] >= 0) {
+                    const float4 o = __ldg(reinterpret_cast<const float4*>(obuf + (size_t)rows[j] * d) + v);
+                    acc.x += o.x; acc.y += o.y; acc.z += o.z; acc.w += o.w;
+                }
+            }
+            if constexpr (BF16) {
+                if (residual) {
+                    const uint2 rq = __ldg(reinterpret_cast<const uint2*>(
+                        reinterpret_cast<const __nv_bfloat16*>(residual) + (size_t)t * d) + v);
+                    acc.x = __uint_as_float(rq.x << 16) + acc.x;
+                    acc.y = __uint_as_float(rq.x & 0xFFFF0000u) + acc.y;
+                    acc.z = __uint_as_float(rq.y << 16) + acc.z;
+                    acc.w = __uint_as_float(rq.y & 0xFFFF0000u) + acc.w;
+                }
+                __nv_bfloat162 lo = __floats2bfloat162_rn(acc.x, acc.y);
+                __nv_bfloat162 hi = __floats2bfloat162_rn(acc.z, acc.w);
+                uint2 out;
+                out.x = *reinterpret_cast<uint32_t*>(&lo);
+                out.y = *reinterpret_cast<uint32_t*>(&hi);
+                reinterpret_cast<uint2*>(reinterpret_cast<__nv_bfloat16*>(y) + (size_t)t * d)[v] = out;
+            } else {
+                if (residual) {
+                    const float4 r = __ldg(reinterpret_cast<const float4*>(
+                        reinterpret_cast<const float*>(residual) + (size_t)t * d) + v);
+                    acc.x = r.x + acc.x; acc.y = r.y + acc.y; acc.z = r.z + acc.z; acc.w = r.w + acc.w;
+                }
+                reinterpret_cast<float4*>(reinterpret_cast<float*>(y) + (size_t)t * d)[v] = acc;
+            }
+        }
+    }
+}
+
+int row_grid(int rows) {
+    int dev = 0, sms = 148;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    const int need = (rows + kRowWarps - 1) / kRowWarps;
+    return need < sms * 8 ? need : sms * 8;
+}
+
+}  // namespace
+
+unsigned int* device_error_word() {
+    static unsigned int* cache[64] = {nullptr};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return nullptr;
+    if (dev < 64 && cache[dev]) return cache[dev];
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_dev_err) != cudaSuccess) return nullptr;
+    if (dev < 64) cache[dev] = static_cast<unsigned int*>(p);
+    return static_cast<unsigned int*>(p);
+}
+
+cudaError_t read_clear_device_errors(unsigned int* out) {
+    unsigned int zero = 0;
+    cudaError_t e = cudaMemcpyFromSymbol(out, g_dev_err, sizeof(unsigned int));
+    if (e == cudaSuccess) e = cudaMemcpyToSymbol(g_dev_err, &zero, sizeof(zero));
+    return e;
+}
+
+cudaError_t launch_permute(const int32_t* idx, int n, int E, int32_t* offsets, int32_t* perm,
+                           int32_t* inv, cudaStream_t s) {
+    permute_kernel<<<1, kPermThreads, 0, s>>>(idx, n, E, offsets, perm, inv);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_gather_rows_bf16(const __nv_bfloat16* x, const int32_t* perm, int rows, int d,
+                                    int k, __nv_bfloat16* x_perm, cudaStream_t s) {
+    gather_rows_kernel<<<row_grid(rows), kRowWarps * 32, 0, s>>>(x, perm, rows, d, k, x_perm);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_combine(const float* obuf, const int32_t* inv, const void* residual, int T,
+                           int d, int k, bool bf16, void* y, cudaStream_t s) {
+    if (bf16)
+        combine_kernel<true><<<row_grid(T), kRowWarps * 32, 0, s>>>(obuf, inv, residual, T, d, k, y);
+    else
+        combine_kernel<false><<<row_grid(T), kRowWarps * 32, 0, s>>>(obuf, inv, residual, T, d, k, y);
+    return cudaGetLastError();
+}
+
+}  // namespace moe

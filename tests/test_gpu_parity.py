@@ -1,0 +1,281 @@
+"""Parity of the CUDA path (through the C ABI) with the fp64 oracle.
+
+Indices and the permutation must match bit for bit; gate weights to 1e-6;
+outputs within max|y - y_ref| <= 1e-2 max|y_ref| (bf16) or 1e-5 (fp32).
+Small shapes are checked on every token and span several 128-row tiles
+with ragged tails; the full Mixtral shapes (decode T = 32, prefill
+T = 4096, skewed T = 16384) are checked on every token's routing and on a
+stratified sample of tokens for the outputs, in the launch configuration
+the benchmark times."""
+
+import numpy as np
+import pytest
+
+import synth
+from tests.gpu_util import (assert_close, check_permutation, check_routing, device_inputs, f64,
+                            host_copy, oracle_rows, stratified_tokens)
+
+pytestmark = pytest.mark.gpu
+
+torch = pytest.importorskip("torch")
+if not torch.cuda.is_available():
+    pytest.skip("no CUDA device", allow_module_level=True)
+
+import sparse_mixture_experts_06_b200 as moe  # noqa: E402
+
+
+@pytest.fixture(autouse=True)
+def no_device_errors():
+    yield
+    assert moe.moe_device_errors() == 0
+
+
+def run_layer(t, k, residual=None):
+    return moe.moe_layer_forward_ex(t["x"], t["Wg"], t["W1"], t["W3"], t["W2"], k, residual=residual)
+
+
+def to64(y):
+    return y.float().double().cpu().numpy()
+
+
+def full_check(shape: synth.MoEShape, seed: int = 0):
+    """Every token: routing, permutation and outputs against the oracle."""
+    t = device_inputs(shape, seed)
+    y = run_layer(t, shape.k)
+    idx_g, w_g = moe.moe_router_topk(t["x"], t["Wg"], shape.k)
+    off_g, perm_g, inv_g = moe.moe_permute(idx_g, shape.E)
+    torch.cuda.synchronize()
+    h = host_copy(t)
+    idx_o, _, _ = check_routing(idx_g.cpu().numpy(), w_g.cpu().numpy(), f64(h["x"]), f64(h["Wg"]), shape.k)
+    check_permutation(off_g.cpu().numpy(), perm_g.cpu().numpy(), inv_g.cpu().numpy(), idx_o, shape.E)
+    y_ref, _, _ = oracle_rows(h, shape.k, np.arange(shape.T))
+    return assert_close(to64(y), y_ref, shape.dtype), idx_o
+
+
+# ---------------------------------------------------------------- generator
+
+@pytest.mark.parametrize("dt", ["bf16", "f32"])
+def test_device_generator_matches_host(dt):
+    from synth.device import normal_tensor, to_host_bits
+    start, n = 987654321, 1 << 20
+    dev = to_host_bits(normal_tensor((n,), 5, 11, 0.0125, dt, start=start))
+    host = synth.normal_values(5, 11, n, 0.0125, dt, start=start)
+    np.testing.assert_array_equal(dev, host)
+
+
+# ---------------------------------------------------------------- router
+
+@pytest.mark.parametrize("T,d,E,k,dt", [
+    (16, 64, 8, 2, "f32"), (37, 72, 8, 2, "bf16"), (1, 8, 1, 1, "bf16"), (300, 256, 64, 8, "bf16"),
+    (129, 4096, 8, 2, "bf16"), (250, 96, 5, 3, "f32"),
+])
+def test_router_parity(T, d, E, k, dt):
+    t = device_inputs(synth.MoEShape("r", T, d, 8, E, k, dt), seed=T + E)
+    idx, w = moe.moe_router_topk(t["x"], t["Wg"], k)
+    h = host_copy({"x": t["x"], "Wg": t["Wg"]})
+    _, _, near = check_routing(idx.cpu().numpy(), w.cpu().numpy(), f64(h["x"]), f64(h["Wg"]), k)
+    assert near == 0
+
+
+def test_router_ties_go_to_lower_index():
+    x = torch.zeros((4, 64), dtype=torch.bfloat16, device="cuda")
+    Wg = torch.randn((8, 64), device="cuda").to(torch.bfloat16)
+    idx, w = moe.moe_router_topk(x, Wg, 2)
+    assert idx.cpu().tolist() == [[0, 1]] * 4
+    assert (w.cpu() == 0.5).all()
+    x = torch.ones((2, 64), dtype=torch.bfloat16, device="cuda")
+    Wg = torch.zeros((8, 64), dtype=torch.bfloat16, device="cuda")
+    Wg[6] = 0.25
+    Wg[2] = 0.25
+    idx, w = moe.moe_router_topk(x, Wg, 2)
+    assert idx.cpu().tolist() == [[2, 6]] * 2
+    assert (w.cpu() == 0.5).all()
+
+
+# ---------------------------------------------------------------- permutation
+
+@pytest.mark.parametrize("T,E,k", [(1, 8, 2), (511, 8, 2), (512, 8, 2), (1500, 8, 2), (3000, 64, 8),
+                                   (777, 3, 1), (20000, 8, 2)])
+def test_permute_parity(T, E, k):
+    rng = np.random.default_rng(T)
+    # a skewed draw that leaves some experts empty
+    p = rng.dirichlet(np.ones(E) * 0.3)
+    idx = np.stack([rng.choice(E, size=k, replace=False, p=p) for _ in range(T)]).astype(np.int32)
+    off, perm, inv = moe.moe_permute(torch.from_numpy(idx).cuda(), E)
+    check_permutation(off.cpu().numpy(), perm.cpu().numpy(), inv.cpu().numpy(), idx, E)
+
+
+def test_permute_flags_bad_expert_ids():
+    idx = torch.tensor([[0, 1], [9, 2]], dtype=torch.int32, device="cuda")
+    off, perm, inv = moe.moe_permute(idx, 8)
+    assert moe.moe_device_errors() == 2
+    assert off.cpu().tolist()[-1] == 3 and inv.cpu().tolist()[2] == -1
+
+
+# ---------------------------------------------------------------- whole layer, every token
+
+@pytest.mark.parametrize("shape", [
+    synth.CONFIGS["tiny"],
+    synth.MoEShape("f32-ragged", 37, 72, 136, 8, 2, "f32"),
+    synth.MoEShape("f32-mid", 200, 256, 512, 8, 2, "f32"),
+    synth.MoEShape("bf16-tiles", 1000, 128, 384, 4, 2, "bf16"),     # 500 rows/expert: 3 full tiles + tail
+    synth.MoEShape("bf16-ragged", 37, 72, 136, 8, 2, "bf16"),       # every tile ragged, K tails
+    synth.MoEShape("bf16-wide", 700, 512, 1024, 8, 2, "bf16"),
+    synth.MoEShape("bf16-k1", 300, 256, 256, 8, 1, "bf16"),
+    synth.MoEShape("bf16-E64k8", 256, 128, 128, 64, 8, "bf16"),
+    synth.MoEShape("bf16-T1", 1, 64, 128, 8, 2, "bf16"),
+], ids=lambda s: s.name)
+def test_layer_parity_every_token(shape):
+    rel, _ = full_check(shape)
+    assert rel <= {"f32": 1e-5, "bf16": 1e-2}[shape.dtype]
+
+
+@pytest.mark.parametrize("seed", range(1, 21))
+def test_tiny_fp32_many_seeds(seed):
+    full_check(synth.CONFIGS["tiny"], seed)
+
+
+def test_dense_special_case_E1_k1():
+    """E = 1, k = 1: the layer is one dense SwiGLU FFN."""
+    full_check(synth.MoEShape("dense", 64, 128, 256, 1, 1, "bf16"))
+    full_check(synth.MoEShape("dense32", 64, 128, 256, 1, 1, "f32"))
+
+
+def test_identical_experts_give_single_expert_output():
+    s = synth.MoEShape("ident", 300, 128, 256, 8, 2, "bf16")
+    t = device_inputs(s, 3)
+    for name in ("W1", "W3", "W2"):
+        t[name][:] = t[name][0:1].clone()
+    y = run_layer(t, 2)
+    h = host_copy(t)
+    import oracle
+    ref = oracle.swiglu_expert(f64(h["x"]), f64(h["W1"][0]), f64(h["W3"][0]), f64(h["W2"][0]))
+    assert_close(to64(y), ref, "bf16")
+
+
+def test_empty_experts():
+    """A router that only ever picks experts 5 and 2 leaves six experts empty."""
+    s = synth.MoEShape("empty", 400, 128, 256, 8, 2, "bf16")
+    t = device_inputs(s, 4)
+    t["x"][:, -1] = 4.0
+    t["Wg"][:, -1] = 0.0
+    t["Wg"][5, -1] = 8.0
+    t["Wg"][2, -1] = 6.0
+    y = run_layer(t, 2)
+    idx, _ = moe.moe_router_topk(t["x"], t["Wg"], 2)
+    assert set(np.unique(idx.cpu().numpy()).tolist()) == {2, 5}
+    h = host_copy(t)
+    y_ref, _, _ = oracle_rows(h, 2, np.arange(s.T))
+    assert_close(to64(y), y_ref, "bf16")
+
+
+def test_worked_example_through_the_gpu():
+    """The hand-worked closed-form instance (tests/golden/worked_example.json),
+    zero-padded to d = f = 8 (padding adds exact zeros)."""
+    import json
+    import math
+    import os
+    ex = json.load(open(os.path.join(os.path.dirname(__file__), "golden", "worked_example.json")))
+    sig = lambda z: 1.0 / (1.0 + math.exp(-z))  # noqa: E731
+    y_ref = [eval(s, {"sigma": sig}) for s in ex["y_closed_form"]]
+    for dt, torch_dt, tol in (("f32", torch.float32, 1e-6), ("bf16", torch.bfloat16, 1e-2)):
+        x = torch.zeros((1, 8)); x[0, :2] = torch.tensor(ex["x"])
+        Wg = torch.zeros((3, 8)); Wg[:, :2] = torch.tensor(ex["Wg"])
+        W1 = torch.zeros((3, 8, 8)); W1[:, :1, :2] = torch.tensor(ex["W1"])
+        W3 = torch.zeros((3, 8, 8)); W3[:, :1, :2] = torch.tensor(ex["W3"])
+        W2 = torch.zeros((3, 8, 8)); W2[:, :2, :1] = torch.tensor(ex["W2"])
+        args = [a.to(torch_dt).cuda() for a in (x, Wg, W1, W3, W2)]
+        y = moe.moe_layer_forward_ex(*args, 2)
+        idx, _ = moe.moe_router_topk(args[0], args[1], 2)
+        assert idx.cpu().tolist() == [ex["idx"]]
+        got = y.float().cpu().numpy()[0]
+        np.testing.assert_allclose(got[:2], y_ref, rtol=tol, atol=0)
+        assert (got[2:] == 0).all()
+
+
+def test_residual_add():
+    s = synth.MoEShape("res", 300, 256, 512, 8, 2, "bf16")
+    t = device_inputs(s, 6)
+    y = run_layer(t, 2, residual=t["x"])
+    h = host_copy(t)
+    y_ref, _, _ = oracle_rows(h, 2, np.arange(s.T))
+    assert_close(to64(y), f64(h["x"]) + y_ref, "bf16")
+    s32 = synth.MoEShape("res32", 40, 64, 128, 8, 2, "f32")
+    t = device_inputs(s32, 6)
+    y = run_layer(t, 2, residual=t["x"])
+    h = host_copy(t)
+    y_ref, _, _ = oracle_rows(h, 2, np.arange(s32.T))
+    assert_close(to64(y), f64(h["x"]) + y_ref, "f32")
+
+
+def test_entry_points_agree_and_are_deterministic():
+    """moe_layer_forward (library workspace), moe_layer_forward_ex and the
+    three-call path router -> permute -> expert_ffn give identical bits, run
+    after run."""
+    s = synth.MoEShape("api", 900, 256, 512, 8, 2, "bf16")
+    t = device_inputs(s, 7)
+    a = moe.moe_layer_forward(t["x"], t["Wg"], t["W1"], t["W3"], t["W2"], 2)
+    b = run_layer(t, 2)
+    idx, w = moe.moe_router_topk(t["x"], t["Wg"], 2)
+    off, perm, inv = moe.moe_permute(idx, 8)
+    c = moe.moe_expert_ffn(t["x"], t["W1"], t["W3"], t["W2"], off, perm, inv, w)
+    d_ = moe.moe_layer_forward(t["x"], t["Wg"], t["W1"], t["W3"], t["W2"], 2)
+    for o in (b, c, d_):
+        assert torch.equal(a.view(torch.int16), o.view(torch.int16))
+    moe.moe_release_workspace()
+
+
+def test_zero_tokens_is_a_no_op():
+    s = synth.MoEShape("z", 4, 64, 128, 8, 2, "bf16")
+    t = device_inputs(s, 8)
+    y = torch.full((0, 64), 7.0, dtype=torch.bfloat16, device="cuda")
+    out = moe.moe_layer_forward_ex(t["x"][:0], t["Wg"], t["W1"], t["W3"], t["W2"], 2, y=y)
+    assert out.shape == (0, 64)
+
+
+# ---------------------------------------------------------------- full Mixtral shapes
+
+@pytest.fixture(scope="module")
+def mixtral_weights():
+    """Layer-0 expert weights of seed 0 (shared by the decode, prefill and
+    skewed workloads), on the device and as host bf16 bits."""
+    s = synth.CONFIGS["prefill"]
+    t = device_inputs(s, 0, with_x=False)
+    return t, host_copy({k: t[k] for k in ("W1", "W3", "W2")})
+
+
+def big_check(name, mixtral_weights, sample):
+    s = synth.CONFIGS[name]
+    tw, hw = mixtral_weights
+    t = device_inputs(synth.MoEShape(s.name, s.T, s.d, 8, s.E, s.k, s.dtype, skew=s.skew), 0)
+    t = {"x": t["x"], "Wg": t["Wg"], "W1": tw["W1"], "W3": tw["W3"], "W2": tw["W2"]}
+    y = run_layer(t, s.k)
+    idx_g, w_g = moe.moe_router_topk(t["x"], t["Wg"], s.k)
+    off_g, perm_g, inv_g = moe.moe_permute(idx_g, s.E)
+    torch.cuda.synchronize()
+    h = dict(hw, x=to_bits(t["x"]), Wg=to_bits(t["Wg"]))
+    idx_o, _, _ = check_routing(idx_g.cpu().numpy(), w_g.cpu().numpy(), f64(h["x"]), f64(h["Wg"]), s.k)
+    off, perm, _ = check_permutation(off_g.cpu().numpy(), perm_g.cpu().numpy(), inv_g.cpu().numpy(), idx_o, s.E)
+    toks = np.arange(s.T) if sample is None else stratified_tokens(off, perm, s.k, sample)
+    y_ref, _, _ = oracle_rows(h, s.k, toks)
+    rel = assert_close(to64(y)[toks], y_ref, "bf16")
+    return rel, np.diff(off)
+
+
+def to_bits(t):
+    from synth.device import to_host_bits
+    return to_host_bits(t)
+
+
+def test_decode_full_shape_every_token(mixtral_weights):
+    big_check("decode", mixtral_weights, None)
+
+
+def test_prefill_full_shape(mixtral_weights):
+    big_check("prefill", mixtral_weights, 256)
+
+
+def test_skewed_full_shape(mixtral_weights):
+    _, counts = big_check("skewed", mixtral_weights, 256)
+    share = counts / counts.sum()
+    assert abs(share[0] - 0.35) < 0.005 and (np.diff(share) < 0).all()
