@@ -122,6 +122,24 @@ int moe_layer_forward_ex(const void* x, const void* Wg, const void* W1, const vo
                          int k, int dtype, void* workspace, size_t ws_bytes, void* y,
                          moe_stream_t stream);
 
+/* The whole bf16 layer, like moe_layer_forward, for callers that cannot
+ * allocate device memory while they run: a plug-in inside a host framework
+ * whose allocator owns the device memory, or a server that reserves its
+ * memory at start-up and allows no allocation on the serving path.  No
+ * counterpart in the paper: it is a deployment convenience of this library.
+ * Instead of allocating, it uses a 32 MiB scratch array compiled into the
+ * library (kept by every GPU that loads it until the process exits), which
+ * covers T*k*(2d + 2f + 4d) bytes plus routing buffers: up to 316 tokens at
+ * the Mixtral-8x7B dimensions.  Larger shapes return MOE_ERR_WORKSPACE with a
+ * message naming the bytes needed.  The first call on each device looks up
+ * the array's device address (cudaGetSymbolAddress) with that device
+ * current; make that first call before any stream capture.  All calls on a
+ * device share the array, so calls that overlap on the GPU race: serialise
+ * them.  The caller passes inputs and outputs as for moe_layer_forward. */
+int moe_layer_forward_noalloc(const void* x, const void* Wg, const void* W1, const void* W3,
+                              const void* W2, int T, int d, int f, int E, int k, void* y,
+                              moe_stream_t stream);
+
 /* Frees the workspace moe_layer_forward keeps for the current device
  * (stream-ordered on `stream`). */
 int moe_release_workspace(moe_stream_t stream);

@@ -26,6 +26,7 @@ _SIGS = {
     "moe_expert_ffn": ([_P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _P, _Z, _P, _P], _I),
     "moe_layer_forward": ([_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _P, _P], _I),
     "moe_layer_forward_ex": ([_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _P, _Z, _P, _P], _I),
+    "moe_layer_forward_noalloc": ([_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _P, _P], _I),
     "moe_release_workspace": ([_P], _I),
     "moe_device_errors": ([], ctypes.c_uint),
     "moe_profile_enable": ([_I], _I),
@@ -177,6 +178,18 @@ def moe_layer_forward(x, Wg, W1, W3, W2, k, y=None, stream=None):
     y = torch.empty_like(x) if y is None else y
     _check(lib.moe_layer_forward(_ptr(x), _ptr(Wg), _ptr(W1), _ptr(W3), _ptr(W2), T, d, f, E, k, _ptr(y),
                                  _stream(stream, x)), "moe_layer_forward")
+    return y
+
+
+def moe_layer_forward_noalloc(x, Wg, W1, W3, W2, k, y, stream=None):
+    """The whole bf16 layer using the library's static scratch instead of any
+    allocation (for callers that cannot allocate device memory while they
+    run).  `y` must be given: this wrapper allocates nothing either."""
+    _dev(x, Wg, W1, W3, W2, y)
+    T, d = x.shape
+    E, f, _ = W1.shape
+    _check(lib.moe_layer_forward_noalloc(_ptr(x), _ptr(Wg), _ptr(W1), _ptr(W3), _ptr(W2), T, d, f, E, k, _ptr(y),
+                                         _stream(stream, x)), "moe_layer_forward_noalloc")
     return y
 
 

@@ -78,6 +78,8 @@ int check_ptr(const void* p, const char* name) {
 
 namespace moe {
 
+void set_last_error(const char* msg) { g_last_error = msg ? msg : ""; }
+
 Workspace carve_workspace(void* base, int T, int d, int f, int E, int k, bool bf16) {
     Workspace w{};
     const size_t n = (size_t)T * k;

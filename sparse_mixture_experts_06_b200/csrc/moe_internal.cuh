@@ -12,6 +12,9 @@ namespace moe {
 unsigned int* device_error_word();                 // nullptr if the lookup fails
 cudaError_t read_clear_device_errors(unsigned int* out);
 
+// Sets the text moe_last_error_string() returns on this host thread.
+void set_last_error(const char* msg);
+
 constexpr int kMaxExperts = 64;
 constexpr int kMaxTopK = 8;
 
