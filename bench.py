@@ -136,6 +136,31 @@ def traffic_record(kernel):
     return d
 
 
+# --------------------------------------------------------------------- replicas (N > 1)
+
+def replica_x_seed(rank: int) -> int:
+    """Seed of rank `rank`'s tokens: every replica holds the same weights
+    (seed 0) and its own T tokens."""
+    return 1000 + rank
+
+
+def max_over_ranks(ms: float, dist, device) -> float:
+    """The job's elapsed time: the max of the ranks' device-timed totals.
+    A side reduction of one scalar, outside the timed region; the layer
+    itself exchanges nothing between ranks."""
+    if dist is None:
+        return ms
+    import torch
+    tt = torch.tensor([ms], dtype=torch.float64, device=device)
+    dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+    return float(tt.item())
+
+
+def job_tokens_per_s(world: int, T: int, steps: int, total_ms: float) -> float:
+    """Whole-job throughput: tokens processed by all ranks / the max elapsed."""
+    return world * T * steps / (total_ms * 1e-3)
+
+
 # --------------------------------------------------------------------- oracle (CPU) side
 
 def oracle_weights_f64(t, E):
@@ -209,7 +234,7 @@ def make_inputs(s, rank, device):
     from synth.device import device_inputs, normal_tensor
     t = device_inputs(synth.MoEShape(s.name, s.T, s.d, s.f, s.E, s.k, s.dtype, skew=s.skew), 0,
                       device=device, with_x=False)
-    t["x"] = normal_tensor((s.T, s.d), 1000 + rank, synth.tensor_id(synth.TENSOR_X), 1.0, s.dtype, device)
+    t["x"] = normal_tensor((s.T, s.d), replica_x_seed(rank), synth.tensor_id(synth.TENSOR_X), 1.0, s.dtype, device)
     if s.skew:
         t["x"][:, -1] = 1.0
     torch.cuda.synchronize()
@@ -262,11 +287,7 @@ def bench_workload(args, s, rank, world, device, dist, extras_for_decode=False):
     moe.moe_profile_enable(False)
     prof = moe.moe_profile_read()
     step_ms = [a.elapsed_time(b) for a, b in evs]
-    total_ms = sum(step_ms)
-    if dist is not None:
-        tt = torch.tensor([total_ms], dtype=torch.float64, device=device)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        total_ms = float(tt.item())
+    total_ms = max_over_ranks(sum(step_ms), dist, device)
     deverr = moe.moe_device_errors()
     res = {"t": t, "y": y, "ws": ws, "total_ms": total_ms, "step_ms": step_ms, "prof": prof, "clocks": clocks,
            "deverr": deverr, "stream": stream}
@@ -326,7 +347,7 @@ def main():
     r = bench_workload(args, s, rank, world, device, dist)
     K = args.steps
     total_s = r["total_ms"] * 1e-3
-    value = world * s.T * K / total_s
+    value = job_tokens_per_s(world, s.T, K, r["total_ms"])
     tflops = world * s.flops * K / total_s / 1e12
 
     prof = r["prof"]

@@ -39,6 +39,7 @@
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
+#include <cstdlib>
 #include <mutex>
 
 #include "moe_internal.cuh"
@@ -50,19 +51,16 @@ constexpr int BM = 128;            // tile rows (permuted tokens)
 constexpr int BK = 64;             // k per stage: 64 bf16 = one 128-byte swizzle row
 constexpr int UMMA_K = 16;         // k per tcgen05.mma (kind::f16)
 constexpr int MMA_N = 256;         // accumulator columns per tile
-constexpr int STAGES = 4;
-constexpr int A_TILE = BM * BK * 2;            // 16 KiB
-constexpr int B_TILE = MMA_N * BK * 2;         // 32 KiB
-constexpr int B_HALF = B_TILE / 2;             // 128 rows
-constexpr int STAGE_BYTES = A_TILE + B_TILE;   // 48 KiB
+constexpr int A_TILE = BM * BK * 2;            // 16 KiB: 128 rows x 64 k
+constexpr int B_HALF = 128 * BK * 2;           // 16 KiB: 128 rows x 64 k
 constexpr int NUM_THREADS = 192;
 constexpr int TMEM_COLS = 512;                 // 2 accumulators x 256 fp32 columns
-constexpr int SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + 1024;
 constexpr unsigned long long kTimeoutNs = 4000000000ull;
 
 // Instruction descriptor (kind::f16): D fp32 (bits 4-5 = 1), A and B bf16
 // (bits 7-9 = 1, 10-12 = 1), both K-major (bits 15, 16 = 0),
-// N >> 3 in bits 17-22, M >> 4 in bits 24-28.
+// N >> 3 in bits 17-22, M >> 4 in bits 24-28.  This one: M = 128 (single CTA);
+// the pair variant's (M = 256) is Cfg<2>::kIdesc.
 constexpr uint32_t kIdesc = (1u << 4) | (1u << 7) | (1u << 10) |
                             ((uint32_t)(MMA_N >> 3) << 17) | ((uint32_t)(BM >> 4) << 24);
 
@@ -121,22 +119,6 @@ __device__ __forceinline__ void mbar_arrive(uint32_t bar) {
     asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
 }
 
-// Bounded wait: true when the phase completed, false on abort or timeout.
-__device__ __noinline__ bool wait_bounded(uint32_t bar, uint32_t parity, volatile int* abort_flag,
-                                          unsigned int* err) {
-    if (mbar_try_wait(bar, parity)) return true;
-    const unsigned long long t0 = globaltimer();
-    for (;;) {
-        if (mbar_try_wait(bar, parity)) return true;
-        if (*abort_flag) return false;
-        if (globaltimer() - t0 > kTimeoutNs) {
-            *abort_flag = 1;
-            atomicOr(err, 1u);
-            return false;
-        }
-    }
-}
-
 __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map, uint32_t bar,
                                             int c0, int c1) {
     asm volatile(
@@ -193,19 +175,130 @@ __device__ __forceinline__ void tmem_wait_ld() {
 }
 
 // ---------------------------------------------------------------------------
-// Tile enumeration from the expert offsets (identical in every role).
+// Epilogue helpers
 
-__device__ __forceinline__ int count_tiles(const int* s_off, int E, int n_tiles) {
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+    __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+    return *reinterpret_cast<uint32_t*>(&v);
+}
+
+__device__ __forceinline__ float silu_mul(float a, float b) {
+    return __fdividef(a, 1.0f + __expf(-a)) * b;
+}
+
+// ---------------------------------------------------------------------------
+// Pair (cta_group::2) helpers
+
+__device__ __forceinline__ uint32_t cluster_rank() {
+    uint32_t r;
+    asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+    return r;
+}
+
+__device__ __forceinline__ void cluster_sync_all() {
+    asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+
+// Shared::cluster address of the same shared variable in CTA `rank` of the cluster.
+__device__ __forceinline__ uint32_t map_to_rank(uint32_t saddr, uint32_t rank) {
+    uint32_t r;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(saddr), "r"(rank));
+    return r;
+}
+
+__device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_addr) {
+    asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
+}
+
+__device__ __forceinline__ void st_cluster_u32(uint32_t cluster_addr, uint32_t v) {
+    asm volatile("st.shared::cluster.u32 [%0], %1;" ::"r"(cluster_addr), "r"(v) : "memory");
+}
+
+// Bulk tensor load of this CTA's half of a pair tile; completion is counted
+// on the mbarrier of the pair's even CTA (the address with the peer bit cleared).
+__device__ __forceinline__ void tma_load_2d_pair(uint32_t dst, const CUtensorMap* map, uint32_t bar,
+                                                 int c0, int c1) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%2, %3}], [%4];" ::"r"(dst),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(bar & 0xFEFFFFFFu)
+        : "memory");
+}
+
+__device__ __forceinline__ void umma_bf16_pair(uint32_t d_tmem, uint64_t a, uint64_t b, uint32_t idesc, uint32_t acc) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}\n" ::"r"(d_tmem),
+        "l"(a), "l"(b), "r"(idesc), "r"(acc));
+}
+
+// Arrive-one on the mbarrier at the same offset in both CTAs of the pair when
+// the pair's previously issued MMAs complete.
+__device__ __forceinline__ void umma_commit_pair(uint32_t bar) {
+    asm volatile(
+        "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], %1;" ::"r"(bar),
+        "h"((uint16_t)0x3)
+        : "memory");
+}
+
+// Bulk tensor store of a 32-row box from this CTA's shared memory (async
+// proxy); completion is tracked per thread with bulk groups.
+__device__ __forceinline__ void tma_store_2d(const CUtensorMap* map, uint32_t src, int c0, int c1) {
+    asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%1, %2}], [%3];" ::"l"(
+                     reinterpret_cast<uint64_t>(map)),
+                 "r"(c0), "r"(c1), "r"(src)
+                 : "memory");
+}
+__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void bulk_wait_read_le1() { asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory"); }
+__device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+__device__ __forceinline__ void fence_proxy_async_smem() {
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+__device__ __forceinline__ void st_shared_v4(uint32_t addr, uint4 v) {
+    asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w)
+                 : "memory");
+}
+
+// Epilogue staging: each of the 4 epilogue warps owns two 4 KiB buffers
+// (double buffering) holding one 32-row x 128-byte output box in the
+// 128-byte swizzled layout the store's tensor map expects: 16-byte chunk j
+// of row r sits at r * 128 + ((j ^ (r & 7)) << 4), which also makes the 32
+// lanes' shared-memory writes conflict-free.
+constexpr int kOutBoxBytes = 32 * 128;
+constexpr int kOutBytes = 4 * 2 * kOutBoxBytes;
+
+// ---------------------------------------------------------------------------
+// Per-variant constants.  CG = 1: one CTA per 128-row tile, B tile of 256
+// rows in its own shared memory.  CG = 2: a CTA pair per 256-row tile; each
+// CTA holds its 128 rows of A and its 128-row half of B; the even CTA issues
+// M = 256 MMAs that read both CTAs' shared memory and write both CTAs' TMEM.
+
+template <int CG>
+struct Cfg {
+    static constexpr int kTileRows = 128 * CG;               // rows of one tile (pair)
+    static constexpr int kBRows = (CG == 1) ? 256 : 128;     // B rows held by one CTA
+    static constexpr int kBBytes = kBRows * BK * 2;
+    static constexpr int kStageBytes = A_TILE + kBBytes;     // per CTA
+    static constexpr int kStages = (CG == 1) ? 4 : 6;
+    static constexpr int kSmem = 1024 + kStages * kStageBytes + kOutBytes + 1024;
+    static constexpr uint32_t kIdescM = (uint32_t)((128 * CG) >> 4) << 24;
+    static constexpr uint32_t kIdesc = (1u << 4) | (1u << 7) | (1u << 10) |
+                                       ((uint32_t)(MMA_N >> 3) << 17) | kIdescM;
+};
+
+__device__ __forceinline__ int count_tiles_rows(const int* s_off, int E, int n_tiles, int rows_per_tile) {
     int total = 0;
-    for (int e = 0; e < E; ++e) total += ((s_off[e + 1] - s_off[e] + BM - 1) / BM) * n_tiles;
+    for (int e = 0; e < E; ++e) total += ((s_off[e + 1] - s_off[e] + rows_per_tile - 1) / rows_per_tile) * n_tiles;
     return total;
 }
 
-__device__ __forceinline__ void decode_tile(int tile, const int* s_off, int E, int n_tiles, int& e,
-                                            int& m_blk, int& n_blk) {
+__device__ __forceinline__ void decode_tile_rows(int tile, const int* s_off, int E, int n_tiles, int rows_per_tile,
+                                                 int& e, int& m_blk, int& n_blk) {
     int base = 0;
     for (e = 0; e < E; ++e) {
-        const int mt = (s_off[e + 1] - s_off[e] + BM - 1) / BM;
+        const int mt = (s_off[e + 1] - s_off[e] + rows_per_tile - 1) / rows_per_tile;
         const int tiles = mt * n_tiles;
         if (tile < base + tiles) {
             const int local = tile - base;
@@ -218,160 +311,247 @@ __device__ __forceinline__ void decode_tile(int tile, const int* s_off, int E, i
     e = E - 1; m_blk = 0; n_blk = 0;  // not reached for tile < total
 }
 
-__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
-    __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
-    return *reinterpret_cast<uint32_t*>(&v);
+// Bounded wait that, on timeout, also raises the peer CTA's abort flag (pairs).
+__device__ __noinline__ bool wait_bounded_pair(uint32_t bar, uint32_t parity, volatile int* abort_flag,
+                                               unsigned int* err, uint32_t peer_abort_addr) {
+    if (mbar_try_wait(bar, parity)) return true;
+    const unsigned long long t0 = globaltimer();
+    for (;;) {
+        if (mbar_try_wait(bar, parity)) return true;
+        if (*abort_flag) return false;
+        if (globaltimer() - t0 > kTimeoutNs) {
+            *abort_flag = 1;
+            if (peer_abort_addr) st_cluster_u32(peer_abort_addr, 1u);
+            atomicOr(err, 1u);
+            return false;
+        }
+    }
 }
 
-__device__ __forceinline__ float silu_mul(float a, float b) {
-    return __fdividef(a, 1.0f + __expf(-a)) * b;
-}
-
-// ---------------------------------------------------------------------------
-
-template <int MODE>
+template <int MODE, int CG>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
 grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB0,
-                    const __grid_constant__ CUtensorMap tmB1, const KParams p) {
+                    const __grid_constant__ CUtensorMap tmB1, const __grid_constant__ CUtensorMap tmOut,
+                    const KParams p) {
+    using C = Cfg<CG>;
+    constexpr int STG = C::kStages;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t* sA = smem;
-    uint8_t* sB = smem + STAGES * A_TILE;
-    uint64_t* bars = reinterpret_cast<uint64_t*>(sB + STAGES * B_TILE);
+    uint8_t* sB = smem + STG * A_TILE;
+    uint8_t* sOut = sB + STG * C::kBBytes;  // 1024-aligned: stage sizes are multiples of 1 KiB
+    uint64_t* bars = reinterpret_cast<uint64_t*>(sOut + kOutBytes);
     uint64_t* full = bars;
-    uint64_t* empty = bars + STAGES;
-    uint64_t* tfull = bars + 2 * STAGES;
-    uint64_t* tempty = bars + 2 * STAGES + 2;
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * STAGES + 4);
+    uint64_t* empty = bars + STG;
+    uint64_t* tfull = bars + 2 * STG;
+    uint64_t* tempty = bars + 2 * STG + 2;
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * STG + 4);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
     int* s_off = reinterpret_cast<int*>(tmem_slot + 2);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const uint32_t rank = (CG == 2) ? cluster_rank() : 0u;
+    const bool leader = rank == 0;
+    const uint32_t peer_abort = (CG == 2) ? map_to_rank(smem_u32((const void*)abort_flag), rank ^ 1u) : 0u;
 
     if (threadIdx.x == 0) {
-        for (int s = 0; s < STAGES; ++s) {
+        for (int s = 0; s < STG; ++s) {
             mbar_init(smem_u32(&full[s]), 1);
             mbar_init(smem_u32(&empty[s]), 1);
         }
         for (int a = 0; a < 2; ++a) {
             mbar_init(smem_u32(&tfull[a]), 1);
-            mbar_init(smem_u32(&tempty[a]), 128);
+            mbar_init(smem_u32(&tempty[a]), 4 * CG);  // one arrival per epilogue warp of the tile
         }
         *abort_flag = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
     if (threadIdx.x <= p.E) s_off[threadIdx.x] = p.offsets[threadIdx.x];
     if (warp == 1) {
-        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_slot)),
-                     "r"(TMEM_COLS)
-                     : "memory");
-        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+        if constexpr (CG == 1) {
+            asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_slot)),
+                         "r"(TMEM_COLS) : "memory");
+            asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+        } else {
+            asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_slot)),
+                         "r"(TMEM_COLS) : "memory");
+            asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
+        }
     }
     tc_fence_before();
-    __syncthreads();
+    if constexpr (CG == 2) cluster_sync_all(); else __syncthreads();
     tc_fence_after();
     const uint32_t tmem_base = *tmem_slot;
 
-    const int total = count_tiles(s_off, p.E, p.n_tiles);
+    const int total = count_tiles_rows(s_off, p.E, p.n_tiles, C::kTileRows);
     const int kblocks = (p.Kdim + BK - 1) / BK;
+    const int tile0 = (CG == 2) ? (int)(blockIdx.x >> 1) : (int)blockIdx.x;
+    const int tstep = (CG == 2) ? (int)(gridDim.x >> 1) : (int)gridDim.x;
 
     if (warp == 0) {
         if (lane == 0) {
-            // ------------------------------------------------ TMA producer
+            // ------------------------------------------------ TMA producer (both CTAs)
             uint32_t it = 0;
             bool ok = true;
-            for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x) {
+            for (int tile = tile0; tile < total && ok; tile += tstep) {
                 int e, mb, nb;
-                decode_tile(tile, s_off, p.E, p.n_tiles, e, mb, nb);
-                const int rowA = s_off[e] + mb * BM;
-                const int rowB0 = e * p.b_rows_per_expert + nb * (MODE == kUp ? 128 : 256);
-                const int rowB1 = (MODE == kUp) ? rowB0 : rowB0 + 128;
+                decode_tile_rows(tile, s_off, p.E, p.n_tiles, C::kTileRows, e, mb, nb);
+                const int rowA = s_off[e] + mb * C::kTileRows + (int)rank * 128;
+                int rowB0, rowB1;
+                const CUtensorMap* mapB = &tmB0;
+                if constexpr (CG == 1) {
+                    rowB0 = e * p.b_rows_per_expert + nb * (MODE == kUp ? 128 : 256);
+                    rowB1 = (MODE == kUp) ? rowB0 : rowB0 + 128;
+                } else {
+                    if constexpr (MODE == kUp) {
+                        rowB0 = e * p.b_rows_per_expert + nb * 128;   // W1 rows (even CTA) or W3 rows (odd CTA)
+                        if (rank == 1) mapB = &tmB1;
+                    } else {
+                        rowB0 = e * p.b_rows_per_expert + nb * 256 + (int)rank * 128;
+                    }
+                    rowB1 = rowB0;
+                }
                 for (int kb = 0; kb < kblocks; ++kb, ++it) {
-                    const uint32_t s = it % STAGES;
-                    const uint32_t ph = (it / STAGES) & 1u;
-                    if (!wait_bounded(smem_u32(&empty[s]), ph ^ 1u, abort_flag, p.err)) { ok = false; break; }
+                    const uint32_t s = it % STG;
+                    const uint32_t ph = (it / STG) & 1u;
+                    if (!wait_bounded_pair(smem_u32(&empty[s]), ph ^ 1u, abort_flag, p.err, peer_abort)) { ok = false; break; }
                     const uint32_t fb = smem_u32(&full[s]);
-                    mbar_arrive_expect_tx(fb, STAGE_BYTES);
-                    tma_load_2d(smem_u32(sA + s * A_TILE), &tmA, fb, kb * BK, rowA);
-                    tma_load_2d(smem_u32(sB + s * B_TILE), &tmB0, fb, kb * BK, rowB0);
-                    tma_load_2d(smem_u32(sB + s * B_TILE + B_HALF), &tmB1, fb, kb * BK, rowB1);
+                    if constexpr (CG == 1) {
+                        mbar_arrive_expect_tx(fb, C::kStageBytes);
+                        tma_load_2d(smem_u32(sA + s * A_TILE), &tmA, fb, kb * BK, rowA);
+                        tma_load_2d(smem_u32(sB + s * C::kBBytes), &tmB0, fb, kb * BK, rowB0);
+                        tma_load_2d(smem_u32(sB + s * C::kBBytes + B_HALF), &tmB1, fb, kb * BK, rowB1);
+                    } else {
+                        if (leader) mbar_arrive_expect_tx(fb, 2 * C::kStageBytes);  // both CTAs' bytes
+                        tma_load_2d_pair(smem_u32(sA + s * A_TILE), &tmA, fb, kb * BK, rowA);
+                        tma_load_2d_pair(smem_u32(sB + s * C::kBBytes), mapB, fb, kb * BK, rowB0);
+                    }
+                }
+            }
+            // Drain: wait until the MMAs have released the last min(it, STG)
+            // issued stages (use j of a stage completes phase j / STG of its
+            // empty barrier), so no arrival from the pair's commits is still
+            // on its way when the CTA exits.
+            if (ok) {
+                const uint32_t first = it > (uint32_t)STG ? it - (uint32_t)STG : 0u;
+                for (uint32_t j = first; j < it; ++j) {
+                    if (!wait_bounded_pair(smem_u32(&empty[j % STG]), (j / STG) & 1u, abort_flag, p.err, peer_abort))
+                        break;
                 }
             }
         }
         __syncwarp();
     } else if (warp == 1) {
-        if (lane == 0) {
-            // ------------------------------------------------ MMA issuer
+        if (lane == 0 && leader) {
+            // ------------------------------------------------ MMA issuer (even CTA)
             uint32_t it = 0, tcount = 0;
             bool ok = true;
-            for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x, ++tcount) {
+            for (int tile = tile0; tile < total && ok; tile += tstep, ++tcount) {
                 const uint32_t acc = tcount & 1u;
                 const uint32_t use = tcount >> 1;
-                if (!wait_bounded(smem_u32(&tempty[acc]), (use & 1u) ^ 1u, abort_flag, p.err)) break;
+                if (!wait_bounded_pair(smem_u32(&tempty[acc]), (use & 1u) ^ 1u, abort_flag, p.err, peer_abort)) break;
                 tc_fence_after();
                 const uint32_t d_tmem = tmem_base + acc * MMA_N;
                 for (int kb = 0; kb < kblocks; ++kb, ++it) {
-                    const uint32_t s = it % STAGES;
-                    const uint32_t ph = (it / STAGES) & 1u;
-                    if (!wait_bounded(smem_u32(&full[s]), ph, abort_flag, p.err)) { ok = false; break; }
+                    const uint32_t s = it % STG;
+                    const uint32_t ph = (it / STG) & 1u;
+                    if (!wait_bounded_pair(smem_u32(&full[s]), ph, abort_flag, p.err, peer_abort)) { ok = false; break; }
                     tc_fence_after();
                     const uint64_t adesc = sw128_desc(smem_u32(sA + s * A_TILE));
-                    const uint64_t bdesc = sw128_desc(smem_u32(sB + s * B_TILE));
+                    const uint64_t bdesc = sw128_desc(smem_u32(sB + s * C::kBBytes));
 #pragma unroll
                     for (int kk = 0; kk < BK / UMMA_K; ++kk) {
                         // advance 16 bf16 = 32 bytes along K inside the swizzle row
-                        umma_bf16(d_tmem, adesc + (uint64_t)(kk * 2), bdesc + (uint64_t)(kk * 2),
-                                  (kb | kk) != 0 ? 1u : 0u);
+                        if constexpr (CG == 1)
+                            umma_bf16(d_tmem, adesc + (uint64_t)(kk * 2), bdesc + (uint64_t)(kk * 2),
+                                      (kb | kk) != 0 ? 1u : 0u);
+                        else
+                            umma_bf16_pair(d_tmem, adesc + (uint64_t)(kk * 2), bdesc + (uint64_t)(kk * 2), C::kIdesc,
+                                           (kb | kk) != 0 ? 1u : 0u);
                     }
-                    umma_commit(smem_u32(&empty[s]));
+                    if constexpr (CG == 1) umma_commit(smem_u32(&empty[s])); else umma_commit_pair(smem_u32(&empty[s]));
                 }
-                if (ok) umma_commit(smem_u32(&tfull[acc]));
+                if (ok) {
+                    if constexpr (CG == 1) umma_commit(smem_u32(&tfull[acc])); else umma_commit_pair(smem_u32(&tfull[acc]));
+                }
             }
         }
         __syncwarp();
     } else {
-        // ---------------------------------------------------- epilogue
+        // ---------------------------------------------------- epilogue (both CTAs)
         const int quad = warp & 3;  // TMEM lanes 32*quad .. 32*quad+31
-        const int r_in = quad * 32 + lane;
+        const int r_in = (int)rank * 128 + quad * 32 + lane;
         const uint32_t t_lane = tmem_base + ((uint32_t)(quad * 32) << 16);
+        const uint32_t tempty_leader0 = (CG == 2) ? map_to_rank(smem_u32(&tempty[0]), 0) : 0u;
+        const uint32_t out_base = smem_u32(sOut) + (uint32_t)quad * 2u * kOutBoxBytes;
+        uint32_t obox = 0;  // boxes this warp has staged (selects the buffer)
         uint32_t tcount = 0;
-        for (int tile = blockIdx.x; tile < total; tile += gridDim.x, ++tcount) {
+        for (int tile = tile0; tile < total; tile += tstep, ++tcount) {
             int e, mb, nb;
-            decode_tile(tile, s_off, p.E, p.n_tiles, e, mb, nb);
+            decode_tile_rows(tile, s_off, p.E, p.n_tiles, C::kTileRows, e, mb, nb);
             const uint32_t acc = tcount & 1u;
             const uint32_t use = tcount >> 1;
             // every lane waits; the decision to stop is warp-uniform so the
             // .sync.aligned TMEM loads below always run on a converged warp
-            const bool ok = wait_bounded(smem_u32(&tfull[acc]), use & 1u, abort_flag, p.err);
-            if (!__all_sync(0xffffffffu, ok)) break;
+            const bool okw = wait_bounded_pair(smem_u32(&tfull[acc]), use & 1u, abort_flag, p.err, peer_abort);
+            if (!__all_sync(0xffffffffu, okw)) break;
             tc_fence_after();
-            const int row = s_off[e] + mb * BM + r_in;
+            const int row = s_off[e] + mb * C::kTileRows + r_in;
             const bool valid = row < s_off[e + 1];
+            // rows of this warp: whole box stored by TMA when all 32 are the
+            // expert's own; a box straddling the end of the expert's block
+            // uses per-row stores (a full-box store would overwrite the next
+            // expert's rows)
+            const int wrow0 = row - lane;
+            const bool box_ok = wrow0 + 32 <= s_off[e + 1];
             const uint32_t tacc = t_lane + acc * MMA_N;
             if constexpr (MODE == kUp) {
                 __nv_bfloat16* hrow = p.h + (size_t)row * p.n_out;
 #pragma unroll 1
-                for (int c = 0; c < 128; c += 32) {
-                    uint32_t a[32], b[32];
-                    tmem_ld32(tacc + c, a);
-                    tmem_ld32(tacc + 128 + c, b);
-                    tmem_wait_ld();
-                    const int col0 = nb * 128 + c;
-                    if (valid) {
+                for (int c64 = 0; c64 < 128; c64 += 64, ++obox) {
+                    const uint32_t buf = out_base + (obox & 1u) * kOutBoxBytes;
+                    if (box_ok) {
+                        if (lane == 0) bulk_wait_read_le1();  // this buffer's previous store has read it
+                        __syncwarp();
+                    }
+#pragma unroll 1
+                    for (int half = 0; half < 2; ++half) {
+                        const int c = c64 + half * 32;
+                        uint32_t a[32], b[32];
+                        tmem_ld32(tacc + c, a);
+                        tmem_ld32(tacc + 128 + c, b);
+                        tmem_wait_ld();
+                        uint4 pk[4];
 #pragma unroll
                         for (int g = 0; g < 4; ++g) {
-                            if (col0 + g * 8 < p.n_out) {
-                                uint4 pk;
-                                pk.x = pack_bf16x2(silu_mul(__uint_as_float(a[g * 8 + 0]), __uint_as_float(b[g * 8 + 0])),
-                                                   silu_mul(__uint_as_float(a[g * 8 + 1]), __uint_as_float(b[g * 8 + 1])));
-                                pk.y = pack_bf16x2(silu_mul(__uint_as_float(a[g * 8 + 2]), __uint_as_float(b[g * 8 + 2])),
-                                                   silu_mul(__uint_as_float(a[g * 8 + 3]), __uint_as_float(b[g * 8 + 3])));
-                                pk.z = pack_bf16x2(silu_mul(__uint_as_float(a[g * 8 + 4]), __uint_as_float(b[g * 8 + 4])),
-                                                   silu_mul(__uint_as_float(a[g * 8 + 5]), __uint_as_float(b[g * 8 + 5])));
-                                pk.w = pack_bf16x2(silu_mul(__uint_as_float(a[g * 8 + 6]), __uint_as_float(b[g * 8 + 6])),
-                                                   silu_mul(__uint_as_float(a[g * 8 + 7]), __uint_as_float(b[g * 8 + 7])));
-                                *reinterpret_cast<uint4*>(hrow + col0 + g * 8) = pk;
-                            }
+                            pk[g].x = pack_bf16x2(silu_mul(__uint_as_float(a[g * 8 + 0]), __uint_as_float(b[g * 8 + 0])),
+                                                  silu_mul(__uint_as_float(a[g * 8 + 1]), __uint_as_float(b[g * 8 + 1])));
+                            pk[g].y = pack_bf16x2(silu_mul(__uint_as_float(a[g * 8 + 2]), __uint_as_float(b[g * 8 + 2])),
+                                                  silu_mul(__uint_as_float(a[g * 8 + 3]), __uint_as_float(b[g * 8 + 3])));
+                            pk[g].z = pack_bf16x2(silu_mul(__uint_as_float(a[g * 8 + 4]), __uint_as_float(b[g * 8 + 4])),
+                                                  silu_mul(__uint_as_float(a[g * 8 + 5]), __uint_as_float(b[g * 8 + 5])));
+                            pk[g].w = pack_bf16x2(silu_mul(__uint_as_float(a[g * 8 + 6]), __uint_as_float(b[g * 8 + 6])),
+                                                  silu_mul(__uint_as_float(a[g * 8 + 7]), __uint_as_float(b[g * 8 + 7])));
+                        }
+                        if (box_ok) {
+#pragma unroll
+                            for (int g = 0; g < 4; ++g)
+                                st_shared_v4(buf + lane * 128 + ((((half * 4 + g) ^ (lane & 7))) << 4), pk[g]);
+                        } else if (valid) {
+                            const int col0 = nb * 128 + c;
+#pragma unroll
+                            for (int g = 0; g < 4; ++g)
+                                if (col0 + g * 8 < p.n_out) *reinterpret_cast<uint4*>(hrow + col0 + g * 8) = pk[g];
+                        }
+                    }
+                    if (box_ok) {
+                        fence_proxy_async_smem();
+                        __syncwarp();
+                        if (lane == 0) {
+                            // a box wholly past the last column is not stored; the
+                            // (empty) group keeps one group per staged box
+                            if (nb * 128 + c64 < p.n_out) tma_store_2d(&tmOut, buf, nb * 128 + c64, wrow0);
+                            bulk_commit();
                         }
                     }
                 }
@@ -383,37 +563,59 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
                 }
                 float* orow = p.obuf + (size_t)row * p.n_out;
 #pragma unroll 1
-                for (int c = 0; c < MMA_N; c += 32) {
+                for (int c = 0; c < MMA_N; c += 32, ++obox) {
+                    const uint32_t buf = out_base + (obox & 1u) * kOutBoxBytes;
+                    if (box_ok) {
+                        if (lane == 0) bulk_wait_read_le1();
+                        __syncwarp();
+                    }
                     uint32_t o[32];
                     tmem_ld32(tacc + c, o);
                     tmem_wait_ld();
-                    const int col0 = nb * 256 + c;
-                    if (valid) {
+                    uint4 v[8];
 #pragma unroll
-                        for (int g = 0; g < 8; ++g) {
-                            if (col0 + g * 4 < p.n_out) {
-                                float4 v;
-                                v.x = wgt * __uint_as_float(o[g * 4 + 0]);
-                                v.y = wgt * __uint_as_float(o[g * 4 + 1]);
-                                v.z = wgt * __uint_as_float(o[g * 4 + 2]);
-                                v.w = wgt * __uint_as_float(o[g * 4 + 3]);
-                                *reinterpret_cast<float4*>(orow + col0 + g * 4) = v;
-                            }
+                    for (int g = 0; g < 8; ++g) {
+                        v[g].x = __float_as_uint(wgt * __uint_as_float(o[g * 4 + 0]));
+                        v[g].y = __float_as_uint(wgt * __uint_as_float(o[g * 4 + 1]));
+                        v[g].z = __float_as_uint(wgt * __uint_as_float(o[g * 4 + 2]));
+                        v[g].w = __float_as_uint(wgt * __uint_as_float(o[g * 4 + 3]));
+                    }
+                    if (box_ok) {
+#pragma unroll
+                        for (int g = 0; g < 8; ++g) st_shared_v4(buf + lane * 128 + ((g ^ (lane & 7)) << 4), v[g]);
+                        fence_proxy_async_smem();
+                        __syncwarp();
+                        if (lane == 0) {
+                            if (nb * 256 + c < p.n_out) tma_store_2d(&tmOut, buf, nb * 256 + c, wrow0);
+                            bulk_commit();
                         }
+                    } else if (valid) {
+                        const int col0 = nb * 256 + c;
+#pragma unroll
+                        for (int g = 0; g < 8; ++g)
+                            if (col0 + g * 4 < p.n_out) *reinterpret_cast<uint4*>(orow + col0 + g * 4) = v[g];
                     }
                 }
             }
             tc_fence_before();
-            mbar_arrive(smem_u32(&tempty[acc]));
+            __syncwarp();
+            if (lane == 0) {
+                if constexpr (CG == 1) mbar_arrive(smem_u32(&tempty[acc]));
+                else mbar_arrive_cluster(tempty_leader0 + acc * (uint32_t)sizeof(uint64_t));
+            }
         }
+        if (lane == 0) bulk_wait_all();  // stores complete before the CTA's shared memory goes away
+        __syncwarp();
     }
 
     tc_fence_before();
-    __syncthreads();
+    if constexpr (CG == 2) cluster_sync_all(); else __syncthreads();
     if (warp == 1) {
         tc_fence_after();
-        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem_base), "r"(TMEM_COLS)
-                     : "memory");
+        if constexpr (CG == 1)
+            asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem_base), "r"(TMEM_COLS) : "memory");
+        else
+            asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(tmem_base), "r"(TMEM_COLS) : "memory");
     }
 }
 
@@ -435,36 +637,82 @@ void init_encode() {
     g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
 }
 
-// 2-D bf16 row-major [rows, cols] map with a (64 x box_rows) box, 128-byte swizzle.
-bool make_map(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols, uint32_t box_rows) {
+// 2-D row-major [rows, cols] map (bf16 or fp32) with a (box_cols x box_rows)
+// box and 128-byte swizzle; box_cols * element size must be 128 bytes.
+bool make_map(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols, uint32_t box_rows,
+              bool fp32 = false) {
     std::call_once(g_once, init_encode);
     if (!g_encode) return false;
+    const uint32_t esz = fp32 ? 4 : 2;
     cuuint64_t dims[2] = {cols, rows};
-    cuuint64_t strides[1] = {cols * 2};
-    cuuint32_t box[2] = {(cuuint32_t)BK, box_rows};
+    cuuint64_t strides[1] = {cols * esz};
+    cuuint32_t box[2] = {128 / esz, box_rows};
     cuuint32_t estr[2] = {1, 1};
-    CUresult r = g_encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides,
-                          box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-                          CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    CUresult r = g_encode(m, fp32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2,
+                          const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                          CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                          CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     return r == CUDA_SUCCESS;
 }
 
-template <int MODE>
-cudaError_t ensure_smem_attr() {
-    static bool done[64] = {false};
+// Co-resident persistent grid: CTAs (CG = 1) or CTA pairs (CG = 2) that
+// fit on the device at once, capped by an upper bound on the tile count.
+template <int MODE, int CG>
+cudaError_t launch_gemm(const GroupedGemmArgs& a, const CUtensorMap& mA, const CUtensorMap& mB0,
+                        const CUtensorMap& mB1, const CUtensorMap& mOut, const KParams& p, cudaStream_t s) {
+    using C = Cfg<CG>;
+    static int units_cache[64] = {0};
     int dev = 0;
     cudaGetDevice(&dev);
-    if (dev < 64 && done[dev]) return cudaSuccess;
-    cudaError_t e = cudaFuncSetAttribute(grouped_gemm_kernel<MODE>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
-    if (e == cudaSuccess && dev < 64) done[dev] = true;
-    return e;
+    int units = (dev < 64) ? units_cache[dev] : 0;
+    cudaLaunchConfig_t cfg = {};
+    cudaLaunchAttribute attr[1];
+    cfg.blockDim = dim3(NUM_THREADS);
+    cfg.dynamicSmemBytes = C::kSmem;
+    cfg.stream = s;
+    cfg.attrs = attr;
+    cfg.numAttrs = 0;
+    if (CG == 2) {
+        attr[0].id = cudaLaunchAttributeClusterDimension;
+        attr[0].val.clusterDim.x = 2;
+        attr[0].val.clusterDim.y = 1;
+        attr[0].val.clusterDim.z = 1;
+        cfg.numAttrs = 1;
+    }
+    if (!units) {
+        cudaError_t e = cudaFuncSetAttribute(grouped_gemm_kernel<MODE, CG>,
+                                             cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmem);
+        if (e != cudaSuccess) return e;
+        units = a.num_sms / CG;
+        if (CG == 2) {
+            int clusters = 0;
+            cfg.gridDim = dim3(2 * units);
+            if (cudaOccupancyMaxActiveClusters(&clusters, grouped_gemm_kernel<MODE, CG>, &cfg) == cudaSuccess &&
+                clusters > 0 && clusters < units)
+                units = clusters;
+            cudaGetLastError();  // an unsupported query is not an error for the launch
+        }
+        if (dev < 64) units_cache[dev] = units;
+    }
+    const long long ub = (long long)p.n_tiles * ((a.rows + C::kTileRows - 1) / C::kTileRows + a.E);
+    const int grid_units = (int)(ub < units ? ub : units);
+    if (grid_units <= 0) return cudaSuccess;
+    cfg.gridDim = dim3(grid_units * CG);
+    return cudaLaunchKernelEx(&cfg, grouped_gemm_kernel<MODE, CG>, mA, mB0, mB1, mOut, p);
 }
 
-// Persistent grid: one CTA per SM, or fewer if there cannot be that many tiles.
-int gemm_grid(const GroupedGemmArgs& a, int n_tiles) {
-    const long long ub = (long long)n_tiles * ((a.rows + BM - 1) / BM + a.E);
-    return (int)(ub < a.num_sms ? ub : a.num_sms);
+// CTA-pair tiles (M = 256) move a third fewer bytes per MMA from L2 but pad
+// each expert's last tile to 256 rows; measured on B200 the single-CTA
+// 128-row tiles are faster up to ~1000 rows per expert (prefill, T = 4096)
+// and at decode, so pairs are used only when experts average at least 2048
+// rows.  MOE_GEMM_CTA_GROUP = 1 or 2 forces one variant (both are exact; the
+// tests run both).
+int choose_cta_group(const GroupedGemmArgs& a) {
+    if (const char* env = getenv("MOE_GEMM_CTA_GROUP")) {
+        if (env[0] == '1') return 1;
+        if (env[0] == '2') return 2;
+    }
+    return (a.rows >= 2048 * a.E) ? 2 : 1;
 }
 
 }  // namespace
@@ -477,37 +725,35 @@ const char* gemm_init_error() {
 cudaError_t launch_up_swiglu(const GroupedGemmArgs& a, const __nv_bfloat16* x_perm,
                              const __nv_bfloat16* W1, const __nv_bfloat16* W3, __nv_bfloat16* h,
                              cudaStream_t s) {
-    CUtensorMap mA, mB0, mB1;
+    CUtensorMap mA, mB0, mB1, mOut;
     if (!make_map(&mA, x_perm, (uint64_t)a.rows, (uint64_t)a.d, BM) ||
         !make_map(&mB0, W1, (uint64_t)a.E * a.f, (uint64_t)a.d, 128) ||
-        !make_map(&mB1, W3, (uint64_t)a.E * a.f, (uint64_t)a.d, 128))
+        !make_map(&mB1, W3, (uint64_t)a.E * a.f, (uint64_t)a.d, 128) ||
+        !make_map(&mOut, h, (uint64_t)a.rows, (uint64_t)a.f, 32))
         return cudaErrorInvalidValue;
     KParams p{};
     p.offsets = a.offsets; p.E = a.E; p.n_out = a.f; p.Kdim = a.d;
     p.n_tiles = (a.f + 127) / 128; p.b_rows_per_expert = a.f; p.h = h; p.rows = a.rows;
     p.err = a.err;
-    cudaError_t e = ensure_smem_attr<kUp>();
-    if (e != cudaSuccess) return e;
-    grouped_gemm_kernel<kUp><<<gemm_grid(a, p.n_tiles), NUM_THREADS, SMEM_BYTES, s>>>(mA, mB0, mB1, p);
-    return cudaGetLastError();
+    return choose_cta_group(a) == 2 ? launch_gemm<kUp, 2>(a, mA, mB0, mB1, mOut, p, s)
+                                    : launch_gemm<kUp, 1>(a, mA, mB0, mB1, mOut, p, s);
 }
 
 cudaError_t launch_down_scaled(const GroupedGemmArgs& a, const __nv_bfloat16* h,
                                const __nv_bfloat16* W2, const int32_t* perm, const float* topk_w,
                                float* obuf, cudaStream_t s) {
-    CUtensorMap mA, mB;
+    CUtensorMap mA, mB, mOut;
     if (!make_map(&mA, h, (uint64_t)a.rows, (uint64_t)a.f, BM) ||
-        !make_map(&mB, W2, (uint64_t)a.E * a.d, (uint64_t)a.f, 128))
+        !make_map(&mB, W2, (uint64_t)a.E * a.d, (uint64_t)a.f, 128) ||
+        !make_map(&mOut, obuf, (uint64_t)a.rows, (uint64_t)a.d, 32, true))
         return cudaErrorInvalidValue;
     KParams p{};
     p.offsets = a.offsets; p.E = a.E; p.n_out = a.d; p.Kdim = a.f;
     p.n_tiles = (a.d + 255) / 256; p.b_rows_per_expert = a.d;
     p.perm = perm; p.topk_w = topk_w; p.obuf = obuf; p.rows = a.rows;
     p.err = a.err;
-    cudaError_t e = ensure_smem_attr<kDown>();
-    if (e != cudaSuccess) return e;
-    grouped_gemm_kernel<kDown><<<gemm_grid(a, p.n_tiles), NUM_THREADS, SMEM_BYTES, s>>>(mA, mB, mB, p);
-    return cudaGetLastError();
+    return choose_cta_group(a) == 2 ? launch_gemm<kDown, 2>(a, mA, mB, mB, mOut, p, s)
+                                    : launch_gemm<kDown, 1>(a, mA, mB, mB, mOut, p, s);
 }
 
 }  // namespace moe

@@ -6,6 +6,10 @@
 //  gather_rows      x_perm[r] = x[perm[r] / k]            (bf16 path)
 //  combine_kernel   y[t] = (residual[t] +) sum_j obuf[inv[t*k + j]]
 //
+// The gather and the combine are flat: one thread per 16-byte piece, so
+// every piece's loads are in flight at once (HBM-bound, not latency-bound,
+// for any T).
+//
 // The scatter is stable and deterministic without global atomics: the
 // assignments are walked in tiles of 1024 in increasing id; inside a warp,
 // __match_any_sync groups lanes with the same expert and a lane's rank is
@@ -89,81 +93,122 @@ permute_kernel(const int32_t* __restrict__ idx, int n, int E, int32_t* __restric
     }
 }
 
-constexpr int kRowWarps = 8;
+constexpr int kFlatThreads = 256;
 
-__global__ void __launch_bounds__(kRowWarps * 32)
+// One thread per 16-byte piece of x_perm: x_perm[r, 8v..8v+7] = x[perm[r] / k, 8v..8v+7].
+// Each thread handles kUnroll pieces per pass (grid-strided), all loads first.
+constexpr int kUnroll = 4;
+
+__global__ void __launch_bounds__(kFlatThreads)
 gather_rows_kernel(const __nv_bfloat16* __restrict__ x, const int32_t* __restrict__ perm, int rows,
                    int d, int k, __nv_bfloat16* __restrict__ xp) {
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int nvec = d / 8;
-    for (int r = blockIdx.x * kRowWarps + warp; r < rows; r += gridDim.x * kRowWarps) {
-        const int q = perm[r];
-        uint4* dst = reinterpret_cast<uint4*>(xp + (size_t)r * d);
-        if ((unsigned)q >= (unsigned)rows) {  // not a valid assignment id: zero row
-            for (int v = lane; v < nvec; v += 32) dst[v] = make_uint4(0, 0, 0, 0);
-            continue;
+    const long long total = (long long)rows * nvec;
+    const long long stride = (long long)gridDim.x * kFlatThreads;
+    for (long long base = (long long)blockIdx.x * kFlatThreads + threadIdx.x; base < total; base += stride * kUnroll) {
+        uint4 val[kUnroll];
+        long long item[kUnroll];
+#pragma unroll
+        for (int u = 0; u < kUnroll; ++u) {
+            item[u] = base + u * stride;
+            val[u] = make_uint4(0, 0, 0, 0);  // (a row with an invalid assignment id stays zero)
+            if (item[u] < total) {
+                const int r = (int)(item[u] / nvec), v = (int)(item[u] - (long long)r * nvec);
+                const int q = __ldg(perm + r);
+                if ((unsigned)q < (unsigned)rows)
+                    val[u] = __ldg(reinterpret_cast<const uint4*>(x + (size_t)(q / k) * d) + v);
+            }
         }
-        const uint4* src = reinterpret_cast<const uint4*>(x + (size_t)(q / k) * d);
-        for (int v = lane; v < nvec; v += 32) dst[v] = __ldg(src + v);
+#pragma unroll
+        for (int u = 0; u < kUnroll; ++u)
+            if (item[u] < total) reinterpret_cast<uint4*>(xp)[item[u]] = val[u];
+    }
+}
+
+// One thread per 4 output features of one token:
+// y[t, 4v..4v+3] = (residual +) sum_j obuf[inv[t*k + j], 4v..4v+3], slot order.
+// kUnroll pieces per thread per pass, loads first.
+template <bool BF16>
+__device__ __forceinline__ void combine_store(const float4& acc0, const void* residual, void* y, int t, int v,
+                                              int d) {
+    float4 acc = acc0;
+    if constexpr (BF16) {
+        if (residual) {
+            const uint2 rq = __ldg(reinterpret_cast<const uint2*>(
+                reinterpret_cast<const __nv_bfloat16*>(residual) + (size_t)t * d) + v);
+            acc.x = __uint_as_float(rq.x << 16) + acc.x;
+            acc.y = __uint_as_float(rq.x & 0xFFFF0000u) + acc.y;
+            acc.z = __uint_as_float(rq.y << 16) + acc.z;
+            acc.w = __uint_as_float(rq.y & 0xFFFF0000u) + acc.w;
+        }
+        __nv_bfloat162 lo = __floats2bfloat162_rn(acc.x, acc.y);
+        __nv_bfloat162 hi = __floats2bfloat162_rn(acc.z, acc.w);
+        uint2 out;
+        out.x = *reinterpret_cast<uint32_t*>(&lo);
+        out.y = *reinterpret_cast<uint32_t*>(&hi);
+        reinterpret_cast<uint2*>(reinterpret_cast<__nv_bfloat16*>(y) + (size_t)t * d)[v] = out;
+    } else {
+        if (residual) {
+            const float4 r = __ldg(reinterpret_cast<const float4*>(
+                reinterpret_cast<const float*>(residual) + (size_t)t * d) + v);
+            acc.x = r.x + acc.x; acc.y = r.y + acc.y; acc.z = r.z + acc.z; acc.w = r.w + acc.w;
+        }
+        reinterpret_cast<float4*>(reinterpret_cast<float*>(y) + (size_t)t * d)[v] = acc;
     }
 }
 
 template <bool BF16>
-__global__ void __launch_bounds__(kRowWarps * 32)
+__global__ void __launch_bounds__(kFlatThreads)
 combine_kernel(const float* __restrict__ obuf, const int32_t* __restrict__ inv,
                const void* __restrict__ residual, int T, int d, int k, void* __restrict__ y) {
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int nvec = d / 4;
-    for (int t = blockIdx.x * kRowWarps + warp; t < T; t += gridDim.x * kRowWarps) {
-        int rows[kMaxTopK];
+    const long long total = (long long)T * nvec;
+    const unsigned n = (unsigned)(T * k);
+    const long long stride = (long long)gridDim.x * kFlatThreads;
+    for (long long base = (long long)blockIdx.x * kFlatThreads + threadIdx.x; base < total; base += stride * kUnroll) {
+        float4 acc[kUnroll];
 #pragma unroll
-        for (int j = 0; j < kMaxTopK; ++j) {
-            rows[j] = (j < k) ? inv[(size_t)t * k + j] : -1;
-            if ((unsigned)rows[j] >= (unsigned)(T * k)) rows[j] = -1;  // unrouted slot adds nothing
+        for (int u = 0; u < kUnroll; ++u) {
+            acc[u] = make_float4(0.f, 0.f, 0.f, 0.f);
+            const long long it = base + u * stride;
+            if (it >= total) continue;
+            const int t = (int)(it / nvec), v = (int)(it - (long long)t * nvec);
+            for (int j = 0; j < k; ++j) {
+                const int r = __ldg(inv + (size_t)t * k + j);
+                if ((unsigned)r >= n) continue;  // unrouted slot adds nothing
+                const float4 o = __ldg(reinterpret_cast<const float4*>(obuf + (size_t)r * d) + v);
+                if (j == 0) {
+                    acc[u] = o;
+                } else {
+                    acc[u].x += o.x; acc[u].y += o.y; acc[u].z += o.z; acc[u].w += o.w;
+                }
+            }
         }
-        for (int v = lane; v < nvec; v += 32) {
-            float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-            if (rows[0] >= 0) acc = __ldg(reinterpret_cast<const float4*>(obuf + (size_t)rows[0] * d) + v);
 #pragma unroll
-            for (int j = 1; j < kMaxTopK; ++j) {
-                if (rows[j] >= 0) {
-                    const float4 o = __ldg(reinterpret_cast<const float4*>(obuf + (size_t)rows[j] * d) + v);
-                    acc.x += o.x; acc.y += o.y; acc.z += o.z; acc.w += o.w;
-                }
-            }
-            if constexpr (BF16) {
-                if (residual) {
-                    const uint2 rq = __ldg(reinterpret_cast<const uint2*>(
-                        reinterpret_cast<const __nv_bfloat16*>(residual) + (size_t)t * d) + v);
-                    acc.x = __uint_as_float(rq.x << 16) + acc.x;
-                    acc.y = __uint_as_float(rq.x & 0xFFFF0000u) + acc.y;
-                    acc.z = __uint_as_float(rq.y << 16) + acc.z;
-                    acc.w = __uint_as_float(rq.y & 0xFFFF0000u) + acc.w;
-                }
-                __nv_bfloat162 lo = __floats2bfloat162_rn(acc.x, acc.y);
-                __nv_bfloat162 hi = __floats2bfloat162_rn(acc.z, acc.w);
-                uint2 out;
-                out.x = *reinterpret_cast<uint32_t*>(&lo);
-                out.y = *reinterpret_cast<uint32_t*>(&hi);
-                reinterpret_cast<uint2*>(reinterpret_cast<__nv_bfloat16*>(y) + (size_t)t * d)[v] = out;
-            } else {
-                if (residual) {
-                    const float4 r = __ldg(reinterpret_cast<const float4*>(
-                        reinterpret_cast<const float*>(residual) + (size_t)t * d) + v);
-                    acc.x = r.x + acc.x; acc.y = r.y + acc.y; acc.z = r.z + acc.z; acc.w = r.w + acc.w;
-                }
-                reinterpret_cast<float4*>(reinterpret_cast<float*>(y) + (size_t)t * d)[v] = acc;
-            }
+        for (int u = 0; u < kUnroll; ++u) {
+            const long long it = base + u * stride;
+            if (it >= total) continue;
+            const int t = (int)(it / nvec), v = (int)(it - (long long)t * nvec);
+            combine_store<BF16>(acc[u], residual, y, t, v, d);
         }
     }
 }
 
-int row_grid(int rows) {
-    int dev = 0, sms = 148;
+// Grid for a flat kernel over `items` threads: enough blocks for all of them,
+// capped at 8 resident blocks per SM (the kernels loop with a grid stride).
+int flat_grid(long long items) {
+    static int sms_cache[64] = {0};
+    int dev = 0;
     cudaGetDevice(&dev);
-    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-    const int need = (rows + kRowWarps - 1) / kRowWarps;
-    return need < sms * 8 ? need : sms * 8;
+    int sms = (dev < 64) ? sms_cache[dev] : 0;
+    if (!sms) {
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+        if (sms <= 0) sms = 148;
+        if (dev < 64) sms_cache[dev] = sms;
+    }
+    const long long need = (items + kFlatThreads * kUnroll - 1) / (kFlatThreads * kUnroll);
+    const long long cap = (long long)sms * 8;
+    return (int)(need < cap ? (need > 0 ? need : 1) : cap);
 }
 
 }  // namespace
@@ -194,16 +239,16 @@ cudaError_t launch_permute(const int32_t* idx, int n, int E, int32_t* offsets, i
 
 cudaError_t launch_gather_rows_bf16(const __nv_bfloat16* x, const int32_t* perm, int rows, int d,
                                     int k, __nv_bfloat16* x_perm, cudaStream_t s) {
-    gather_rows_kernel<<<row_grid(rows), kRowWarps * 32, 0, s>>>(x, perm, rows, d, k, x_perm);
+    gather_rows_kernel<<<flat_grid((long long)rows * (d / 8)), kFlatThreads, 0, s>>>(x, perm, rows, d, k, x_perm);
     return cudaGetLastError();
 }
 
 cudaError_t launch_combine(const float* obuf, const int32_t* inv, const void* residual, int T,
                            int d, int k, bool bf16, void* y, cudaStream_t s) {
     if (bf16)
-        combine_kernel<true><<<row_grid(T), kRowWarps * 32, 0, s>>>(obuf, inv, residual, T, d, k, y);
+        combine_kernel<true><<<flat_grid((long long)T * (d / 4)), kFlatThreads, 0, s>>>(obuf, inv, residual, T, d, k, y);
     else
-        combine_kernel<false><<<row_grid(T), kRowWarps * 32, 0, s>>>(obuf, inv, residual, T, d, k, y);
+        combine_kernel<false><<<flat_grid((long long)T * (d / 4)), kFlatThreads, 0, s>>>(obuf, inv, residual, T, d, k, y);
     return cudaGetLastError();
 }
 

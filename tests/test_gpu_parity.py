@@ -114,20 +114,35 @@ def test_permute_flags_bad_expert_ids():
 
 # ---------------------------------------------------------------- whole layer, every token
 
-@pytest.mark.parametrize("shape", [
+F32_SHAPES = [
     synth.CONFIGS["tiny"],
     synth.MoEShape("f32-ragged", 37, 72, 136, 8, 2, "f32"),
     synth.MoEShape("f32-mid", 200, 256, 512, 8, 2, "f32"),
-    synth.MoEShape("bf16-tiles", 1000, 128, 384, 4, 2, "bf16"),     # 500 rows/expert: 3 full tiles + tail
+]
+BF16_SHAPES = [
+    synth.MoEShape("bf16-tiles", 1000, 128, 384, 4, 2, "bf16"),     # 500 rows/expert: several tiles + tail
     synth.MoEShape("bf16-ragged", 37, 72, 136, 8, 2, "bf16"),       # every tile ragged, K tails
     synth.MoEShape("bf16-wide", 700, 512, 1024, 8, 2, "bf16"),
     synth.MoEShape("bf16-k1", 300, 256, 256, 8, 1, "bf16"),
     synth.MoEShape("bf16-E64k8", 256, 128, 128, 64, 8, "bf16"),
     synth.MoEShape("bf16-T1", 1, 64, 128, 8, 2, "bf16"),
-], ids=lambda s: s.name)
-def test_layer_parity_every_token(shape):
+    synth.MoEShape("bf16-many-tiles", 2500, 256, 768, 8, 2, "bf16"),  # 625 rows/expert, 2-3 pair tiles
+]
+
+
+@pytest.mark.parametrize("shape", F32_SHAPES, ids=lambda s: s.name)
+def test_layer_parity_every_token_f32(shape):
     rel, _ = full_check(shape)
-    assert rel <= {"f32": 1e-5, "bf16": 1e-2}[shape.dtype]
+    assert rel <= 1e-5
+
+
+@pytest.mark.parametrize("cta_group", ["1", "2"])
+@pytest.mark.parametrize("shape", BF16_SHAPES, ids=lambda s: s.name)
+def test_layer_parity_every_token_bf16(shape, cta_group, monkeypatch):
+    """Both GEMM variants (single-CTA 128-row tiles, CTA-pair 256-row tiles)."""
+    monkeypatch.setenv("MOE_GEMM_CTA_GROUP", cta_group)
+    rel, _ = full_check(shape)
+    assert rel <= 1e-2
 
 
 @pytest.mark.parametrize("seed", range(1, 21))
@@ -273,6 +288,13 @@ def test_decode_full_shape_every_token(mixtral_weights):
 
 def test_prefill_full_shape(mixtral_weights):
     big_check("prefill", mixtral_weights, 256)
+
+
+@pytest.mark.parametrize("name,cta_group", [("decode", "2"), ("prefill", "1")])
+def test_full_shapes_other_gemm_variant(name, cta_group, mixtral_weights, monkeypatch):
+    """The variant the size heuristic does not pick, at the full shapes."""
+    monkeypatch.setenv("MOE_GEMM_CTA_GROUP", cta_group)
+    big_check(name, mixtral_weights, None if name == "decode" else 256)
 
 
 def test_skewed_full_shape(mixtral_weights):
