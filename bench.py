@@ -294,6 +294,49 @@ def bench_workload(args, s, rank, world, device, dist, extras_for_decode=False):
     return res
 
 
+def bench_stack(steps, device, pk):
+    """The 32-layer stack (T = 8192, 90 GB of per-layer weights, residual
+    between layers) as one moe_stack_forward call captured in a CUDA graph."""
+    import torch
+    import sparse_mixture_experts_06_b200 as moe
+    import synth
+    from synth.device import device_inputs, normal_tensor
+    import dataclasses
+    s = synth.CONFIGS["stack"]
+    one = dataclasses.replace(s, name="stack-layer", layers=1)
+    layers = []
+    for l in range(s.layers):
+        w = device_inputs(one, 0, layer=l, device=device, with_x=False)
+        layers.append((w["Wg"], w["W1"], w["W3"], w["W2"]))
+    x = normal_tensor((s.T, s.d), replica_x_seed(0), synth.tensor_id(synth.TENSOR_X), 1.0, s.dtype, device)
+    y = torch.empty_like(x)
+    scratch = torch.empty_like(x)
+    ws = torch.empty(moe.moe_workspace_size(s.T, s.d, s.f, s.E, s.k, 0), dtype=torch.uint8, device=device)
+    moe.moe_stack_forward(x, layers, s.k, y=y, scratch=scratch, workspace=ws)  # one-time set-up, uncaptured
+    torch.cuda.synchronize(device)
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        moe.moe_stack_forward(x, layers, s.k, y=y, scratch=scratch, workspace=ws)
+    g.replay()
+    torch.cuda.synchronize(device)
+    stream = torch.cuda.current_stream(device)
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    for _ in range(steps):
+        g.replay()
+    b.record(stream)
+    torch.cuda.synchronize(device)
+    ms = a.elapsed_time(b) / steps
+    out = {"workload": "32-layer Mixtral-8x7B MoE stack, T=%d tokens, residual between layers, per-layer weights "
+                       "(%.1f GB, W2 scaled by 1/4 so the residual stream stays finite), one CUDA graph"
+                       % (s.T, s.weight_bytes / 1e9),
+           "ms_per_step": ms, "tokens_per_s": s.T / (ms * 1e-3), "tflops": s.flops / (ms * 1e-3) / 1e12,
+           "frac_of_bf16_peak": s.flops / (ms * 1e-3) / 1e12 / pk["bf16_tflops"], "ms_per_layer": ms / s.layers,
+           "steps": steps, "device_error_flags": moe.moe_device_errors()}
+    del g, layers
+    return out
+
+
 def e2e_leg(args, s, t, device, steps):
     """Same layer through the public entry point moe_layer_forward (library
     workspace), with the step's tokens copied in from pinned host memory and
@@ -416,6 +459,22 @@ def main():
                           "device_error_flags": rd["deverr"]}
         del rd, counts
         torch.cuda.empty_cache()
+        sk = synth.CONFIGS["skewed"]
+        sargs = argparse.Namespace(**vars(args))
+        sargs.steps = max(10, min(60, K))
+        rs = bench_workload(sargs, sk, rank, world, device, dist, extras_for_decode=True)
+        sms = rs["total_ms"] / sargs.steps
+        line["skewed"] = {"workload": workload_desc(sk, world)["workload"] + ", Zipf-shaped load (hottest expert 35%)",
+                          "ms_per_step": sms, "tokens_per_s": world * sk.T / (sms * 1e-3),
+                          "tflops": sk.flops / (sms * 1e-3) / 1e12,
+                          "frac_of_bf16_peak": sk.flops / (sms * 1e-3) / 1e12 / pk["bf16_tflops"],
+                          "stages_ms_per_step": {k: round(v[0] / sargs.steps, 4) for k, v in rs["prof"].items() if v[1]},
+                          "device_error_flags": rs["deverr"]}
+        del rs
+        torch.cuda.empty_cache()
+        if world == 1:
+            line["stack"] = bench_stack(max(3, min(10, K)), device, pk)
+            torch.cuda.empty_cache()
 
     if rank == 0 and world == 1 and not args.no_extras:
         import numpy as np

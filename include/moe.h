@@ -30,7 +30,7 @@
  *    caller's next synchronisation, as in CUDA; conditions the kernels
  *    detect themselves (an expert id out of range, a pipeline wait that
  *    timed out) set device flags read by moe_device_errors().
- *  - Limits on the GPU path: 1 <= E <= 64, 1 <= k <= min(E, 8), T >= 0
+ *  - Limits on the GPU path: 1 <= E <= 64, 1 <= k <= E, T >= 0
  *    (T = 0 is a no-op), d and f >= 8 and multiples of 8 (16-byte rows for
  *    the tensor-memory-accelerator copies), all pointers 16-byte aligned.
  *    Non-finite inputs give undefined outputs.
@@ -59,7 +59,7 @@ typedef enum { MOE_BF16 = 0, MOE_F32 = 1 } moe_dtype;
 enum {
     MOE_OK = 0,
     MOE_ERR_INVALID_ARG = 1, /* null pointer, size out of range, misalignment      */
-    MOE_ERR_UNSUPPORTED = 2, /* valid for the method but not on this GPU path (k>8) */
+    MOE_ERR_UNSUPPORTED = 2, /* valid for the method but not on this GPU path         */
     MOE_ERR_WORKSPACE = 3,   /* workspace null or smaller than moe_workspace_size   */
     MOE_ERR_CUDA = 4         /* a CUDA call failed; see moe_last_error_string()     */
 };
@@ -93,6 +93,20 @@ int moe_router_topk(const void* x, const void* Wg, int T, int d, int E, int k, i
 int moe_permute(const int32_t* topk_idx, int T, int E, int k, int32_t* offsets, int32_t* perm,
                 int32_t* inv, moe_stream_t stream);
 
+/* Routing statistics ("Mixtral of Experts" §5, tab. 5, routing analysis) of
+ * a routing topk_idx [T, k] (as produced by moe_router_topk), written to
+ * out[E + 3] (uint32, zeroed by the call):
+ *   out[e]     assignments to expert e (the expert load histogram)
+ *   out[E]     consecutive token pairs whose first choices agree
+ *   out[E+1]   consecutive token pairs whose kept expert sets intersect (the
+ *              "first or second choice" repetition for k = 2)
+ *   out[E+2]   consecutive pairs counted: token t >= 1 that does not start a
+ *              sequence of seq_len tokens (seq_len <= 0: one sequence).
+ * Under uniform routing the two rates are 1/E and 1 - C(E-k,k)/C(E,k)
+ * (12.5% and 13/28 = 46.4% for E = 8, k = 2).  Exact integer counts. */
+int moe_routing_stats(const int32_t* topk_idx, int T, int E, int k, int seq_len, unsigned int* out,
+                      moe_stream_t stream);
+
 /* The experts and the combine ("Mixtral of Experts" §2.1 display 3; Method,
  * step 4; SwiGLU expert).  For every permuted row r of expert e with
  * assignment q = perm[r] = t*k + j:  h_r = SiLU(W1_e x_t) * (W3_e x_t)
@@ -121,6 +135,21 @@ int moe_layer_forward_ex(const void* x, const void* Wg, const void* W1, const vo
                          const void* W2, const void* residual, int T, int d, int f, int E,
                          int k, int dtype, void* workspace, size_t ws_bytes, void* y,
                          moe_stream_t stream);
+
+/* A stack of L layers with the residual stream between them (Method, step 5;
+ * tab. 1: 32 layers): x_{l+1} = x_l + MoE_l(x_l) for l = 0 .. L-1, y = x_L.
+ * The residual is added in the combine kernel of each layer (no extra
+ * pass).  Wg, W1, W3, W2 are HOST arrays of L device pointers (layer l's
+ * weights, layouts as above).  scratch: a caller [T, d] device buffer of the
+ * activation dtype (the layers ping-pong between y and scratch; unused when
+ * L = 1); x is left untouched; x, y and scratch must be distinct.
+ * workspace: moe_workspace_size() bytes, reused by every layer.  Nothing is
+ * allocated, so the whole call can be captured into one CUDA graph (after
+ * one uncaptured call has done the library's one-time set-up). */
+int moe_stack_forward(const void* x, const void* const* Wg, const void* const* W1,
+                      const void* const* W3, const void* const* W2, int L, int T, int d, int f,
+                      int E, int k, int dtype, void* scratch, void* workspace, size_t ws_bytes,
+                      void* y, moe_stream_t stream);
 
 /* The whole bf16 layer, like moe_layer_forward, for callers that cannot
  * allocate device memory while they run: a plug-in inside a host framework

@@ -190,3 +190,30 @@ def permute(idx: np.ndarray, E: int):
         inv[q] = r
         nxt[e] = r + 1
     return offsets.astype(np.int32), perm.astype(np.int32), inv.astype(np.int32)
+
+
+def routing_stats(idx: np.ndarray, E: int, seq_len: int = 0) -> np.ndarray:
+    """Routing statistics of "Mixtral of Experts" §5 / tab. 5, by their
+    definition, with plain loops.  Returns int64 [E + 3]:
+    loads of the E experts (assignments per expert); then, over consecutive
+    token pairs (t-1, t) inside a sequence (sequences of seq_len tokens;
+    seq_len <= 0: one sequence), the number whose first choices agree, the
+    number whose kept expert sets intersect (the card's "first or second
+    choice" repetition for k = 2, whose uniform-routing rate 1 - C(6,2)/C(8,2)
+    = 13/28 matches the quoted ~46%), and the number of pairs counted."""
+    idx = np.asarray(idx)
+    T, k = idx.shape
+    load = [0] * E
+    for t in range(T):
+        for j in range(k):
+            load[int(idx[t, j])] += 1
+    first = overlap = pairs = 0
+    for t in range(1, T):
+        if seq_len > 0 and t % seq_len == 0:
+            continue
+        pairs += 1
+        if idx[t, 0] == idx[t - 1, 0]:
+            first += 1
+        if set(idx[t].tolist()) & set(idx[t - 1].tolist()):
+            overlap += 1
+    return np.array(load + [first, overlap, pairs], dtype=np.int64)

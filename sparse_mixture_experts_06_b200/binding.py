@@ -23,10 +23,12 @@ _SIGS = {
     "moe_workspace_size": ([_I, _I, _I, _I, _I, _I], ctypes.c_size_t),
     "moe_router_topk": ([_P, _P, _I, _I, _I, _I, _I, _P, _P, _P], _I),
     "moe_permute": ([_P, _I, _I, _I, _P, _P, _P, _P], _I),
+    "moe_routing_stats": ([_P, _I, _I, _I, _I, _P, _P], _I),
     "moe_expert_ffn": ([_P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _P, _Z, _P, _P], _I),
     "moe_layer_forward": ([_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _P, _P], _I),
     "moe_layer_forward_ex": ([_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _P, _Z, _P, _P], _I),
     "moe_layer_forward_noalloc": ([_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _P, _P], _I),
+    "moe_stack_forward": ([_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _P, _P, _Z, _P, _P], _I),
     "moe_release_workspace": ([_P], _I),
     "moe_device_errors": ([], ctypes.c_uint),
     "moe_profile_enable": ([_I], _I),
@@ -145,6 +147,18 @@ def moe_permute(topk_idx, E, offsets=None, perm=None, inv=None, stream=None):
     return offsets, perm, inv
 
 
+def moe_routing_stats(topk_idx, E, seq_len=0, out=None, stream=None):
+    """Expert loads and consecutive-token repetition counts (uint32 [E + 3]):
+    loads[0:E], first-choice repeats, kept-set overlaps, pairs counted."""
+    import torch
+    _dev(topk_idx)
+    T, k = topk_idx.shape
+    out = torch.empty(E + 3, dtype=torch.int32, device=topk_idx.device) if out is None else out
+    _check(lib.moe_routing_stats(_ptr(topk_idx), T, E, k, seq_len, _ptr(out), _stream(stream, topk_idx)),
+           "moe_routing_stats")
+    return out
+
+
 def _workspace(T, d, f, E, k, dt, device, workspace):
     import torch
     need = moe_workspace_size(T, d, f, E, k, dt)
@@ -204,6 +218,24 @@ def moe_layer_forward_ex(x, Wg, W1, W3, W2, k, residual=None, y=None, workspace=
     ws, nb = _workspace(T, d, f, E, k, dt, x.device, workspace)
     _check(lib.moe_layer_forward_ex(_ptr(x), _ptr(Wg), _ptr(W1), _ptr(W3), _ptr(W2), _ptr(residual), T, d, f, E, k,
                                     dt, _ptr(ws), nb, _ptr(y), _stream(stream, x)), "moe_layer_forward_ex")
+    return y
+
+
+def moe_stack_forward(x, layers, k, y=None, scratch=None, workspace=None, stream=None):
+    """L layers with the residual between them: `layers` is a list of
+    (Wg, W1, W3, W2) device tensors; returns y = x_L."""
+    import torch
+    L = len(layers)
+    _dev(x, *[w for lay in layers for w in lay])
+    T, d = x.shape
+    E, f, _ = layers[0][1].shape
+    dt = _dtype_code(x)
+    y = torch.empty_like(x) if y is None else y
+    scratch = torch.empty_like(x) if (scratch is None and L > 1) else scratch
+    ws, nb = _workspace(T, d, f, E, k, dt, x.device, workspace)
+    arr = [(ctypes.c_void_p * L)(*[lay[i].data_ptr() for lay in layers]) for i in range(4)]
+    _check(lib.moe_stack_forward(_ptr(x), arr[0], arr[1], arr[2], arr[3], L, T, d, f, E, k, dt, _ptr(scratch),
+                                 _ptr(ws), nb, _ptr(y), _stream(stream, x)), "moe_stack_forward")
     return y
 
 

@@ -702,17 +702,18 @@ cudaError_t launch_gemm(const GroupedGemmArgs& a, const CUtensorMap& mA, const C
 }
 
 // CTA-pair tiles (M = 256) move a third fewer bytes per MMA from L2 but pad
-// each expert's last tile to 256 rows; measured on B200 the single-CTA
-// 128-row tiles are faster up to ~1000 rows per expert (prefill, T = 4096)
-// and at decode, so pairs are used only when experts average at least 2048
-// rows.  MOE_GEMM_CTA_GROUP = 1 or 2 forces one variant (both are exact; the
-// tests run both).
-int choose_cta_group(const GroupedGemmArgs& a) {
+// each expert's last tile to 256 rows.  Measured on B200 (prefill T = 4096
+// and skewed T = 16384): the down-projection (K = f = 14336) gains from
+// pairs once experts average >= 512 rows; the up-projection (K = d) does not
+// (the padding costs as much as the pair saves), and neither does decode.
+// MOE_GEMM_CTA_GROUP = 1 or 2 forces one variant for both GEMMs (both are
+// exact; the tests run both).
+int choose_cta_group(const GroupedGemmArgs& a, int mode) {
     if (const char* env = getenv("MOE_GEMM_CTA_GROUP")) {
         if (env[0] == '1') return 1;
         if (env[0] == '2') return 2;
     }
-    return (a.rows >= 2048 * a.E) ? 2 : 1;
+    return (mode == kDown && a.rows >= 512 * a.E) ? 2 : 1;
 }
 
 }  // namespace
@@ -735,7 +736,7 @@ cudaError_t launch_up_swiglu(const GroupedGemmArgs& a, const __nv_bfloat16* x_pe
     p.offsets = a.offsets; p.E = a.E; p.n_out = a.f; p.Kdim = a.d;
     p.n_tiles = (a.f + 127) / 128; p.b_rows_per_expert = a.f; p.h = h; p.rows = a.rows;
     p.err = a.err;
-    return choose_cta_group(a) == 2 ? launch_gemm<kUp, 2>(a, mA, mB0, mB1, mOut, p, s)
+    return choose_cta_group(a, kUp) == 2 ? launch_gemm<kUp, 2>(a, mA, mB0, mB1, mOut, p, s)
                                     : launch_gemm<kUp, 1>(a, mA, mB0, mB1, mOut, p, s);
 }
 
@@ -752,7 +753,7 @@ cudaError_t launch_down_scaled(const GroupedGemmArgs& a, const __nv_bfloat16* h,
     p.n_tiles = (a.d + 255) / 256; p.b_rows_per_expert = a.d;
     p.perm = perm; p.topk_w = topk_w; p.obuf = obuf; p.rows = a.rows;
     p.err = a.err;
-    return choose_cta_group(a) == 2 ? launch_gemm<kDown, 2>(a, mA, mB, mB, mOut, p, s)
+    return choose_cta_group(a, kDown) == 2 ? launch_gemm<kDown, 2>(a, mA, mB, mB, mOut, p, s)
                                     : launch_gemm<kDown, 1>(a, mA, mB, mB, mOut, p, s);
 }
 

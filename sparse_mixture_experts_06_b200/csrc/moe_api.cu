@@ -238,6 +238,19 @@ int moe_permute(const int32_t* topk_idx, int T, int E, int k, int32_t* offsets, 
     return e == cudaSuccess ? MOE_OK : cuda_fail(e, "permute");
 }
 
+int moe_routing_stats(const int32_t* topk_idx, int T, int E, int k, int seq_len, unsigned int* out,
+                      moe_stream_t stream) {
+    g_last_error.clear();
+    if (T < 0) return fail(MOE_ERR_INVALID_ARG, "T = %d < 0", T);
+    if (E < 1 || E > moe::kMaxExperts) return fail(MOE_ERR_INVALID_ARG, "E = %d outside [1, %d]", E, moe::kMaxExperts);
+    if (k < 1 || k > E) return fail(MOE_ERR_INVALID_ARG, "k = %d outside [1, E = %d]", k, E);
+    if ((long long)T * k > 0x7fffffffLL) return fail(MOE_ERR_INVALID_ARG, "T*k exceeds 2^31-1");
+    if (!out) return fail(MOE_ERR_INVALID_ARG, "out is NULL");
+    if (T > 0 && !topk_idx) return fail(MOE_ERR_INVALID_ARG, "topk_idx is NULL");
+    cudaError_t e = moe::launch_routing_stats(topk_idx, T, E, k, seq_len, out, reinterpret_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? MOE_OK : cuda_fail(e, "routing_stats");
+}
+
 int moe_expert_ffn(const void* x, const void* W1, const void* W3, const void* W2,
                    const int32_t* offsets, const int32_t* perm, const int32_t* inv,
                    const float* topk_w, int T, int d, int f, int E, int k, int dtype,
@@ -298,6 +311,36 @@ int moe_layer_forward_ex(const void* x, const void* Wg, const void* W1, const vo
     if (e != cudaSuccess) return cuda_fail(e, "permute");
     return run_ffn(x, W1, W3, W2, w.offsets, w.perm, w.inv, w.topk_w, residual, T, d, f, E, k, bf16, w,
                    y, s);
+}
+
+int moe_stack_forward(const void* x, const void* const* Wg, const void* const* W1, const void* const* W3,
+                      const void* const* W2, int L, int T, int d, int f, int E, int k, int dtype,
+                      void* scratch, void* workspace, size_t ws_bytes, void* y, moe_stream_t stream) {
+    g_last_error.clear();
+    if (L < 1) return fail(MOE_ERR_INVALID_ARG, "L = %d < 1", L);
+    if (!Wg || !W1 || !W3 || !W2) return fail(MOE_ERR_INVALID_ARG, "per-layer weight arrays must not be NULL");
+    CHECK(check_shape(T, d, f, E, k, dtype, true));
+    if (T == 0) return MOE_OK;
+    CHECK(check_ptr(x, "x"));
+    CHECK(check_ptr(y, "y"));
+    if (L > 1) CHECK(check_ptr(scratch, "scratch"));
+    if (x == y || x == scratch || y == scratch) return fail(MOE_ERR_INVALID_ARG, "x, y and scratch must be distinct");
+    for (int l = 0; l < L; ++l)
+        if (!Wg[l] || !W1[l] || !W3[l] || !W2[l]) return fail(MOE_ERR_INVALID_ARG, "layer %d has a NULL weight", l);
+    // Layer l writes y when (L - 1 - l) is even, else scratch, so the last
+    // layer lands in y and no layer reads the buffer it writes.
+    const void* cur = x;
+    for (int l = 0; l < L; ++l) {
+        void* out = ((L - 1 - l) % 2 == 0) ? y : scratch;
+        const int rc = moe_layer_forward_ex(cur, Wg[l], W1[l], W3[l], W2[l], cur, T, d, f, E, k, dtype, workspace,
+                                            ws_bytes, out, stream);
+        if (rc != MOE_OK) {
+            std::string msg = g_last_error;
+            return fail(rc, "layer %d: %s", l, msg.c_str());
+        }
+        cur = out;
+    }
+    return MOE_OK;
 }
 
 int moe_layer_forward(const void* x, const void* Wg, const void* W1, const void* W3,

@@ -16,7 +16,7 @@ cudaError_t read_clear_device_errors(unsigned int* out);
 void set_last_error(const char* msg);
 
 constexpr int kMaxExperts = 64;
-constexpr int kMaxTopK = 8;
+constexpr int kMaxTopK = kMaxExperts;  // any k <= E
 
 // 256-byte aligned carve-up of one workspace blob.
 struct Workspace {
@@ -42,6 +42,9 @@ cudaError_t launch_gather_rows_bf16(const __nv_bfloat16* x, const int32_t* perm,
                                     int k, __nv_bfloat16* x_perm, cudaStream_t s);
 cudaError_t launch_combine(const float* obuf, const int32_t* inv, const void* residual, int T,
                            int d, int k, bool bf16, void* y, cudaStream_t s);
+
+cudaError_t launch_routing_stats(const int32_t* idx, int T, int E, int k, int seq_len, unsigned int* out,
+                                 cudaStream_t s);
 
 // tcgen05 grouped GEMMs (gemm_sm100.cu)
 struct GroupedGemmArgs {

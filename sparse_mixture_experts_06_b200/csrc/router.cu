@@ -175,9 +175,14 @@ router_topk_kernel(const void* __restrict__ x, const void* __restrict__ Wg, int 
     if (rank != 0 || threadIdx.x >= kTok || !tok_ok) return;
 
     const double* lg = reinterpret_cast<const double*>(sm.wg) + (size_t)threadIdx.x * E;
+    // k rounds of arg-max; indices are written as they are found and the
+    // fp32 softmax numerators exp(l_j - l_0) are parked in w_out, then
+    // divided by their slot-ordered sum (any k <= E, no per-k arrays)
     uint64_t taken = 0;
-    int sel[kMaxTopK];
-    double lsel[kMaxTopK];
+    double l0 = 0.0;
+    float sum = 0.f;
+    int32_t* io = idx_out + (size_t)t * k;
+    float* wo = w_out + (size_t)t * k;
     for (int j = 0; j < k; ++j) {
         int bi = -1;
         double best = 0.0;
@@ -187,19 +192,13 @@ router_topk_kernel(const void* __restrict__ x, const void* __restrict__ Wg, int 
             if (bi < 0 || v > best) { best = v; bi = e; }
         }
         taken |= 1ull << bi;
-        sel[j] = bi;
-        lsel[j] = best;
+        if (j == 0) l0 = best;
+        const float ex = expf((float)(best - l0));
+        io[j] = bi;
+        wo[j] = ex;
+        sum += ex;
     }
-    float ex[kMaxTopK];
-    float sum = 0.f;
-    for (int j = 0; j < k; ++j) {
-        ex[j] = expf((float)(lsel[j] - lsel[0]));
-        sum += ex[j];
-    }
-    for (int j = 0; j < k; ++j) {
-        idx_out[(size_t)t * k + j] = sel[j];
-        w_out[(size_t)t * k + j] = ex[j] / sum;
-    }
+    for (int j = 0; j < k; ++j) wo[j] = wo[j] / sum;
 }
 
 template <bool BF16>

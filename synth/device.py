@@ -54,7 +54,8 @@ def device_inputs(shape: gen.MoEShape, seed: int = 0, layer: int = 0, device="cu
     out["Wg"] = normal_tensor((E, d), seed, gen.tensor_id(gen.TENSOR_WG, layer), gen.sigma_of(gen.TENSOR_WG, d, f), dt, device)
     out["W1"] = normal_tensor((E, f, d), seed, gen.tensor_id(gen.TENSOR_W1, layer), gen.sigma_of(gen.TENSOR_W1, d, f), dt, device)
     out["W3"] = normal_tensor((E, f, d), seed, gen.tensor_id(gen.TENSOR_W3, layer), gen.sigma_of(gen.TENSOR_W3, d, f), dt, device)
-    out["W2"] = normal_tensor((E, d, f), seed, gen.tensor_id(gen.TENSOR_W2, layer), gen.sigma_of(gen.TENSOR_W2, d, f), dt, device)
+    out["W2"] = normal_tensor((E, d, f), seed, gen.tensor_id(gen.TENSOR_W2, layer),
+                              gen.sigma_of(gen.TENSOR_W2, d, f, shape.w2_scale), dt, device)
     if shape.skew:
         beta = gen.SKEW_BETA if skew_beta is None else skew_beta
         b = gen.skew_biases(E, beta, dt)

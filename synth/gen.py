@@ -95,14 +95,16 @@ def normal_values(seed: int, tid: int, count: int, sigma: float, dtype: str,
     return out
 
 
-def sigma_of(kind: int, d: int, f: int) -> float:
-    """Scale of each tensor: x ~ N(0,1); Wg, W1, W3 ~ N(0, 1/d); W2 ~ N(0, 1/f)."""
+def sigma_of(kind: int, d: int, f: int, w2_scale: float = 1.0) -> float:
+    """Scale of each tensor: x ~ N(0,1); Wg, W1, W3 ~ N(0, 1/d); W2 ~ N(0, 1/f)
+    times w2_scale^2 (w2_scale is a power of two, so the fp32 scale stays the
+    exact multiple of the unscaled one)."""
     if kind == TENSOR_X:
         return 1.0
     if kind in (TENSOR_WG, TENSOR_W1, TENSOR_W3):
         return float(np.float32(1.0 / math.sqrt(d)))
     if kind == TENSOR_W2:
-        return float(np.float32(1.0 / math.sqrt(f)))
+        return float(np.float32(w2_scale / math.sqrt(f)))
     raise ValueError(kind)
 
 
@@ -123,6 +125,7 @@ class MoEShape:
     dtype: str          # "bf16" or "f32"
     skew: bool = False  # constant channel + Zipf log-prior in Wg
     layers: int = 1
+    w2_scale: float = 1.0  # W2 ~ N(0, w2_scale^2 / f)
 
     @property
     def flops(self) -> float:
@@ -141,7 +144,12 @@ CONFIGS = {
     "decode": MoEShape("decode", 32, 4096, 14336, 8, 2, "bf16"),
     "prefill": MoEShape("prefill", 4096, 4096, 14336, 8, 2, "bf16"),
     "skewed": MoEShape("skewed", 16384, 4096, 14336, 8, 2, "bf16", skew=True),
-    "stack": MoEShape("stack", 8192, 4096, 14336, 8, 2, "bf16", layers=32),
+    # Residual-only stacking of random SwiGLU layers (no RMSNorm between them,
+    # as the stack workload prescribes) grows the residual stream doubly
+    # exponentially: Var(x_{l+1}) ~ Var(x_l) + Var(x_l)^2 / 4, which
+    # overflows bf16 by layer ~11 at the unscaled W2.  The stack therefore
+    # draws W2 with a 1/4 scale (RMS of x ~1.3 after 32 layers).
+    "stack": MoEShape("stack", 8192, 4096, 14336, 8, 2, "bf16", layers=32, w2_scale=0.25),
 }
 
 
@@ -167,7 +175,7 @@ def host_inputs(shape: MoEShape, seed: int = 0, layer: int = 0, with_x: bool = T
     out["W3"] = normal_values(seed, tensor_id(TENSOR_W3, layer), E * f * d,
                               sigma_of(TENSOR_W3, d, f), dt).reshape(E, f, d)
     out["W2"] = normal_values(seed, tensor_id(TENSOR_W2, layer), E * d * f,
-                              sigma_of(TENSOR_W2, d, f), dt).reshape(E, d, f)
+                              sigma_of(TENSOR_W2, d, f, shape.w2_scale), dt).reshape(E, d, f)
     if shape.skew:
         apply_skew(out, E, SKEW_BETA if skew_beta is None else skew_beta, dt)
     return out

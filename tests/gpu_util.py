@@ -101,3 +101,15 @@ def oracle_rows(h: dict, k: int, tokens, routing=None):
 
 __all__ = ["device_inputs", "host_copy", "check_routing", "check_permutation", "assert_close",
            "stratified_tokens", "oracle_rows", "f64", "TOL"]
+
+
+def assert_residual_close(gpu64, x64, moe_ref, what="x_{l+1}"):
+    """Residual layers: gpu = round_bf16(x + MoE(x)).  Bound: the bf16 layer
+    tolerance on the MoE part, 1e-2 * max|MoE_ref|, plus the final bf16
+    rounding of the sum, 2^-8 |x + MoE_ref| (twice the half-ulp)."""
+    ref = x64 + moe_ref
+    bound = 1e-2 * np.abs(moe_ref).max() + 2.0 ** -8 * np.abs(ref)
+    err = np.abs(gpu64 - ref)
+    assert np.isfinite(gpu64).all(), what + " has non-finite values"
+    assert (err <= bound).all(), "%s: worst excess %.3e" % (what, (err - bound).max())
+    return float((err / np.abs(moe_ref).max()).max())

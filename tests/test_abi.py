@@ -59,7 +59,7 @@ def test_workspace_size(shape, dt):
 
 
 @pytest.mark.parametrize("bad", [dict(T=-1), dict(d=0), dict(d=12), dict(f=100), dict(E=0), dict(E=65),
-                                 dict(k=0), dict(k=9, E=9), dict(dt=7)])
+                                 dict(k=0), dict(k=10, E=9), dict(dt=7)])
 def test_workspace_size_invalid_is_zero(bad):
     a = dict(T=16, d=64, f=128, E=8, k=2, dt=0)
     a.update(bad)
@@ -82,7 +82,8 @@ def test_router_rejects_invalid_arguments():
     assert call_router(T=-3) == 1
     assert call_router(E=0) == 1
     assert call_router(k=3, E=2) == 1
-    assert call_router(k=9, E=16) == 2          # valid for the method, beyond the GPU path: UNSUPPORTED
+    assert call_router(k=17, E=16) == 1         # k > E
+    assert call_router(E=65, k=2) == 1          # more experts than the GPU path holds
     assert call_router(d=60) == 1
     assert call_router(dt=3) == 1
     # T = 0 is a no-op (nothing to launch), even with null pointers
@@ -122,3 +123,21 @@ def test_layer_rejects_invalid_arguments():
     ffn = moe.lib.moe_expert_ffn
     assert ffn(P(16), P(16), P(16), P(16), None, P(16), P(16), P(16), 4, 64, 128, 8, 2, 0, P(256), 10 ** 9,
                P(512), None) == 1   # offsets NULL
+
+
+def test_stack_rejects_invalid_arguments():
+    P = ctypes.c_void_p
+    arr = (ctypes.c_void_p * 2)(16, 16)
+    nul = (ctypes.c_void_p * 2)(16, 0)
+    f = moe.lib.moe_stack_forward
+    base = [P(16), arr, arr, arr, arr, 2, 4, 64, 128, 8, 2, 0, P(256), P(512), 10 ** 9, P(768), None]
+    bad = list(base); bad[5] = 0
+    assert f(*bad) == 1                                   # L < 1
+    bad = list(base); bad[1] = None
+    assert f(*bad) == 1                                   # NULL weight array
+    bad = list(base); bad[2] = nul
+    assert f(*bad) == 1 and "layer 1" in moe.moe_last_error_string()
+    bad = list(base); bad[12] = P(768)
+    assert f(*bad) == 1                                   # scratch aliases y
+    bad = list(base); bad[14] = 100
+    assert f(*bad) == 1 or f(*bad) == 3                   # never launched: fails before or at the workspace check

@@ -67,7 +67,8 @@ def test_device_generator_matches_host(dt):
 
 @pytest.mark.parametrize("T,d,E,k,dt", [
     (16, 64, 8, 2, "f32"), (37, 72, 8, 2, "bf16"), (1, 8, 1, 1, "bf16"), (300, 256, 64, 8, "bf16"),
-    (129, 4096, 8, 2, "bf16"), (250, 96, 5, 3, "f32"),
+    (129, 4096, 8, 2, "bf16"), (250, 96, 5, 3, "f32"), (100, 128, 8, 8, "bf16"), (70, 64, 64, 64, "f32"),
+    (64, 256, 16, 12, "bf16"),
 ])
 def test_router_parity(T, d, E, k, dt):
     t = device_inputs(synth.MoEShape("r", T, d, 8, E, k, dt), seed=T + E)
@@ -112,6 +113,33 @@ def test_permute_flags_bad_expert_ids():
     assert off.cpu().tolist()[-1] == 3 and inv.cpu().tolist()[2] == -1
 
 
+# ---------------------------------------------------------------- routing statistics
+
+@pytest.mark.parametrize("T,E,k,seq_len", [(1, 8, 2, 0), (5000, 8, 2, 0), (4096, 8, 2, 512), (3000, 64, 8, 0),
+                                           (777, 16, 3, 100)])
+def test_routing_stats_parity(T, E, k, seq_len):
+    import oracle
+    rng = np.random.default_rng(T + E)
+    idx = np.stack([rng.permutation(E)[:k] for _ in range(T)]).astype(np.int32)
+    idx[1::7] = idx[0::7][: len(idx[1::7])]          # plant some repeats
+    out = moe.moe_routing_stats(torch.from_numpy(idx).cuda(), E, seq_len)
+    np.testing.assert_array_equal(out.cpu().numpy().astype(np.int64), oracle.routing_stats(idx, E, seq_len))
+
+
+def test_routing_stats_of_the_synthetic_router():
+    """The seeded near-uniform router shows the uniform baselines quoted with
+    tab. 5 (first choice ~1/8, first or second ~13/28)."""
+    import math
+    s = synth.CONFIGS["prefill"]
+    t = device_inputs(synth.MoEShape("st", s.T, s.d, 8, s.E, s.k, "bf16"), 0)
+    idx, _ = moe.moe_router_topk(t["x"], t["Wg"], 2)
+    st = moe.moe_routing_stats(idx, 8).cpu().numpy().astype(np.int64)
+    n = st[10]
+    assert n == s.T - 1 and st[:8].sum() == 2 * s.T
+    assert abs(st[8] / n - 1 / 8) < 4 * math.sqrt(1 / 8 * 7 / 8 / n)
+    assert abs(st[9] / n - 13 / 28) < 4 * math.sqrt(13 / 28 * 15 / 28 / n)
+
+
 # ---------------------------------------------------------------- whole layer, every token
 
 F32_SHAPES = [
@@ -127,6 +155,8 @@ BF16_SHAPES = [
     synth.MoEShape("bf16-E64k8", 256, 128, 128, 64, 8, "bf16"),
     synth.MoEShape("bf16-T1", 1, 64, 128, 8, 2, "bf16"),
     synth.MoEShape("bf16-many-tiles", 2500, 256, 768, 8, 2, "bf16"),  # 625 rows/expert, 2-3 pair tiles
+    synth.MoEShape("bf16-k-eq-E", 150, 128, 256, 8, 8, "bf16"),       # K = E: dense softmax mixture
+    synth.MoEShape("bf16-E16k12", 120, 128, 256, 16, 12, "bf16"),
 ]
 
 

@@ -302,6 +302,33 @@ def test_mixtral_parameter_counts_from_table_1():
     assert abs(total / 1e9 - 46.7) < 0.05 and abs(active / 1e9 - 12.9) < 0.05
 
 
+def test_routing_stats_hand_counted():
+    idx = np.array([[0, 1], [1, 2], [3, 4], [3, 0], [5, 6], [6, 5]])
+    st = oracle.routing_stats(idx, 8)
+    # loads 0:2 1:2 2:1 3:2 4:1 5:2 6:2 7:0; first-choice repeats: (3,3) only;
+    # overlapping pairs: {1,2}&{0,1}, {3,0}&{3,4}, {6,5}&{5,6}; 5 pairs
+    assert st.tolist() == [2, 2, 1, 2, 1, 2, 2, 0, 1, 3, 5]
+    # sequences of 3 tokens: pairs (0,1),(1,2),(3,4),(4,5); the (2,3) pair is dropped
+    st3 = oracle.routing_stats(idx, 8, seq_len=3)
+    assert st3.tolist()[8:] == [0, 2, 4]
+
+
+@pytest.mark.parametrize("E,k", [(8, 2), (8, 1), (16, 3), (4, 2)])
+def test_routing_stats_uniform_closed_forms(E, k):
+    """Uniformly random ordered k-subsets: first choices agree with rate 1/E
+    and kept sets meet with rate 1 - C(E-k, k)/C(E, k)."""
+    rng = np.random.default_rng(E * 10 + k)
+    T = 20000
+    idx = np.stack([rng.permutation(E)[:k] for _ in range(T)])
+    st = oracle.routing_stats(idx, E)
+    n = st[E + 2]
+    p1 = 1.0 / E
+    p2 = 1.0 - math.comb(E - k, k) / math.comb(E, k)
+    assert n == T - 1 and st[:E].sum() == T * k
+    assert abs(st[E] / n - p1) < 4 * math.sqrt(p1 * (1 - p1) / n)
+    assert abs(st[E + 1] / n - p2) < 4 * math.sqrt(p2 * (1 - p2) / n)
+
+
 def test_uniform_routing_baselines_on_synthetic_router():
     """With Wg ~ N(0, 1/d) the synthetic router is close to uniform: the first
     choice repeats on consecutive tokens about 1/8 of the time and the kept
@@ -310,12 +337,12 @@ def test_uniform_routing_baselines_on_synthetic_router():
     s = synth.MoEShape("stat", 4096, 256, 8, 8, 2, "bf16")
     t = synth.host_inputs(s, seed=3, with_experts=False)
     idx, _, _ = oracle.route(synth.bf16_bits_to_f64(t["x"]), synth.bf16_bits_to_f64(t["Wg"]), 2)
-    first = np.mean(idx[1:, 0] == idx[:-1, 0])
-    overlap = np.mean([len(set(a) & set(b)) > 0 for a, b in zip(idx[1:].tolist(), idx[:-1].tolist())])
-    n = len(idx) - 1
+    st = oracle.routing_stats(idx, 8)
+    n = st[10]
+    first, overlap = st[8] / n, st[9] / n
     assert abs(first - 1 / 8) < 4 * math.sqrt(1 / 8 * 7 / 8 / n)
     assert abs(overlap - 13 / 28) < 4 * math.sqrt(13 / 28 * 15 / 28 / n)
-    load = np.bincount(idx.ravel(), minlength=8) / idx.size
+    load = st[:8] / idx.size
     assert np.abs(load - 1 / 8).max() < 0.03
 
 
