@@ -6,9 +6,8 @@
 //  gather_rows      x_perm[r] = x[perm[r] / k]            (bf16 path)
 //  combine_kernel   y[t] = (residual[t] +) sum_j obuf[inv[t*k + j]]
 //
-// The gather and the combine are flat: one thread per 16-byte piece, so
-// every piece's loads are in flight at once (HBM-bound, not latency-bound,
-// for any T).
+// The gather and the combine give each row a block of threads that keep
+// 4 sixteen-byte loads each in flight (HBM-bound, not latency-bound).
 //
 // The scatter is stable and deterministic without global atomics: the
 // assignments are walked in tiles of 1024 in increasing id; inside a warp,
@@ -95,39 +94,40 @@ permute_kernel(const int32_t* __restrict__ idx, int n, int E, int32_t* __restric
 
 constexpr int kFlatThreads = 256;
 
-// One thread per 16-byte piece of x_perm: x_perm[r, 8v..8v+7] = x[perm[r] / k, 8v..8v+7].
-// Each thread handles kUnroll pieces per pass (grid-strided), all loads first.
+// Row kernels: a 256-thread block per row (grid-strided over rows), each
+// thread moving kUnroll 16-byte pieces per pass with all loads issued first.
+// No integer division on the hot path.
 constexpr int kUnroll = 4;
 
+// x_perm[r, :] = x[perm[r] / k, :]  (a row with an invalid assignment id is zero)
 __global__ void __launch_bounds__(kFlatThreads)
 gather_rows_kernel(const __nv_bfloat16* __restrict__ x, const int32_t* __restrict__ perm, int rows,
                    int d, int k, __nv_bfloat16* __restrict__ xp) {
     const int nvec = d / 8;
-    const long long total = (long long)rows * nvec;
-    const long long stride = (long long)gridDim.x * kFlatThreads;
-    for (long long base = (long long)blockIdx.x * kFlatThreads + threadIdx.x; base < total; base += stride * kUnroll) {
-        uint4 val[kUnroll];
-        long long item[kUnroll];
+    for (int r = blockIdx.x; r < rows; r += gridDim.x) {
+        const int q = __ldg(perm + r);
+        const bool ok = (unsigned)q < (unsigned)rows;
+        const uint4* src = reinterpret_cast<const uint4*>(x + (size_t)(ok ? q / k : 0) * d);
+        uint4* dst = reinterpret_cast<uint4*>(xp + (size_t)r * d);
+        for (int v0 = threadIdx.x; v0 < nvec; v0 += kFlatThreads * kUnroll) {
+            uint4 val[kUnroll];
 #pragma unroll
-        for (int u = 0; u < kUnroll; ++u) {
-            item[u] = base + u * stride;
-            val[u] = make_uint4(0, 0, 0, 0);  // (a row with an invalid assignment id stays zero)
-            if (item[u] < total) {
-                const int r = (int)(item[u] / nvec), v = (int)(item[u] - (long long)r * nvec);
-                const int q = __ldg(perm + r);
-                if ((unsigned)q < (unsigned)rows)
-                    val[u] = __ldg(reinterpret_cast<const uint4*>(x + (size_t)(q / k) * d) + v);
+            for (int u = 0; u < kUnroll; ++u) {
+                const int v = v0 + u * kFlatThreads;
+                val[u] = (ok && v < nvec) ? __ldg(src + v) : make_uint4(0, 0, 0, 0);
+            }
+#pragma unroll
+            for (int u = 0; u < kUnroll; ++u) {
+                const int v = v0 + u * kFlatThreads;
+                if (v < nvec) dst[v] = val[u];
             }
         }
-#pragma unroll
-        for (int u = 0; u < kUnroll; ++u)
-            if (item[u] < total) reinterpret_cast<uint4*>(xp)[item[u]] = val[u];
     }
 }
 
-// One thread per 4 output features of one token:
-// y[t, 4v..4v+3] = (residual +) sum_j obuf[inv[t*k + j], 4v..4v+3], slot order.
-// kUnroll pieces per thread per pass, loads first.
+// y[t, :] = (residual[t, :] +) sum_j obuf[inv[t*k + j], :]  (slot order; fp32
+// sum, one rounding to y's dtype).  A slot whose row id is out of range adds
+// nothing.
 template <bool BF16>
 __device__ __forceinline__ void combine_store(const float4& acc0, const void* residual, void* y, int t, int v,
                                               int d) {
@@ -162,40 +162,42 @@ __global__ void __launch_bounds__(kFlatThreads)
 combine_kernel(const float* __restrict__ obuf, const int32_t* __restrict__ inv,
                const void* __restrict__ residual, int T, int d, int k, void* __restrict__ y) {
     const int nvec = d / 4;
-    const long long total = (long long)T * nvec;
     const unsigned n = (unsigned)(T * k);
-    const long long stride = (long long)gridDim.x * kFlatThreads;
-    for (long long base = (long long)blockIdx.x * kFlatThreads + threadIdx.x; base < total; base += stride * kUnroll) {
-        float4 acc[kUnroll];
+    for (int t = blockIdx.x; t < T; t += gridDim.x) {
+        for (int v0 = threadIdx.x; v0 < nvec; v0 += kFlatThreads * kUnroll) {
+            float4 acc[kUnroll];
 #pragma unroll
-        for (int u = 0; u < kUnroll; ++u) {
-            acc[u] = make_float4(0.f, 0.f, 0.f, 0.f);
-            const long long it = base + u * stride;
-            if (it >= total) continue;
-            const int t = (int)(it / nvec), v = (int)(it - (long long)t * nvec);
+            for (int u = 0; u < kUnroll; ++u) acc[u] = make_float4(0.f, 0.f, 0.f, 0.f);
             for (int j = 0; j < k; ++j) {
                 const int r = __ldg(inv + (size_t)t * k + j);
                 if ((unsigned)r >= n) continue;  // unrouted slot adds nothing
-                const float4 o = __ldg(reinterpret_cast<const float4*>(obuf + (size_t)r * d) + v);
-                if (j == 0) {
-                    acc[u] = o;
-                } else {
-                    acc[u].x += o.x; acc[u].y += o.y; acc[u].z += o.z; acc[u].w += o.w;
+                const float4* row = reinterpret_cast<const float4*>(obuf + (size_t)r * d);
+                float4 o[kUnroll];
+#pragma unroll
+                for (int u = 0; u < kUnroll; ++u) {
+                    const int v = v0 + u * kFlatThreads;
+                    o[u] = (v < nvec) ? __ldg(row + v) : make_float4(0.f, 0.f, 0.f, 0.f);
+                }
+#pragma unroll
+                for (int u = 0; u < kUnroll; ++u) {
+                    if (j == 0) {
+                        acc[u] = o[u];
+                    } else {
+                        acc[u].x += o[u].x; acc[u].y += o[u].y; acc[u].z += o[u].z; acc[u].w += o[u].w;
+                    }
                 }
             }
-        }
 #pragma unroll
-        for (int u = 0; u < kUnroll; ++u) {
-            const long long it = base + u * stride;
-            if (it >= total) continue;
-            const int t = (int)(it / nvec), v = (int)(it - (long long)t * nvec);
-            combine_store<BF16>(acc[u], residual, y, t, v, d);
+            for (int u = 0; u < kUnroll; ++u) {
+                const int v = v0 + u * kFlatThreads;
+                if (v < nvec) combine_store<BF16>(acc[u], residual, y, t, v, d);
+            }
         }
     }
 }
 
-// Grid for a flat kernel over `items` threads: enough blocks for all of them,
-// capped at 8 resident blocks per SM (the kernels loop with a grid stride).
+// Grid for a row kernel over `items` rows: one block per row, capped at 8
+// resident blocks per SM (the kernels loop with a grid stride).
 int flat_grid(long long items) {
     static int sms_cache[64] = {0};
     int dev = 0;
@@ -206,7 +208,7 @@ int flat_grid(long long items) {
         if (sms <= 0) sms = 148;
         if (dev < 64) sms_cache[dev] = sms;
     }
-    const long long need = (items + kFlatThreads * kUnroll - 1) / (kFlatThreads * kUnroll);
+    const long long need = items;
     const long long cap = (long long)sms * 8;
     return (int)(need < cap ? (need > 0 ? need : 1) : cap);
 }
@@ -239,16 +241,16 @@ cudaError_t launch_permute(const int32_t* idx, int n, int E, int32_t* offsets, i
 
 cudaError_t launch_gather_rows_bf16(const __nv_bfloat16* x, const int32_t* perm, int rows, int d,
                                     int k, __nv_bfloat16* x_perm, cudaStream_t s) {
-    gather_rows_kernel<<<flat_grid((long long)rows * (d / 8)), kFlatThreads, 0, s>>>(x, perm, rows, d, k, x_perm);
+    gather_rows_kernel<<<flat_grid(rows), kFlatThreads, 0, s>>>(x, perm, rows, d, k, x_perm);
     return cudaGetLastError();
 }
 
 cudaError_t launch_combine(const float* obuf, const int32_t* inv, const void* residual, int T,
                            int d, int k, bool bf16, void* y, cudaStream_t s) {
     if (bf16)
-        combine_kernel<true><<<flat_grid((long long)T * (d / 4)), kFlatThreads, 0, s>>>(obuf, inv, residual, T, d, k, y);
+        combine_kernel<true><<<flat_grid(T), kFlatThreads, 0, s>>>(obuf, inv, residual, T, d, k, y);
     else
-        combine_kernel<false><<<flat_grid((long long)T * (d / 4)), kFlatThreads, 0, s>>>(obuf, inv, residual, T, d, k, y);
+        combine_kernel<false><<<flat_grid(T), kFlatThreads, 0, s>>>(obuf, inv, residual, T, d, k, y);
     return cudaGetLastError();
 }
 

@@ -6,10 +6,9 @@
 // the expert choice agrees with that of the exact logits except inside
 // ~1e-13 relative near-ties.
 //
-// Work split: a thread-block cluster of 8 CTAs serves a group of 32 tokens.
-// CTA r of the cluster takes the r-th eighth of the d features; inside it
-// each lane owns one token (lane = token) and the 8 warps split the CTA's
-// features.  The router weight slice is widened to fp64 once per CTA and
+// Work split: a thread-block cluster of 8 CTAs serves a group of 32 tokens.  CTA r of the cluster takes the r-th
+// share of the d features; inside it each lane owns one token (lane =
+// token) and the 8 warps split the CTA's features.  The router weight slice is widened to fp64 once per CTA and
 // kept in shared memory as [feature][expert], so every lane reads the 8
 // expert weights of a feature with four broadcast 16-byte loads and the
 // fp64 conversions are paid once per weight, not once per product.  Each
@@ -17,11 +16,12 @@
 //
 // Reduction (fixed order, so the result is deterministic): each lane sums
 // its features in increasing order; the 8 warps' partials are added in warp
-// order in shared memory; CTA 0 of the cluster adds the 8 CTAs' partials in
+// order in shared memory; CTA 0 of the cluster adds the CTAs' partials in
 // rank order through distributed shared memory, then one thread per token
 // does the top-k (k rounds of a strict-greater arg-max in increasing expert
 // order, so an exact tie keeps the lower index; slot 0 = largest) and the
-// fp32 softmax of the kept logits.
+// fp32 softmax of the kept logits.  The cluster size changes the summation
+// order but not the rule: logits are fp64 sums of exact products.
 
 #include <cooperative_groups.h>
 
@@ -32,7 +32,7 @@ namespace cg = cooperative_groups;
 namespace moe {
 namespace {
 
-constexpr int kCluster = 8;        // CTAs per token group (d split 8 ways)
+constexpr int kMaxCluster = 8;     // CTAs per token group (d split up to 8 ways)
 constexpr int kWarps = 8;          // warps per CTA
 constexpr int kTok = 32;           // tokens per group (one per lane)
 constexpr int kChunk = 512;        // features staged per pass (512 x 8 experts x 8 B = 32 KiB)
@@ -82,21 +82,22 @@ __device__ __forceinline__ double load_w(const void* Wg, size_t idx) {
 }
 
 template <bool BF16>
-__global__ void __cluster_dims__(kCluster, 1, 1) __launch_bounds__(kWarps * 32)
+__global__ void __launch_bounds__(kWarps * 32)
 router_topk_kernel(const void* __restrict__ x, const void* __restrict__ Wg, int T, int d, int E, int k,
                    int32_t* __restrict__ idx_out, float* __restrict__ w_out) {
     extern __shared__ __align__(16) unsigned char smem_raw[];
     RouterSmem& sm = *reinterpret_cast<RouterSmem*>(smem_raw);
     cg::cluster_group cluster = cg::this_cluster();
     const int rank = (int)cluster.block_rank();
+    const int nranks = (int)cluster.num_blocks();
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int group = blockIdx.x / kCluster;  // clusters tile grid.x
+    const int group = blockIdx.x / nranks;  // clusters tile grid.x
     const int t = group * kTok + lane;
     const bool tok_ok = t < T;
     const void* xr = reinterpret_cast<const char*>(x) + (size_t)(tok_ok ? t : 0) * d * (BF16 ? 2 : 4);
 
     // this CTA's feature range (multiples of 8)
-    const int slice = ((d + kCluster * 8 - 1) / (kCluster * 8)) * 8;
+    const int slice = ((d + nranks * 8 - 1) / (nranks * 8)) * 8;
     const int f0 = min(d, rank * slice), f1 = min(d, f0 + slice);
 
     for (int eg = 0; eg < E; eg += 8) {
@@ -164,7 +165,7 @@ router_topk_kernel(const void* __restrict__ x, const void* __restrict__ Wg, int 
         for (int i = threadIdx.x; i < kTok * E; i += kWarps * 32) {
             const int tk = i / E, e = i - tk * E;
             double s = 0.0;
-            for (int r = 0; r < kCluster; ++r) {
+            for (int r = 0; r < nranks; ++r) {
                 const RouterSmem* peer = cluster.map_shared_rank(&sm, r);
                 s += peer->part[tk][e];
             }
@@ -213,9 +214,22 @@ cudaError_t launch_impl(const void* x, const void* Wg, int T, int d, int E, int 
         if (e != cudaSuccess) return e;
         attr_done[dev] = true;
     }
-    const dim3 grid(kCluster * ((T + kTok - 1) / kTok));
-    router_topk_kernel<BF16><<<grid, kWarps * 32, smem, s>>>(x, Wg, T, d, E, k, idx, w);
-    return cudaGetLastError();
+    // d is split 8 ways (a 4-way split, with half the CTAs, measured slower
+    // at T = 4096 on B200).
+    const int nranks = kMaxCluster;
+    cudaLaunchConfig_t cfg = {};
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = nranks;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.gridDim = dim3(nranks * ((T + kTok - 1) / kTok));
+    cfg.blockDim = dim3(kWarps * 32);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, router_topk_kernel<BF16>, x, Wg, T, d, E, k, idx, w);
 }
 
 }  // namespace
