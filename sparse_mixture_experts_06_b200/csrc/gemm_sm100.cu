@@ -50,19 +50,11 @@ namespace {
 constexpr int BM = 128;            // tile rows (permuted tokens)
 constexpr int BK = 64;             // k per stage: 64 bf16 = one 128-byte swizzle row
 constexpr int UMMA_K = 16;         // k per tcgen05.mma (kind::f16)
-constexpr int MMA_N = 256;         // accumulator columns per tile
 constexpr int A_TILE = BM * BK * 2;            // 16 KiB: 128 rows x 64 k
-constexpr int B_HALF = 128 * BK * 2;           // 16 KiB: 128 rows x 64 k
 constexpr int NUM_THREADS = 192;
 constexpr int TMEM_COLS = 512;                 // 2 accumulators x 256 fp32 columns
 constexpr unsigned long long kTimeoutNs = 4000000000ull;
 
-// Instruction descriptor (kind::f16): D fp32 (bits 4-5 = 1), A and B bf16
-// (bits 7-9 = 1, 10-12 = 1), both K-major (bits 15, 16 = 0),
-// N >> 3 in bits 17-22, M >> 4 in bits 24-28.  This one: M = 128 (single CTA);
-// the pair variant's (M = 256) is Cfg<2>::kIdesc.
-constexpr uint32_t kIdesc = (1u << 4) | (1u << 7) | (1u << 10) |
-                            ((uint32_t)(MMA_N >> 3) << 17) | ((uint32_t)(BM >> 4) << 24);
 
 enum Mode { kUp = 0, kDown = 1 };
 
@@ -137,12 +129,12 @@ __device__ __forceinline__ uint64_t sw128_desc(uint32_t saddr) {
            ((uint64_t)(1024 >> 4) << 32) | ((uint64_t)1 << 46) | ((uint64_t)2 << 61);
 }
 
-__device__ __forceinline__ void umma_bf16(uint32_t d_tmem, uint64_t a, uint64_t b, uint32_t acc) {
+__device__ __forceinline__ void umma_bf16(uint32_t d_tmem, uint64_t a, uint64_t b, uint32_t idesc, uint32_t acc) {
     asm volatile(
         "{\n\t.reg .pred p;\n\t"
         "setp.ne.b32 p, %4, 0;\n\t"
         "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}\n" ::"r"(d_tmem),
-        "l"(a), "l"(b), "r"(kIdesc), "r"(acc));
+        "l"(a), "l"(b), "r"(idesc), "r"(acc));
 }
 
 __device__ __forceinline__ void umma_commit(uint32_t bar) {
@@ -270,22 +262,35 @@ constexpr int kOutBoxBytes = 32 * 128;
 constexpr int kOutBytes = 4 * 2 * kOutBoxBytes;
 
 // ---------------------------------------------------------------------------
-// Per-variant constants.  CG = 1: one CTA per 128-row tile, B tile of 256
-// rows in its own shared memory.  CG = 2: a CTA pair per 256-row tile; each
-// CTA holds its 128 rows of A and its 128-row half of B; the even CTA issues
+// Per-variant constants.  BN = accumulator columns of a tile (the MMA's N):
+// 256 or 128.  CG = 1: one CTA per 128-row tile, the whole BN-row B tile in
+// its own shared memory.  CG = 2: a CTA pair per 256-row tile; each CTA
+// holds its 128 rows of A and its BN/2-row half of B; the even CTA issues
 // M = 256 MMAs that read both CTAs' shared memory and write both CTAs' TMEM.
+// The stage ring fills 192 KiB of shared memory.
+//
+// Instruction descriptor (kind::f16): D fp32 (bits 4-5 = 1), A and B bf16
+// (bits 7-9 = 1, 10-12 = 1), both K-major (bits 15, 16 = 0), N >> 3 in
+// bits 17-22, M >> 4 in bits 24-28.
 
-template <int CG>
+template <int CG, int BN, int RB>
 struct Cfg {
-    static constexpr int kTileRows = 128 * CG;               // rows of one tile (pair)
-    static constexpr int kBRows = (CG == 1) ? 256 : 128;     // B rows held by one CTA
+    // RB (single CTA only): token rows loaded per tile, 128 or 32.  With 32
+    // the TMA fills only the first 32 rows of the 128-row A buffer; the MMA
+    // still computes 128 rows, and rows 32..127 (stale shared memory) give
+    // accumulator rows that are never stored: row i of the product depends
+    // on row i of A alone.  For decode, where experts hold a few rows each.
+    static_assert(CG == 1 || RB == 128, "pairs load 128 rows per CTA");
+    static constexpr int kTileRows = (CG == 1) ? RB : 256;   // rows of one tile (pair)
+    static constexpr int kABytes = ((CG == 1) ? RB : 128) * BK * 2;  // A bytes loaded per stage
+    static constexpr int kBRows = (CG == 1) ? BN : BN / 2;   // B rows held by one CTA
+    static constexpr int kBHalf = (BN / 2) * BK * 2;         // bytes of BN/2 rows of B
     static constexpr int kBBytes = kBRows * BK * 2;
-    static constexpr int kStageBytes = A_TILE + kBBytes;     // per CTA
-    static constexpr int kStages = (CG == 1) ? 4 : 6;
+    static constexpr int kStageBytes = A_TILE + kBBytes;     // per CTA (A buffer always 128 rows)
+    static constexpr int kStages = (196608 / kStageBytes) > 8 ? 8 : (196608 / kStageBytes);
     static constexpr int kSmem = 1024 + kStages * kStageBytes + kOutBytes + 1024;
-    static constexpr uint32_t kIdescM = (uint32_t)((128 * CG) >> 4) << 24;
-    static constexpr uint32_t kIdesc = (1u << 4) | (1u << 7) | (1u << 10) |
-                                       ((uint32_t)(MMA_N >> 3) << 17) | kIdescM;
+    static constexpr uint32_t kIdesc = (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(BN >> 3) << 17) |
+                                       ((uint32_t)((128 * CG) >> 4) << 24);
 };
 
 __device__ __forceinline__ int count_tiles_rows(const int* s_off, int E, int n_tiles, int rows_per_tile) {
@@ -328,12 +333,12 @@ __device__ __noinline__ bool wait_bounded_pair(uint32_t bar, uint32_t parity, vo
     }
 }
 
-template <int MODE, int CG>
+template <int MODE, int CG, int BN, int RB>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
 grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB0,
                     const __grid_constant__ CUtensorMap tmB1, const __grid_constant__ CUtensorMap tmOut,
                     const KParams p) {
-    using C = Cfg<CG>;
+    using C = Cfg<CG, BN, RB>;
     constexpr int STG = C::kStages;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -400,14 +405,14 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
                 int rowB0, rowB1;
                 const CUtensorMap* mapB = &tmB0;
                 if constexpr (CG == 1) {
-                    rowB0 = e * p.b_rows_per_expert + nb * (MODE == kUp ? 128 : 256);
-                    rowB1 = (MODE == kUp) ? rowB0 : rowB0 + 128;
+                    rowB0 = e * p.b_rows_per_expert + nb * (MODE == kUp ? BN / 2 : BN);
+                    rowB1 = (MODE == kUp) ? rowB0 : rowB0 + BN / 2;
                 } else {
                     if constexpr (MODE == kUp) {
-                        rowB0 = e * p.b_rows_per_expert + nb * 128;   // W1 rows (even CTA) or W3 rows (odd CTA)
+                        rowB0 = e * p.b_rows_per_expert + nb * (BN / 2);  // W1 rows (even CTA) or W3 rows (odd CTA)
                         if (rank == 1) mapB = &tmB1;
                     } else {
-                        rowB0 = e * p.b_rows_per_expert + nb * 256 + (int)rank * 128;
+                        rowB0 = e * p.b_rows_per_expert + nb * BN + (int)rank * (BN / 2);
                     }
                     rowB1 = rowB0;
                 }
@@ -417,10 +422,10 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
                     if (!wait_bounded_pair(smem_u32(&empty[s]), ph ^ 1u, abort_flag, p.err, peer_abort)) { ok = false; break; }
                     const uint32_t fb = smem_u32(&full[s]);
                     if constexpr (CG == 1) {
-                        mbar_arrive_expect_tx(fb, C::kStageBytes);
+                        mbar_arrive_expect_tx(fb, C::kABytes + C::kBBytes);
                         tma_load_2d(smem_u32(sA + s * A_TILE), &tmA, fb, kb * BK, rowA);
                         tma_load_2d(smem_u32(sB + s * C::kBBytes), &tmB0, fb, kb * BK, rowB0);
-                        tma_load_2d(smem_u32(sB + s * C::kBBytes + B_HALF), &tmB1, fb, kb * BK, rowB1);
+                        tma_load_2d(smem_u32(sB + s * C::kBBytes + C::kBHalf), &tmB1, fb, kb * BK, rowB1);
                     } else {
                         if (leader) mbar_arrive_expect_tx(fb, 2 * C::kStageBytes);  // both CTAs' bytes
                         tma_load_2d_pair(smem_u32(sA + s * A_TILE), &tmA, fb, kb * BK, rowA);
@@ -451,7 +456,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
                 const uint32_t use = tcount >> 1;
                 if (!wait_bounded_pair(smem_u32(&tempty[acc]), (use & 1u) ^ 1u, abort_flag, p.err, peer_abort)) break;
                 tc_fence_after();
-                const uint32_t d_tmem = tmem_base + acc * MMA_N;
+                const uint32_t d_tmem = tmem_base + acc * BN;
                 for (int kb = 0; kb < kblocks; ++kb, ++it) {
                     const uint32_t s = it % STG;
                     const uint32_t ph = (it / STG) & 1u;
@@ -463,7 +468,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
                     for (int kk = 0; kk < BK / UMMA_K; ++kk) {
                         // advance 16 bf16 = 32 bytes along K inside the swizzle row
                         if constexpr (CG == 1)
-                            umma_bf16(d_tmem, adesc + (uint64_t)(kk * 2), bdesc + (uint64_t)(kk * 2),
+                            umma_bf16(d_tmem, adesc + (uint64_t)(kk * 2), bdesc + (uint64_t)(kk * 2), C::kIdesc,
                                       (kb | kk) != 0 ? 1u : 0u);
                         else
                             umma_bf16_pair(d_tmem, adesc + (uint64_t)(kk * 2), bdesc + (uint64_t)(kk * 2), C::kIdesc,
@@ -497,18 +502,19 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
             if (!__all_sync(0xffffffffu, okw)) break;
             tc_fence_after();
             const int row = s_off[e] + mb * C::kTileRows + r_in;
-            const bool valid = row < s_off[e + 1];
+            const int tile_end = min(s_off[e + 1], s_off[e] + (mb + 1) * C::kTileRows);
+            const bool valid = row < tile_end;
             // rows of this warp: whole box stored by TMA when all 32 are the
             // expert's own; a box straddling the end of the expert's block
             // uses per-row stores (a full-box store would overwrite the next
             // expert's rows)
             const int wrow0 = row - lane;
-            const bool box_ok = wrow0 + 32 <= s_off[e + 1];
-            const uint32_t tacc = t_lane + acc * MMA_N;
+            const bool box_ok = wrow0 + 32 <= tile_end;
+            const uint32_t tacc = t_lane + acc * BN;
             if constexpr (MODE == kUp) {
                 __nv_bfloat16* hrow = p.h + (size_t)row * p.n_out;
 #pragma unroll 1
-                for (int c64 = 0; c64 < 128; c64 += 64, ++obox) {
+                for (int c64 = 0; c64 < BN / 2; c64 += 64, ++obox) {
                     const uint32_t buf = out_base + (obox & 1u) * kOutBoxBytes;
                     if (box_ok) {
                         if (lane == 0) bulk_wait_read_le1();  // this buffer's previous store has read it
@@ -519,7 +525,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
                         const int c = c64 + half * 32;
                         uint32_t a[32], b[32];
                         tmem_ld32(tacc + c, a);
-                        tmem_ld32(tacc + 128 + c, b);
+                        tmem_ld32(tacc + BN / 2 + c, b);
                         tmem_wait_ld();
                         uint4 pk[4];
 #pragma unroll
@@ -538,7 +544,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
                             for (int g = 0; g < 4; ++g)
                                 st_shared_v4(buf + lane * 128 + ((((half * 4 + g) ^ (lane & 7))) << 4), pk[g]);
                         } else if (valid) {
-                            const int col0 = nb * 128 + c;
+                            const int col0 = nb * (BN / 2) + c;
 #pragma unroll
                             for (int g = 0; g < 4; ++g)
                                 if (col0 + g * 8 < p.n_out) *reinterpret_cast<uint4*>(hrow + col0 + g * 8) = pk[g];
@@ -550,7 +556,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
                         if (lane == 0) {
                             // a box wholly past the last column is not stored; the
                             // (empty) group keeps one group per staged box
-                            if (nb * 128 + c64 < p.n_out) tma_store_2d(&tmOut, buf, nb * 128 + c64, wrow0);
+                            if (nb * (BN / 2) + c64 < p.n_out) tma_store_2d(&tmOut, buf, nb * (BN / 2) + c64, wrow0);
                             bulk_commit();
                         }
                     }
@@ -563,7 +569,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
                 }
                 float* orow = p.obuf + (size_t)row * p.n_out;
 #pragma unroll 1
-                for (int c = 0; c < MMA_N; c += 32, ++obox) {
+                for (int c = 0; c < BN; c += 32, ++obox) {
                     const uint32_t buf = out_base + (obox & 1u) * kOutBoxBytes;
                     if (box_ok) {
                         if (lane == 0) bulk_wait_read_le1();
@@ -586,11 +592,11 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
                         fence_proxy_async_smem();
                         __syncwarp();
                         if (lane == 0) {
-                            if (nb * 256 + c < p.n_out) tma_store_2d(&tmOut, buf, nb * 256 + c, wrow0);
+                            if (nb * BN + c < p.n_out) tma_store_2d(&tmOut, buf, nb * BN + c, wrow0);
                             bulk_commit();
                         }
                     } else if (valid) {
-                        const int col0 = nb * 256 + c;
+                        const int col0 = nb * BN + c;
 #pragma unroll
                         for (int g = 0; g < 8; ++g)
                             if (col0 + g * 4 < p.n_out) *reinterpret_cast<uint4*>(orow + col0 + g * 4) = v[g];
@@ -657,10 +663,10 @@ bool make_map(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols, ui
 
 // Co-resident persistent grid: CTAs (CG = 1) or CTA pairs (CG = 2) that
 // fit on the device at once, capped by an upper bound on the tile count.
-template <int MODE, int CG>
+template <int MODE, int CG, int BN, int RB>
 cudaError_t launch_gemm(const GroupedGemmArgs& a, const CUtensorMap& mA, const CUtensorMap& mB0,
                         const CUtensorMap& mB1, const CUtensorMap& mOut, const KParams& p, cudaStream_t s) {
-    using C = Cfg<CG>;
+    using C = Cfg<CG, BN, RB>;
     static int units_cache[64] = {0};
     int dev = 0;
     cudaGetDevice(&dev);
@@ -680,14 +686,14 @@ cudaError_t launch_gemm(const GroupedGemmArgs& a, const CUtensorMap& mA, const C
         cfg.numAttrs = 1;
     }
     if (!units) {
-        cudaError_t e = cudaFuncSetAttribute(grouped_gemm_kernel<MODE, CG>,
+        cudaError_t e = cudaFuncSetAttribute(grouped_gemm_kernel<MODE, CG, BN, RB>,
                                              cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmem);
         if (e != cudaSuccess) return e;
         units = a.num_sms / CG;
         if (CG == 2) {
             int clusters = 0;
             cfg.gridDim = dim3(2 * units);
-            if (cudaOccupancyMaxActiveClusters(&clusters, grouped_gemm_kernel<MODE, CG>, &cfg) == cudaSuccess &&
+            if (cudaOccupancyMaxActiveClusters(&clusters, grouped_gemm_kernel<MODE, CG, BN, RB>, &cfg) == cudaSuccess &&
                 clusters > 0 && clusters < units)
                 units = clusters;
             cudaGetLastError();  // an unsupported query is not an error for the launch
@@ -698,7 +704,7 @@ cudaError_t launch_gemm(const GroupedGemmArgs& a, const CUtensorMap& mA, const C
     const int grid_units = (int)(ub < units ? ub : units);
     if (grid_units <= 0) return cudaSuccess;
     cfg.gridDim = dim3(grid_units * CG);
-    return cudaLaunchKernelEx(&cfg, grouped_gemm_kernel<MODE, CG>, mA, mB0, mB1, mOut, p);
+    return cudaLaunchKernelEx(&cfg, grouped_gemm_kernel<MODE, CG, BN, RB>, mA, mB0, mB1, mOut, p);
 }
 
 // CTA-pair tiles (M = 256) move a third fewer bytes per MMA from L2 but pad
@@ -723,28 +729,67 @@ const char* gemm_init_error() {
     return g_init_err;
 }
 
+namespace {
+
+// N width of the up-projection tiles: 256 (128 hidden units of W1 and of
+// W3).  128-wide tiles (64 + 64) exist for finer load balance, but measured
+// on B200 at decode (T = 32) they were slower (0.336 vs 0.323 ms): twice the
+// tiles cost more per-tile work than the shorter last wave saves.
+// MOE_GEMM_BN = 128 selects them (exact; the tests run both widths).
+int choose_up_bn(const GroupedGemmArgs&) {
+    if (const char* env = getenv("MOE_GEMM_BN")) {
+        if (env[0] == '1') return 128;
+    }
+    return 256;
+}
+
+// Token rows per single-CTA tile: 32 when experts average at most 16 rows
+// (decode), so tiles do not stream 128 mostly unused A rows from L2 for every
+// weight tile; 128 otherwise.  MOE_GEMM_RB = 32 or 128 forces it.
+int choose_rb(const GroupedGemmArgs& a) {
+    if (const char* env = getenv("MOE_GEMM_RB")) {
+        if (env[0] == '3') return 32;
+        if (env[0] == '1') return 128;
+    }
+    return a.rows <= 16 * a.E ? 32 : 128;
+}
+
+template <int MODE, int BN>
+cudaError_t launch_variant(const GroupedGemmArgs& a, const CUtensorMap& mA, const CUtensorMap& mA32,
+                           const CUtensorMap& mB0, const CUtensorMap& mB1, const CUtensorMap& mOut, const KParams& p,
+                           cudaStream_t s) {
+    if (choose_cta_group(a, MODE) == 2) return launch_gemm<MODE, 2, BN, 128>(a, mA, mB0, mB1, mOut, p, s);
+    return choose_rb(a) == 32 ? launch_gemm<MODE, 1, BN, 32>(a, mA32, mB0, mB1, mOut, p, s)
+                              : launch_gemm<MODE, 1, BN, 128>(a, mA, mB0, mB1, mOut, p, s);
+}
+
+}  // namespace
+
 cudaError_t launch_up_swiglu(const GroupedGemmArgs& a, const __nv_bfloat16* x_perm,
                              const __nv_bfloat16* W1, const __nv_bfloat16* W3, __nv_bfloat16* h,
                              cudaStream_t s) {
-    CUtensorMap mA, mB0, mB1, mOut;
+    const int bn = choose_up_bn(a);
+    CUtensorMap mA, mA32, mB0, mB1, mOut;
     if (!make_map(&mA, x_perm, (uint64_t)a.rows, (uint64_t)a.d, BM) ||
-        !make_map(&mB0, W1, (uint64_t)a.E * a.f, (uint64_t)a.d, 128) ||
-        !make_map(&mB1, W3, (uint64_t)a.E * a.f, (uint64_t)a.d, 128) ||
+        !make_map(&mA32, x_perm, (uint64_t)a.rows, (uint64_t)a.d, 32) ||
+        !make_map(&mB0, W1, (uint64_t)a.E * a.f, (uint64_t)a.d, bn / 2) ||
+        !make_map(&mB1, W3, (uint64_t)a.E * a.f, (uint64_t)a.d, bn / 2) ||
         !make_map(&mOut, h, (uint64_t)a.rows, (uint64_t)a.f, 32))
         return cudaErrorInvalidValue;
     KParams p{};
     p.offsets = a.offsets; p.E = a.E; p.n_out = a.f; p.Kdim = a.d;
-    p.n_tiles = (a.f + 127) / 128; p.b_rows_per_expert = a.f; p.h = h; p.rows = a.rows;
+    p.n_tiles = (a.f + bn / 2 - 1) / (bn / 2); p.b_rows_per_expert = a.f; p.h = h; p.rows = a.rows;
     p.err = a.err;
-    return choose_cta_group(a, kUp) == 2 ? launch_gemm<kUp, 2>(a, mA, mB0, mB1, mOut, p, s)
-                                    : launch_gemm<kUp, 1>(a, mA, mB0, mB1, mOut, p, s);
+    return bn == 128 ? launch_variant<kUp, 128>(a, mA, mA32, mB0, mB1, mOut, p, s)
+                     : launch_variant<kUp, 256>(a, mA, mA32, mB0, mB1, mOut, p, s);
 }
 
 cudaError_t launch_down_scaled(const GroupedGemmArgs& a, const __nv_bfloat16* h,
                                const __nv_bfloat16* W2, const int32_t* perm, const float* topk_w,
                                float* obuf, cudaStream_t s) {
-    CUtensorMap mA, mB, mOut;
+    CUtensorMap mA, mA32, mB, mOut;
     if (!make_map(&mA, h, (uint64_t)a.rows, (uint64_t)a.f, BM) ||
+        !make_map(&mA32, h, (uint64_t)a.rows, (uint64_t)a.f, 32) ||
         !make_map(&mB, W2, (uint64_t)a.E * a.d, (uint64_t)a.f, 128) ||
         !make_map(&mOut, obuf, (uint64_t)a.rows, (uint64_t)a.d, 32, true))
         return cudaErrorInvalidValue;
@@ -753,8 +798,7 @@ cudaError_t launch_down_scaled(const GroupedGemmArgs& a, const __nv_bfloat16* h,
     p.n_tiles = (a.d + 255) / 256; p.b_rows_per_expert = a.d;
     p.perm = perm; p.topk_w = topk_w; p.obuf = obuf; p.rows = a.rows;
     p.err = a.err;
-    return choose_cta_group(a, kDown) == 2 ? launch_gemm<kDown, 2>(a, mA, mB, mB, mOut, p, s)
-                                    : launch_gemm<kDown, 1>(a, mA, mB, mB, mOut, p, s);
+    return launch_variant<kDown, 256>(a, mA, mA32, mB, mB, mOut, p, s);
 }
 
 }  // namespace moe

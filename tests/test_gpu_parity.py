@@ -166,11 +166,19 @@ def test_layer_parity_every_token_f32(shape):
     assert rel <= 1e-5
 
 
-@pytest.mark.parametrize("cta_group", ["1", "2"])
+GEMM_VARIANTS = [("1", "256", "128"), ("1", "128", "128"), ("1", "256", "32"), ("1", "128", "32"),
+                 ("2", "256", "128"), ("2", "128", "128")]
+
+
+@pytest.mark.parametrize("variant", GEMM_VARIANTS, ids=lambda v: "cg%s-bn%s-rb%s" % v)
 @pytest.mark.parametrize("shape", BF16_SHAPES, ids=lambda s: s.name)
-def test_layer_parity_every_token_bf16(shape, cta_group, monkeypatch):
-    """Both GEMM variants (single-CTA 128-row tiles, CTA-pair 256-row tiles)."""
+def test_layer_parity_every_token_bf16(shape, variant, monkeypatch):
+    """Every GEMM variant: single-CTA tiles of 128 or 32 token rows, CTA-pair
+    256-row tiles, and 256- or 128-column up-projection tiles."""
+    cta_group, bn, rb = variant
     monkeypatch.setenv("MOE_GEMM_CTA_GROUP", cta_group)
+    monkeypatch.setenv("MOE_GEMM_BN", bn)
+    monkeypatch.setenv("MOE_GEMM_RB", rb)
     rel, _ = full_check(shape)
     assert rel <= 1e-2
 
@@ -320,10 +328,14 @@ def test_prefill_full_shape(mixtral_weights):
     big_check("prefill", mixtral_weights, 256)
 
 
-@pytest.mark.parametrize("name,cta_group", [("decode", "2"), ("prefill", "1")])
-def test_full_shapes_other_gemm_variant(name, cta_group, mixtral_weights, monkeypatch):
-    """The variant the size heuristic does not pick, at the full shapes."""
+@pytest.mark.parametrize("name,cta_group,bn,rb", [("decode", "2", "256", "128"), ("decode", "1", "256", "128"),
+                                                  ("prefill", "1", "128", "128"), ("prefill", "2", "256", "128"),
+                                                  ("prefill", "1", "256", "32")])
+def test_full_shapes_other_gemm_variant(name, cta_group, bn, rb, mixtral_weights, monkeypatch):
+    """Variants the size heuristics do not pick, at the full shapes."""
     monkeypatch.setenv("MOE_GEMM_CTA_GROUP", cta_group)
+    monkeypatch.setenv("MOE_GEMM_BN", bn)
+    monkeypatch.setenv("MOE_GEMM_RB", rb)
     big_check(name, mixtral_weights, None if name == "decode" else 256)
 
 
