@@ -316,19 +316,27 @@ __device__ __forceinline__ void decode_tile_rows(int tile, const int* s_off, int
     e = E - 1; m_blk = 0; n_blk = 0;  // not reached for tile < total
 }
 
-// Bounded wait that, on timeout, also raises the peer CTA's abort flag (pairs).
-__device__ __noinline__ bool wait_bounded_pair(uint32_t bar, uint32_t parity, volatile int* abort_flag,
-                                               unsigned int* err, uint32_t peer_abort_addr) {
-    if (mbar_try_wait(bar, parity)) return true;
-    const unsigned long long t0 = globaltimer();
-    for (;;) {
+// Bounded wait that, on timeout, also raises the peer CTA's abort flag
+// (pairs).  The hot path is a bare try_wait spin; the abort flag and the
+// clock are consulted only every 1024 tries, so a phase that completes
+// while the waiter spins is seen within one try (a timer read costs
+// hundreds of cycles, which would delay the next MMA issue).
+__device__ __forceinline__ bool wait_bounded_pair(uint32_t bar, uint32_t parity, volatile int* abort_flag,
+                                                  unsigned int* err, uint32_t peer_abort_addr) {
+    unsigned long long t0 = 0;
+    for (uint32_t i = 1;; ++i) {
         if (mbar_try_wait(bar, parity)) return true;
-        if (*abort_flag) return false;
-        if (globaltimer() - t0 > kTimeoutNs) {
-            *abort_flag = 1;
-            if (peer_abort_addr) st_cluster_u32(peer_abort_addr, 1u);
-            atomicOr(err, 1u);
-            return false;
+        if ((i & 1023u) == 0) {
+            if (*abort_flag) return false;
+            const unsigned long long now = globaltimer();
+            if (t0 == 0) {
+                t0 = now;
+            } else if (now - t0 > kTimeoutNs) {
+                *abort_flag = 1;
+                if (peer_abort_addr) st_cluster_u32(peer_abort_addr, 1u);
+                atomicOr(err, 1u);
+                return false;
+            }
         }
     }
 }
