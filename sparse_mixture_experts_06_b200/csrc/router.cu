@@ -32,17 +32,19 @@ namespace cg = cooperative_groups;
 namespace moe {
 namespace {
 
-constexpr int kMaxCluster = 8;     // CTAs per token group (d split up to 8 ways)
+constexpr int kMaxCluster = 8;     // CTAs per token group (d split 8 ways)
 constexpr int kWarps = 8;          // warps per CTA
 constexpr int kTok = 32;           // tokens per group (one per lane)
+constexpr int kMaxGroups = 4;      // token groups per CTA (the staged weights are reused)
 constexpr int kChunk = 512;        // features staged per pass (512 x 8 experts x 8 B = 32 KiB)
 constexpr int kWarpFeat = kChunk / kWarps;  // 64 features per warp per pass
 
-struct RouterSmem {
-    double wg[kChunk][8];                 // fp64 router weights, [feature][expert in group]
-    double red[kWarps][kTok][8];          // per-warp partial logits of one expert group
-    double part[kTok][kMaxExperts];       // this CTA's partial logits, all experts
-};
+// Dynamic shared memory: the fp64 weight slice wg[kChunk][8], the per-warp
+// partial sums red[kWarps][kTok][8], and this CTA's partial logits of every
+// token group part[g][token][expert] (E doubles per token).
+__host__ __device__ constexpr size_t router_smem_bytes(int E, int groups) {
+    return sizeof(double) * ((size_t)kChunk * 8 + (size_t)kWarps * kTok * 8 + (size_t)groups * kTok * E);
+}
 
 template <bool BF16>
 __device__ __forceinline__ void load_x_vec(const void* xr, int col, uint4 (&q)[BF16 ? 1 : 2]) {
@@ -81,31 +83,45 @@ __device__ __forceinline__ double load_w(const void* Wg, size_t idx) {
     }
 }
 
+// x vectors of this warp's 64 features of the chunk for one token.
+template <bool BF16>
+__device__ __forceinline__ void load_x_chunk(const void* xr, bool ok, int c0, int wf0, int clen,
+                                             uint4 (&q)[8][BF16 ? 1 : 2]) {
+#pragma unroll
+    for (int vv = 0; vv < 8; ++vv) {
+        const int col = wf0 + vv * 8;
+        if (ok && col < clen) load_x_vec<BF16>(xr, c0 + col, q[vv]);
+    }
+}
+
 template <bool BF16>
 __global__ void __launch_bounds__(kWarps * 32)
 router_topk_kernel(const void* __restrict__ x, const void* __restrict__ Wg, int T, int d, int E, int k,
-                   int32_t* __restrict__ idx_out, float* __restrict__ w_out) {
+                   int groups, int32_t* __restrict__ idx_out, float* __restrict__ w_out) {
     extern __shared__ __align__(16) unsigned char smem_raw[];
-    RouterSmem& sm = *reinterpret_cast<RouterSmem*>(smem_raw);
+    double (*wg)[8] = reinterpret_cast<double (*)[8]>(smem_raw);               // [kChunk][8]
+    double (*red)[kTok][8] =
+        reinterpret_cast<double (*)[kTok][8]>(reinterpret_cast<double*>(smem_raw) + (size_t)kChunk * 8);  // [kWarps][kTok][8]
+    double* part = reinterpret_cast<double*>(smem_raw) + (size_t)kChunk * 8 + (size_t)kWarps * kTok * 8;  // [groups][kTok][E]
     cg::cluster_group cluster = cg::this_cluster();
     const int rank = (int)cluster.block_rank();
     const int nranks = (int)cluster.num_blocks();
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int group = blockIdx.x / nranks;  // clusters tile grid.x
-    const int t = group * kTok + lane;
-    const bool tok_ok = t < T;
-    const void* xr = reinterpret_cast<const char*>(x) + (size_t)(tok_ok ? t : 0) * d * (BF16 ? 2 : 4);
+    const int tok0 = (blockIdx.x / nranks) * groups * kTok;  // first token of this cluster
+    const size_t row_bytes = (size_t)d * (BF16 ? 2 : 4);
 
     // this CTA's feature range (multiples of 8)
     const int slice = ((d + nranks * 8 - 1) / (nranks * 8)) * 8;
     const int f0 = min(d, rank * slice), f1 = min(d, f0 + slice);
+    const int wf0 = warp * kWarpFeat;
+
+    for (int i = threadIdx.x; i < groups * kTok * E; i += kWarps * 32) part[i] = 0.0;
 
     for (int eg = 0; eg < E; eg += 8) {
         const int ne = min(8, E - eg);
-        double acc[8] = {0, 0, 0, 0, 0, 0, 0, 0};
         for (int c0 = f0; c0 < f1; c0 += kChunk) {
             const int clen = min(kChunk, f1 - c0);
-            __syncthreads();  // previous chunk's weights are no longer read
+            __syncthreads();  // the previous pass no longer reads wg
             for (int i = threadIdx.x; i < kChunk; i += kWarps * 32) {
                 double v[8];
 #pragma unroll
@@ -113,93 +129,114 @@ router_topk_kernel(const void* __restrict__ x, const void* __restrict__ Wg, int 
                     v[e] = (i < clen && e < ne) ? load_w<BF16>(Wg, (size_t)(eg + e) * d + c0 + i) : 0.0;
 #pragma unroll
                 for (int e = 0; e < 8; e += 2)
-                    *reinterpret_cast<double2*>(&sm.wg[i][e]) = make_double2(v[e], v[e + 1]);
+                    *reinterpret_cast<double2*>(&wg[i][e]) = make_double2(v[e], v[e + 1]);
+            }
+            // first group's x loads overlap the staging
+            uint4 q[8][BF16 ? 1 : 2];
+            {
+                const int t = tok0 + lane;
+                load_x_chunk<BF16>(reinterpret_cast<const char*>(x) + (size_t)(t < T ? t : 0) * row_bytes, t < T, c0,
+                                   wf0, clen, q);
             }
             __syncthreads();
-            // this warp's 64 features of the chunk, 8 vectors of 8, all loads first
-            const int wf0 = warp * kWarpFeat;
-            uint4 q[8][BF16 ? 1 : 2];
+            for (int g = 0; g < groups; ++g) {
+                const int t = tok0 + g * kTok + lane;
+                const bool ok = t < T;
+                double a8[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+                uint4 qn[8][BF16 ? 1 : 2];
+                if (g + 1 < groups) {  // prefetch the next group's x
+                    const int tn = t + kTok;
+                    load_x_chunk<BF16>(reinterpret_cast<const char*>(x) + (size_t)(tn < T ? tn : 0) * row_bytes,
+                                       tn < T, c0, wf0, clen, qn);
+                }
 #pragma unroll
-            for (int vv = 0; vv < 8; ++vv) {
-                const int col = wf0 + vv * 8;
-                if (tok_ok && col < clen) load_x_vec<BF16>(xr, c0 + col, q[vv]);
-            }
+                for (int vv = 0; vv < 8; ++vv) {
+                    const int col = wf0 + vv * 8;
+                    if (!ok || col >= clen) continue;  // (features past the chunk: nothing to add)
+                    double xd[8];
+                    widen8<BF16>(q[vv], xd);
 #pragma unroll
-            for (int vv = 0; vv < 8; ++vv) {
-                const int col = wf0 + vv * 8;
-                if (!tok_ok || col >= clen) continue;  // (features past the chunk: nothing to add)
-                double xd[8];
-                widen8<BF16>(q[vv], xd);
+                    for (int i = 0; i < 8; ++i) {
+                        const double2* wrow = reinterpret_cast<const double2*>(&wg[col + i][0]);
+                        const double2 w01 = wrow[0], w23 = wrow[1], w45 = wrow[2], w67 = wrow[3];
+                        a8[0] = fma(xd[i], w01.x, a8[0]);
+                        a8[1] = fma(xd[i], w01.y, a8[1]);
+                        a8[2] = fma(xd[i], w23.x, a8[2]);
+                        a8[3] = fma(xd[i], w23.y, a8[3]);
+                        a8[4] = fma(xd[i], w45.x, a8[4]);
+                        a8[5] = fma(xd[i], w45.y, a8[5]);
+                        a8[6] = fma(xd[i], w67.x, a8[6]);
+                        a8[7] = fma(xd[i], w67.y, a8[7]);
+                    }
+                }
+                // per-warp partials -> this CTA's partial logits (warp order)
 #pragma unroll
-                for (int i = 0; i < 8; ++i) {
-                    const double2* wrow = reinterpret_cast<const double2*>(&sm.wg[col + i][0]);
-                    const double2 w01 = wrow[0], w23 = wrow[1], w45 = wrow[2], w67 = wrow[3];
-                    acc[0] = fma(xd[i], w01.x, acc[0]);
-                    acc[1] = fma(xd[i], w01.y, acc[1]);
-                    acc[2] = fma(xd[i], w23.x, acc[2]);
-                    acc[3] = fma(xd[i], w23.y, acc[3]);
-                    acc[4] = fma(xd[i], w45.x, acc[4]);
-                    acc[5] = fma(xd[i], w45.y, acc[5]);
-                    acc[6] = fma(xd[i], w67.x, acc[6]);
-                    acc[7] = fma(xd[i], w67.y, acc[7]);
+                for (int e = 0; e < 8; ++e) red[warp][lane][e] = a8[e];
+                __syncthreads();
+                {
+                    const int tk = threadIdx.x >> 3, e = threadIdx.x & 7;  // 256 threads = 32 tokens x 8 experts
+                    double s = 0.0;
+#pragma unroll
+                    for (int w = 0; w < kWarps; ++w) s += red[w][tk][e];
+                    if (e < ne) part[((size_t)g * kTok + tk) * E + eg + e] += s;
+                }
+                __syncthreads();
+                if (g + 1 < groups) {
+#pragma unroll
+                    for (int vv = 0; vv < 8; ++vv) q[vv][0] = qn[vv][0];
+                    if constexpr (!BF16) {
+#pragma unroll
+                        for (int vv = 0; vv < 8; ++vv) q[vv][1] = qn[vv][1];
+                    }
                 }
             }
         }
-        // warp partials -> CTA partial, summed in warp order
-#pragma unroll
-        for (int e = 0; e < 8; ++e) sm.red[warp][lane][e] = acc[e];
-        __syncthreads();
-        {
-            const int tk = threadIdx.x >> 3, e = threadIdx.x & 7;  // 256 threads = 32 tokens x 8 experts
-            double s = 0.0;
-#pragma unroll
-            for (int w = 0; w < kWarps; ++w) s += sm.red[w][tk][e];
-            if (e < ne) sm.part[tk][eg + e] = s;
-        }
-        __syncthreads();
     }
 
     cluster.sync();  // every CTA's partial logits are complete and visible
     if (rank == 0) {
-        // logits = sum over the 8 CTAs in rank order, one thread per (token, expert)
-        for (int i = threadIdx.x; i < kTok * E; i += kWarps * 32) {
-            const int tk = i / E, e = i - tk * E;
+        // logits = sum over the CTAs in rank order, written over wg and red
+        // (both free now; the launch keeps groups * 32 * E within their
+        // kChunk * 8 + kWarps * kTok * 8 doubles, so part is never overwritten)
+        double* lg_all = reinterpret_cast<double*>(smem_raw);
+        for (int i = threadIdx.x; i < groups * kTok * E; i += kWarps * 32) {
             double s = 0.0;
-            for (int r = 0; r < nranks; ++r) {
-                const RouterSmem* peer = cluster.map_shared_rank(&sm, r);
-                s += peer->part[tk][e];
-            }
-            reinterpret_cast<double*>(sm.wg)[i] = s;  // reuse the weight area for the final logits
+            for (int r = 0; r < nranks; ++r) s += cluster.map_shared_rank(part, r)[i];
+            lg_all[i] = s;
         }
     }
     cluster.sync();  // peers keep their shared memory until CTA 0 has read it
-    if (rank != 0 || threadIdx.x >= kTok || !tok_ok) return;
-
-    const double* lg = reinterpret_cast<const double*>(sm.wg) + (size_t)threadIdx.x * E;
-    // k rounds of arg-max; indices are written as they are found and the
-    // fp32 softmax numerators exp(l_j - l_0) are parked in w_out, then
-    // divided by their slot-ordered sum (any k <= E, no per-k arrays)
-    uint64_t taken = 0;
-    double l0 = 0.0;
-    float sum = 0.f;
-    int32_t* io = idx_out + (size_t)t * k;
-    float* wo = w_out + (size_t)t * k;
-    for (int j = 0; j < k; ++j) {
-        int bi = -1;
-        double best = 0.0;
-        for (int e = 0; e < E; ++e) {
-            if ((taken >> e) & 1ull) continue;
-            const double v = lg[e];
-            if (bi < 0 || v > best) { best = v; bi = e; }
+    if (rank != 0) return;
+    __syncthreads();
+    for (int tl = threadIdx.x; tl < groups * kTok; tl += kWarps * 32) {
+        const int t = tok0 + tl;
+        if (t >= T) continue;
+        const double* lg = reinterpret_cast<const double*>(smem_raw) + (size_t)tl * E;
+        // k rounds of arg-max; indices are written as they are found and the
+        // fp32 softmax numerators exp(l_j - l_0) are parked in w_out, then
+        // divided by their slot-ordered sum (any k <= E, no per-k arrays)
+        uint64_t taken = 0;
+        double l0 = 0.0;
+        float sum = 0.f;
+        int32_t* io = idx_out + (size_t)t * k;
+        float* wo = w_out + (size_t)t * k;
+        for (int j = 0; j < k; ++j) {
+            int bi = -1;
+            double best = 0.0;
+            for (int e = 0; e < E; ++e) {
+                if ((taken >> e) & 1ull) continue;
+                const double v = lg[e];
+                if (bi < 0 || v > best) { best = v; bi = e; }
+            }
+            taken |= 1ull << bi;
+            if (j == 0) l0 = best;
+            const float ex = expf((float)(best - l0));
+            io[j] = bi;
+            wo[j] = ex;
+            sum += ex;
         }
-        taken |= 1ull << bi;
-        if (j == 0) l0 = best;
-        const float ex = expf((float)(best - l0));
-        io[j] = bi;
-        wo[j] = ex;
-        sum += ex;
+        for (int j = 0; j < k; ++j) wo[j] = wo[j] / sum;
     }
-    for (int j = 0; j < k; ++j) wo[j] = wo[j] / sum;
 }
 
 template <bool BF16>
@@ -208,14 +245,18 @@ cudaError_t launch_impl(const void* x, const void* Wg, int T, int d, int E, int 
     static bool attr_done[64] = {false};
     int dev = 0;
     cudaGetDevice(&dev);
-    const int smem = (int)sizeof(RouterSmem);
     if (dev < 64 && !attr_done[dev]) {
-        cudaError_t e = cudaFuncSetAttribute(router_topk_kernel<BF16>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+        cudaError_t e = cudaFuncSetAttribute(router_topk_kernel<BF16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             (int)router_smem_bytes(kMaxExperts, kMaxGroups));
         if (e != cudaSuccess) return e;
         attr_done[dev] = true;
     }
-    // d is split 8 ways (a 4-way split, with half the CTAs, measured slower
-    // at T = 4096 on B200).
+    // token groups per cluster: reuse the staged weights for up to 4 groups
+    // once there are enough groups to fill the GPU with clusters anyway
+    const int ngroups = (T + kTok - 1) / kTok;
+    int groups = ngroups >= 4 * 64 ? kMaxGroups : (ngroups >= 2 * 64 ? 2 : 1);
+    const int fit = (kChunk * 8 + kWarps * kTok * 8) / (kTok * E);  // final logits must fit wg + red
+    if (groups > fit) groups = fit > 0 ? fit : 1;
     const int nranks = kMaxCluster;
     cudaLaunchConfig_t cfg = {};
     cudaLaunchAttribute attr[1];
@@ -223,13 +264,13 @@ cudaError_t launch_impl(const void* x, const void* Wg, int T, int d, int E, int 
     attr[0].val.clusterDim.x = nranks;
     attr[0].val.clusterDim.y = 1;
     attr[0].val.clusterDim.z = 1;
-    cfg.gridDim = dim3(nranks * ((T + kTok - 1) / kTok));
+    cfg.gridDim = dim3(nranks * ((ngroups + groups - 1) / groups));
     cfg.blockDim = dim3(kWarps * 32);
-    cfg.dynamicSmemBytes = smem;
+    cfg.dynamicSmemBytes = router_smem_bytes(E, groups);
     cfg.stream = s;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, router_topk_kernel<BF16>, x, Wg, T, d, E, k, idx, w);
+    return cudaLaunchKernelEx(&cfg, router_topk_kernel<BF16>, x, Wg, T, d, E, k, groups, idx, w);
 }
 
 }  // namespace

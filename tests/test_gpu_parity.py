@@ -69,6 +69,8 @@ def test_device_generator_matches_host(dt):
     (16, 64, 8, 2, "f32"), (37, 72, 8, 2, "bf16"), (1, 8, 1, 1, "bf16"), (300, 256, 64, 8, "bf16"),
     (129, 4096, 8, 2, "bf16"), (250, 96, 5, 3, "f32"), (100, 128, 8, 8, "bf16"), (70, 64, 64, 64, "f32"),
     (64, 256, 16, 12, "bf16"),
+    # many tokens: several token groups per cluster (2, 4, and 3 for E = 64), ragged last group
+    (4100, 256, 8, 2, "bf16"), (8229, 512, 8, 2, "bf16"), (8200, 128, 64, 8, "bf16"), (9000, 64, 8, 2, "f32"),
 ])
 def test_router_parity(T, d, E, k, dt):
     t = device_inputs(synth.MoEShape("r", T, d, 8, E, k, dt), seed=T + E)
