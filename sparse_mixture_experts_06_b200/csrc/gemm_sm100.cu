@@ -71,7 +71,13 @@ struct KParams {
     float* obuf;             // down output [rows, d]
     int rows;                // T*k
     unsigned int* err;       // device error word (MOE_DEVERR_*)
+    int row_mode;            // rows of each expert to cover: kAllRows, kFullPairBlocks or kPairRemainders
 };
+
+// Row ranges: all rows of each expert; only its whole 256-row blocks; or
+// only the rows after them.  A layer can run the pair kernel on the blocks
+// and the single-CTA kernel (128-row tiles, less padding) on the rest.
+enum RowMode { kAllRows = 0, kFullPairBlocks = 1, kPairRemainders = 2 };
 
 // ---------------------------------------------------------------------------
 // PTX wrappers
@@ -293,17 +299,19 @@ struct Cfg {
                                        ((uint32_t)((128 * CG) >> 4) << 24);
 };
 
-__device__ __forceinline__ int count_tiles_rows(const int* s_off, int E, int n_tiles, int rows_per_tile) {
+// Tiles of expert e cover rows [s_beg[e], s_end[e]) in blocks of rows_per_tile.
+__device__ __forceinline__ int count_tiles_rows(const int* s_beg, const int* s_end, int E, int n_tiles,
+                                                int rows_per_tile) {
     int total = 0;
-    for (int e = 0; e < E; ++e) total += ((s_off[e + 1] - s_off[e] + rows_per_tile - 1) / rows_per_tile) * n_tiles;
+    for (int e = 0; e < E; ++e) total += ((s_end[e] - s_beg[e] + rows_per_tile - 1) / rows_per_tile) * n_tiles;
     return total;
 }
 
-__device__ __forceinline__ void decode_tile_rows(int tile, const int* s_off, int E, int n_tiles, int rows_per_tile,
-                                                 int& e, int& m_blk, int& n_blk) {
+__device__ __forceinline__ void decode_tile_rows(int tile, const int* s_beg, const int* s_end, int E, int n_tiles,
+                                                 int rows_per_tile, int& e, int& m_blk, int& n_blk) {
     int base = 0;
     for (e = 0; e < E; ++e) {
-        const int mt = (s_off[e + 1] - s_off[e] + rows_per_tile - 1) / rows_per_tile;
+        const int mt = (s_end[e] - s_beg[e] + rows_per_tile - 1) / rows_per_tile;
         const int tiles = mt * n_tiles;
         if (tile < base + tiles) {
             const int local = tile - base;
@@ -360,7 +368,8 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
     uint64_t* tempty = bars + 2 * STG + 2;
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * STG + 4);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
-    int* s_off = reinterpret_cast<int*>(tmem_slot + 2);
+    int* s_beg = reinterpret_cast<int*>(tmem_slot + 2);  // [E] first row of expert e's range
+    int* s_end = s_beg + kMaxExperts;                   // [E] end of expert e's range
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const uint32_t rank = (CG == 2) ? cluster_rank() : 0u;
@@ -379,7 +388,12 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
         *abort_flag = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
-    if (threadIdx.x <= p.E) s_off[threadIdx.x] = p.offsets[threadIdx.x];
+    if (threadIdx.x < p.E) {
+        const int o0 = p.offsets[threadIdx.x], o1 = p.offsets[threadIdx.x + 1];
+        const int split = o0 + ((o1 - o0) / 256) * 256;  // end of the whole 256-row blocks
+        s_beg[threadIdx.x] = (p.row_mode == kPairRemainders) ? split : o0;
+        s_end[threadIdx.x] = (p.row_mode == kFullPairBlocks) ? split : o1;
+    }
     if (warp == 1) {
         if constexpr (CG == 1) {
             asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_slot)),
@@ -396,7 +410,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
     tc_fence_after();
     const uint32_t tmem_base = *tmem_slot;
 
-    const int total = count_tiles_rows(s_off, p.E, p.n_tiles, C::kTileRows);
+    const int total = count_tiles_rows(s_beg, s_end, p.E, p.n_tiles, C::kTileRows);
     const int kblocks = (p.Kdim + BK - 1) / BK;
     const int tile0 = (CG == 2) ? (int)(blockIdx.x >> 1) : (int)blockIdx.x;
     const int tstep = (CG == 2) ? (int)(gridDim.x >> 1) : (int)gridDim.x;
@@ -408,8 +422,8 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
             bool ok = true;
             for (int tile = tile0; tile < total && ok; tile += tstep) {
                 int e, mb, nb;
-                decode_tile_rows(tile, s_off, p.E, p.n_tiles, C::kTileRows, e, mb, nb);
-                const int rowA = s_off[e] + mb * C::kTileRows + (int)rank * 128;
+                decode_tile_rows(tile, s_beg, s_end, p.E, p.n_tiles, C::kTileRows, e, mb, nb);
+                const int rowA = s_beg[e] + mb * C::kTileRows + (int)rank * 128;
                 int rowB0, rowB1;
                 const CUtensorMap* mapB = &tmB0;
                 if constexpr (CG == 1) {
@@ -501,7 +515,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
         uint32_t tcount = 0;
         for (int tile = tile0; tile < total; tile += tstep, ++tcount) {
             int e, mb, nb;
-            decode_tile_rows(tile, s_off, p.E, p.n_tiles, C::kTileRows, e, mb, nb);
+            decode_tile_rows(tile, s_beg, s_end, p.E, p.n_tiles, C::kTileRows, e, mb, nb);
             const uint32_t acc = tcount & 1u;
             const uint32_t use = tcount >> 1;
             // every lane waits; the decision to stop is warp-uniform so the
@@ -509,8 +523,8 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
             const bool okw = wait_bounded_pair(smem_u32(&tfull[acc]), use & 1u, abort_flag, p.err, peer_abort);
             if (!__all_sync(0xffffffffu, okw)) break;
             tc_fence_after();
-            const int row = s_off[e] + mb * C::kTileRows + r_in;
-            const int tile_end = min(s_off[e + 1], s_off[e] + (mb + 1) * C::kTileRows);
+            const int row = s_beg[e] + mb * C::kTileRows + r_in;
+            const int tile_end = min(s_end[e], s_beg[e] + (mb + 1) * C::kTileRows);
             const bool valid = row < tile_end;
             // rows of this warp: whole box stored by TMA when all 32 are the
             // expert's own; a box straddling the end of the expert's block
@@ -715,17 +729,26 @@ cudaError_t launch_gemm(const GroupedGemmArgs& a, const CUtensorMap& mA, const C
     return cudaLaunchKernelEx(&cfg, grouped_gemm_kernel<MODE, CG, BN, RB>, mA, mB0, mB1, mOut, p);
 }
 
-// CTA-pair tiles (M = 256) move a third fewer bytes per MMA from L2 but pad
-// each expert's last tile to 256 rows.  Measured on B200 (prefill T = 4096
-// and skewed T = 16384): the down-projection (K = f = 14336) gains from
-// pairs once experts average >= 512 rows; the up-projection (K = d) does not
-// (the padding costs as much as the pair saves), and neither does decode.
-// MOE_GEMM_CTA_GROUP = 1 or 2 forces one variant for both GEMMs (both are
-// exact; the tests run both).
+// Variant choice: 1 = single-CTA tiles, 2 = CTA-pair tiles, 3 = hybrid.
+// Measured on B200 with Mixtral shapes:
+//  * pairs (M = 256) move a third fewer bytes per MMA from L2 and ran ~10%
+//    faster per row (one-expert 8192-row layer: up 1.34 vs 1.48 ms, down
+//    0.66 vs 0.77 ms), but pad every expert to a multiple of 256 rows;
+//  * grouped prefill (T = 4096, ~1000 rows per expert): single-CTA tiles are
+//    best for the up-projection (K = d), pairs for the down-projection
+//    (K = f): 1.55 + 0.77 ms;
+//  * the hybrid (pairs on each expert's whole 256-row blocks, then a
+//    single-CTA launch on the remaining rows) was slower (1.62 + 0.93 ms):
+//    the second launch has only 1-2 row tiles per weight tile and streams
+//    every expert's weights from HBM again;
+//  * decode (a few rows per expert): single-CTA tiles.
+// MOE_GEMM_CTA_GROUP = 1, 2 or h forces a variant (all exact; the tests run
+// each).
 int choose_cta_group(const GroupedGemmArgs& a, int mode) {
     if (const char* env = getenv("MOE_GEMM_CTA_GROUP")) {
         if (env[0] == '1') return 1;
         if (env[0] == '2') return 2;
+        if (env[0] == 'h') return 3;
     }
     return (mode == kDown && a.rows >= 512 * a.E) ? 2 : 1;
 }
@@ -766,7 +789,16 @@ template <int MODE, int BN>
 cudaError_t launch_variant(const GroupedGemmArgs& a, const CUtensorMap& mA, const CUtensorMap& mA32,
                            const CUtensorMap& mB0, const CUtensorMap& mB1, const CUtensorMap& mOut, const KParams& p,
                            cudaStream_t s) {
-    if (choose_cta_group(a, MODE) == 2) return launch_gemm<MODE, 2, BN, 128>(a, mA, mB0, mB1, mOut, p, s);
+    const int cg = choose_cta_group(a, MODE);
+    if (cg == 2) return launch_gemm<MODE, 2, BN, 128>(a, mA, mB0, mB1, mOut, p, s);
+    if (cg == 3) {  // hybrid: pairs on whole 256-row blocks, then single CTAs on the rest (same stream)
+        KParams pf = p, pr = p;
+        pf.row_mode = kFullPairBlocks;
+        pr.row_mode = kPairRemainders;
+        cudaError_t e = launch_gemm<MODE, 2, BN, 128>(a, mA, mB0, mB1, mOut, pf, s);
+        if (e != cudaSuccess) return e;
+        return launch_gemm<MODE, 1, BN, 128>(a, mA, mB0, mB1, mOut, pr, s);
+    }
     return choose_rb(a) == 32 ? launch_gemm<MODE, 1, BN, 32>(a, mA32, mB0, mB1, mOut, p, s)
                               : launch_gemm<MODE, 1, BN, 128>(a, mA, mB0, mB1, mOut, p, s);
 }

@@ -169,14 +169,15 @@ def test_layer_parity_every_token_f32(shape):
 
 
 GEMM_VARIANTS = [("1", "256", "128"), ("1", "128", "128"), ("1", "256", "32"), ("1", "128", "32"),
-                 ("2", "256", "128"), ("2", "128", "128")]
+                 ("2", "256", "128"), ("2", "128", "128"), ("h", "256", "128"), ("h", "128", "128")]
 
 
 @pytest.mark.parametrize("variant", GEMM_VARIANTS, ids=lambda v: "cg%s-bn%s-rb%s" % v)
 @pytest.mark.parametrize("shape", BF16_SHAPES, ids=lambda s: s.name)
 def test_layer_parity_every_token_bf16(shape, variant, monkeypatch):
     """Every GEMM variant: single-CTA tiles of 128 or 32 token rows, CTA-pair
-    256-row tiles, and 256- or 128-column up-projection tiles."""
+    256-row tiles, the hybrid (pairs on whole 256-row blocks, single CTAs on
+    the rest), and 256- or 128-column up-projection tiles."""
     cta_group, bn, rb = variant
     monkeypatch.setenv("MOE_GEMM_CTA_GROUP", cta_group)
     monkeypatch.setenv("MOE_GEMM_BN", bn)
@@ -331,8 +332,9 @@ def test_prefill_full_shape(mixtral_weights):
 
 
 @pytest.mark.parametrize("name,cta_group,bn,rb", [("decode", "2", "256", "128"), ("decode", "1", "256", "128"),
+                                                  ("decode", "h", "256", "128"),
                                                   ("prefill", "1", "128", "128"), ("prefill", "2", "256", "128"),
-                                                  ("prefill", "1", "256", "32")])
+                                                  ("prefill", "1", "256", "128"), ("prefill", "1", "256", "32")])
 def test_full_shapes_other_gemm_variant(name, cta_group, bn, rb, mixtral_weights, monkeypatch):
     """Variants the size heuristics do not pick, at the full shapes."""
     monkeypatch.setenv("MOE_GEMM_CTA_GROUP", cta_group)
