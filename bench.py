@@ -337,6 +337,29 @@ def bench_stack(steps, device, pk):
     return out
 
 
+def graph_step_ms(r, s, device, steps):
+    """The same layer call captured once in a CUDA graph and replayed
+    (no per-kernel launch gaps; how a serving loop would run decode)."""
+    import torch
+    import sparse_mixture_experts_06_b200 as moe
+    t, y, ws = r["t"], r["y"], r["ws"]
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        moe.moe_layer_forward_ex(t["x"], t["Wg"], t["W1"], t["W3"], t["W2"], s.k, y=y, workspace=ws)
+    for _ in range(3):
+        g.replay()
+    torch.cuda.synchronize(device)
+    stream = torch.cuda.current_stream(device)
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    for _ in range(steps):
+        g.replay()
+    b.record(stream)
+    torch.cuda.synchronize(device)
+    del g
+    return a.elapsed_time(b) / steps
+
+
 def e2e_leg(args, s, t, device, steps):
     """Same layer through the public entry point moe_layer_forward (library
     workspace), with the step's tokens copied in from pinned host memory and
@@ -449,7 +472,13 @@ def main():
         wbytes = 3.0 * d.E * d.d * d.f * 2  # all 8 experts are touched at T=32 with near-uniform routing
         ups, upn = p["up_swiglu_gemm"]
         dns, dnn = p["down_scaled_gemm"]
+        gms = graph_step_ms(rd, d, device, dargs.steps)
         line["decode"] = {"workload": workload_desc(d, world)["workload"], "ms_per_step": dms,
+                          "ms_per_step_cuda_graph": gms,
+                          "cuda_graph_note": "one captured layer replayed back to back; no L2 flush (the 2.82 GB "
+                                             "of weights exceed L2)",
+                          "weight_GBps_cuda_graph": wbytes / (gms * 1e-3) / 1e9,
+                          "frac_of_hbm_cuda_graph": wbytes / (gms * 1e-3) / 1e9 / pk["hbm_gbs"],
                           "tokens_per_s": world * d.T / (dms * 1e-3),
                           "weight_GBps": wbytes / (dms * 1e-3) / 1e9,
                           "frac_of_hbm": wbytes / (dms * 1e-3) / 1e9 / pk["hbm_gbs"],

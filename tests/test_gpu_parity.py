@@ -98,21 +98,28 @@ def test_router_ties_go_to_lower_index():
 # ---------------------------------------------------------------- permutation
 
 @pytest.mark.parametrize("T,E,k", [(1, 8, 2), (511, 8, 2), (512, 8, 2), (1500, 8, 2), (3000, 64, 8),
-                                   (777, 3, 1), (20000, 8, 2)])
+                                   (777, 3, 1), (20000, 8, 2), (16384, 8, 2), (5000, 16, 4), (2000, 17, 3),
+                                   (0, 8, 2),
+                                   # the one-pass kernel (E <= 16, 4096..16384 assignments)
+                                   (4096, 8, 2), (2049, 8, 2), (8192, 8, 2), (2048, 16, 4), (4100, 5, 3)])
 def test_permute_parity(T, E, k):
     rng = np.random.default_rng(T)
     # a skewed draw that leaves some experts empty
     p = rng.dirichlet(np.ones(E) * 0.3)
-    idx = np.stack([rng.choice(E, size=k, replace=False, p=p) for _ in range(T)]).astype(np.int32)
+    idx = np.stack([rng.choice(E, size=k, replace=False, p=p) for _ in range(T)]).astype(np.int32) if T else \
+        np.zeros((0, k), dtype=np.int32)
     off, perm, inv = moe.moe_permute(torch.from_numpy(idx).cuda(), E)
     check_permutation(off.cpu().numpy(), perm.cpu().numpy(), inv.cpu().numpy(), idx, E)
 
 
-def test_permute_flags_bad_expert_ids():
-    idx = torch.tensor([[0, 1], [9, 2]], dtype=torch.int32, device="cuda")
-    off, perm, inv = moe.moe_permute(idx, 8)
+@pytest.mark.parametrize("E,T", [(8, 3), (20, 3), (8, 3000)])  # the general and the one-pass kernel
+def test_permute_flags_bad_expert_ids(E, T):
+    rows = [[0, 1], [E + 1, 2], [-3, 4]] + [[5, 6]] * (T - 3)
+    idx = torch.tensor(rows, dtype=torch.int32, device="cuda")
+    off, perm, inv = moe.moe_permute(idx, E)
     assert moe.moe_device_errors() == 2
-    assert off.cpu().tolist()[-1] == 3 and inv.cpu().tolist()[2] == -1
+    assert off.cpu().tolist()[-1] == 2 * T - 2 and inv.cpu().tolist()[2] == -1 and inv.cpu().tolist()[4] == -1
+    assert sorted(perm.cpu().tolist()[:4]) == [0, 1, 3, 5]
 
 
 # ---------------------------------------------------------------- routing statistics
