@@ -50,7 +50,10 @@ def parse():
     ap.add_argument("--workload", default="prefill", choices=["prefill", "decode", "skewed"])
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-extras", action="store_true", help="skip the decode line and the CPU baseline")
-    ap.add_argument("--cpu-sample", type=int, default=32, help="tokens in the oracle's timed sample")
+    ap.add_argument("--cpu-sample", type=int, default=4096,
+                    help="tokens in the oracle's timed CPU-baseline sample (default: the whole prefill batch)")
+    ap.add_argument("--ref-sample", type=int, default=128,
+                    help="tokens per step of --impl reference (keeps --steps K --warmup W within minutes)")
     return ap.parse_args()
 
 
@@ -203,7 +206,7 @@ def run_reference(args):
     x_bits = to_host_bits(t["x"])
     del t
     torch.cuda.empty_cache()
-    n = args.cpu_sample
+    n = args.ref_sample
     rng = np.random.default_rng(0)
     times = []
     threads = 1
