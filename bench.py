@@ -54,6 +54,9 @@ def parse():
                     help="tokens in the oracle's timed CPU-baseline sample (default: the whole prefill batch)")
     ap.add_argument("--ref-sample", type=int, default=128,
                     help="tokens per step of --impl reference (keeps --steps K --warmup W within minutes)")
+    ap.add_argument("--gemm-vs-cublas", action="store_true",
+                    help="instead of the layer: time the two expert GEMMs against cuBLAS (torch.matmul) "
+                         "on the same shapes and print one JSON line")
     return ap.parse_args()
 
 
@@ -394,10 +397,109 @@ def e2e_leg(args, s, t, device, steps):
     return ms, nbytes, y_h.numel() * y_h.element_size()
 
 
+def gemm_vs_cublas(args, device):
+    """The expert GEMMs of the prefill layer (T = 4096, d = 4096, f = 14336,
+    E = 8, k = 2) against cuBLAS through torch.matmul, for context:
+      * one dense GEMM of all 8192 rows (up: [8192, d] x [d, 2f]; down:
+        [8192, f] x [f, d]), cuBLAS's best case;
+      * cuBLAS per expert on the rows the router actually gave each expert
+        (the grouped work, one call per expert, no SwiGLU or gate fusion);
+      * ours on a one-expert layer of 8192 rows (E = 1, k = 1: no ragged
+        tiles) for each CTA grouping, and ours on the grouped prefill layer,
+        both from the library's stage profiler.
+    cuBLAS here is a measuring stick only; the layer never calls it."""
+    import torch
+    import synth
+    import sparse_mixture_experts_06_b200 as moe
+    from synth.device import device_inputs
+
+    def t_ms(fn, reps=20):
+        for _ in range(3):
+            fn()
+        torch.cuda.synchronize(device)
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        for _ in range(reps):
+            fn()
+        b.record()
+        torch.cuda.synchronize(device)
+        return a.elapsed_time(b) / reps
+
+    s = synth.CONFIGS["prefill"]
+    M, d, f = s.T * s.k, s.d, s.f
+    tf = lambda flop, ms: round(flop / ms / 1e9, 1)  # noqa: E731
+    g = torch.Generator(device=device).manual_seed(0)
+    x = torch.randn(M, d, device=device, generator=g).to(torch.bfloat16)
+    W13 = (torch.randn(2 * f, d, device=device, generator=g) / 64).to(torch.bfloat16)
+    h = torch.randn(M, f, device=device, generator=g).to(torch.bfloat16)
+    W2 = (torch.randn(d, f, device=device, generator=g) / 120).to(torch.bfloat16)
+    out = {"mode": "gemm_vs_cublas", "unit": "TFLOP/s", "rows": M, "d": d, "f": f}
+    up = t_ms(lambda: x @ W13.t())
+    dn = t_ms(lambda: h @ W2.t())
+    out["cublas_dense"] = {"up_ms": round(up, 4), "up": tf(4.0 * M * d * f, up),
+                           "down_ms": round(dn, 4), "down": tf(2.0 * M * d * f, dn)}
+    del x, W13, h, W2
+
+    # grouped: the router's per-expert row counts of the prefill batch
+    t = make_inputs(s, 0, device)
+    idx, _ = moe.moe_router_topk(t["x"], t["Wg"], s.k)
+    counts = torch.bincount(idx.flatten().long(), minlength=s.E).tolist()
+    xs = [torch.randn(c, d, device=device, generator=g).to(torch.bfloat16) for c in counts]
+    hs = [torch.randn(c, f, device=device, generator=g).to(torch.bfloat16) for c in counts]
+    W13e = torch.cat([t["W1"], t["W3"]], dim=1)  # [E, 2f, d]
+    upg = t_ms(lambda: [xe @ W13e[e].t() for e, xe in enumerate(xs)])
+    dng = t_ms(lambda: [he @ t["W2"][e].t() for e, he in enumerate(hs)])
+    out["cublas_per_expert"] = {"counts": counts, "up_ms": round(upg, 4), "up": tf(4.0 * M * d * f, upg),
+                                "down_ms": round(dng, 4), "down": tf(2.0 * M * d * f, dng)}
+    del xs, hs, W13e
+
+    def ours(shape, tt, key, env=None):
+        old = os.environ.get("MOE_GEMM_CTA_GROUP")
+        if env is not None:
+            os.environ["MOE_GEMM_CTA_GROUP"] = env
+        try:
+            y = torch.empty_like(tt["x"])
+            ws = torch.empty(moe.moe_workspace_size(shape.T, d, f, shape.E, shape.k, 0), dtype=torch.uint8,
+                             device=device)
+            run = lambda: moe.moe_layer_forward_ex(tt["x"], tt["Wg"], tt["W1"], tt["W3"], tt["W2"], shape.k,  # noqa: E731
+                                                   y=y, workspace=ws)
+            for _ in range(3):
+                run()
+            torch.cuda.synchronize(device)
+            moe.moe_profile_enable(True)
+            for _ in range(20):
+                run()
+            torch.cuda.synchronize(device)
+            p = moe.moe_profile_read()
+            moe.moe_profile_enable(False)
+        finally:
+            if env is not None:
+                if old is None:
+                    os.environ.pop("MOE_GEMM_CTA_GROUP", None)
+                else:
+                    os.environ["MOE_GEMM_CTA_GROUP"] = old
+        u, w = p["up_swiglu_gemm"][0] / 20, p["down_scaled_gemm"][0] / 20
+        out[key] = {"up_ms": round(u, 4), "up": tf(4.0 * M * d * f, u), "down_ms": round(w, 4),
+                    "down": tf(2.0 * M * d * f, w)}
+
+    one = synth.MoEShape("one-expert", M, d, f, 1, 1, "bf16")
+    t1 = device_inputs(one, 0, device=device)
+    for cg in ("1", "2"):
+        ours(one, t1, "ours_one_expert_cta_group_%s" % cg, env=cg)
+    del t1
+    ours(s, t, "ours_grouped_prefill")
+    print(json.dumps(out))
+    return 0
+
+
 def main():
     args = parse()
     if args.impl == "reference":
         return run_reference(args)
+    if args.gemm_vs_cublas:
+        import torch
+        torch.cuda.set_device(0)
+        return gemm_vs_cublas(args, torch.device("cuda", 0))
     rank = int(os.environ.get("RANK", "0"))
     world = int(os.environ.get("WORLD_SIZE", "1"))
     local = int(os.environ.get("LOCAL_RANK", "0"))

@@ -25,8 +25,15 @@
 // one N = 256 MMA produces a (columns 0-127) and b (128-255) for 128
 // hidden units.  Down tiles: B = 256 rows of W2_e.
 //
+// CTA pairs (cta_group::2) run 256-row tiles as M = 256 MMAs; the last row
+// block of an expert that holds at most 128 rows runs as an M = 128 pair
+// MMA instead (each CTA loads 64 rows of A), so pairs pad an expert to a
+// multiple of 128 rows, not 256.  In a pair up tile each CTA's half of B is
+// 64 rows of W1 followed by the same 64 rows of W3, so that a and b of one
+// hidden unit sit in the same TMEM lane for both MMA shapes.
+//
 // Tiles are enumerated per expert from the device-side offsets (no host
-// round trip): expert e owns ceil(M_e / 128) row blocks x n_tiles column
+// round trip): expert e owns ceil(M_e / tile rows) row blocks x n_tiles column
 // blocks, numbered with the row block fastest so that the CTAs running at
 // the same time share weight tiles through L2.  Ragged row blocks read the
 // next expert's rows (or the zero fill past the end) and simply do not
@@ -273,6 +280,11 @@ constexpr int kOutBytes = 4 * 2 * kOutBoxBytes;
 // its own shared memory.  CG = 2: a CTA pair per 256-row tile; each CTA
 // holds its 128 rows of A and its BN/2-row half of B; the even CTA issues
 // M = 256 MMAs that read both CTAs' shared memory and write both CTAs' TMEM.
+// A short pair tile (an expert's last block, at most 128 rows) loads 64 rows
+// of A per CTA and issues M = 128 MMAs; each CTA's 64 x BN accumulator then
+// occupies TMEM lanes 0-63 for columns 0 .. BN/2-1 and lanes 64-127 for
+// columns BN/2 .. BN-1, both at column offsets 0 .. BN/2-1 (the 2x2
+// datapath layout of the 2-SM M = 128 shape).
 // The stage ring fills 192 KiB of shared memory.
 //
 // Instruction descriptor (kind::f16): D fp32 (bits 4-5 = 1), A and B bf16
@@ -297,7 +309,14 @@ struct Cfg {
     static constexpr int kSmem = 1024 + kStages * kStageBytes + kOutBytes + 1024;
     static constexpr uint32_t kIdesc = (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(BN >> 3) << 17) |
                                        ((uint32_t)((128 * CG) >> 4) << 24);
+    // short pair tiles: M = 128 across the pair, 64 rows of A per CTA
+    static constexpr int kAShortBytes = 64 * BK * 2;
+    static constexpr uint32_t kIdescShort = (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(BN >> 3) << 17) |
+                                            ((uint32_t)(128 >> 4) << 24);
 };
+
+// A pair tile whose rows [start, end) number at most 128 runs as M = 128.
+__device__ __forceinline__ bool short_pair_tile(int start, int end) { return end - start <= 128; }
 
 // Tiles of expert e cover rows [s_beg[e], s_end[e]) in blocks of rows_per_tile.
 __device__ __forceinline__ int count_tiles_rows(const int* s_beg, const int* s_end, int E, int n_tiles,
@@ -351,10 +370,12 @@ __device__ __forceinline__ bool wait_bounded_pair(uint32_t bar, uint32_t parity,
 
 template <int MODE, int CG, int BN, int RB>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
-grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB0,
-                    const __grid_constant__ CUtensorMap tmB1, const __grid_constant__ CUtensorMap tmOut,
-                    const KParams p) {
+grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmAs,
+                    const __grid_constant__ CUtensorMap tmB0, const __grid_constant__ CUtensorMap tmB1,
+                    const __grid_constant__ CUtensorMap tmOut, const KParams p) {
     using C = Cfg<CG, BN, RB>;
+    // pair up tiles interleave 64 rows of W1 and of W3 per CTA (N = 256)
+    static_assert(!(CG == 2 && MODE == kUp) || BN == 256, "pair up-projection tiles are 256 columns wide");
     constexpr int STG = C::kStages;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -423,19 +444,19 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
             for (int tile = tile0; tile < total && ok; tile += tstep) {
                 int e, mb, nb;
                 decode_tile_rows(tile, s_beg, s_end, p.E, p.n_tiles, C::kTileRows, e, mb, nb);
-                const int rowA = s_beg[e] + mb * C::kTileRows + (int)rank * 128;
+                const int start = s_beg[e] + mb * C::kTileRows;
+                const bool shrt = (CG == 2) && short_pair_tile(start, min(s_end[e], start + C::kTileRows));
+                const int rowA = start + (int)rank * (shrt ? 64 : 128);
                 int rowB0, rowB1;
-                const CUtensorMap* mapB = &tmB0;
                 if constexpr (CG == 1) {
                     rowB0 = e * p.b_rows_per_expert + nb * (MODE == kUp ? BN / 2 : BN);
                     rowB1 = (MODE == kUp) ? rowB0 : rowB0 + BN / 2;
+                } else if constexpr (MODE == kUp) {
+                    // this CTA's 64 hidden units: W1 rows, then the same W3 rows
+                    rowB0 = e * p.b_rows_per_expert + nb * (BN / 2) + (int)rank * (BN / 4);
+                    rowB1 = rowB0;
                 } else {
-                    if constexpr (MODE == kUp) {
-                        rowB0 = e * p.b_rows_per_expert + nb * (BN / 2);  // W1 rows (even CTA) or W3 rows (odd CTA)
-                        if (rank == 1) mapB = &tmB1;
-                    } else {
-                        rowB0 = e * p.b_rows_per_expert + nb * BN + (int)rank * (BN / 2);
-                    }
+                    rowB0 = e * p.b_rows_per_expert + nb * BN + (int)rank * (BN / 2);
                     rowB1 = rowB0;
                 }
                 for (int kb = 0; kb < kblocks; ++kb, ++it) {
@@ -449,9 +470,15 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
                         tma_load_2d(smem_u32(sB + s * C::kBBytes), &tmB0, fb, kb * BK, rowB0);
                         tma_load_2d(smem_u32(sB + s * C::kBBytes + C::kBHalf), &tmB1, fb, kb * BK, rowB1);
                     } else {
-                        if (leader) mbar_arrive_expect_tx(fb, 2 * C::kStageBytes);  // both CTAs' bytes
-                        tma_load_2d_pair(smem_u32(sA + s * A_TILE), &tmA, fb, kb * BK, rowA);
-                        tma_load_2d_pair(smem_u32(sB + s * C::kBBytes), mapB, fb, kb * BK, rowB0);
+                        // both CTAs' bytes are counted on the even CTA's barrier
+                        if (leader) mbar_arrive_expect_tx(fb, 2 * ((shrt ? C::kAShortBytes : A_TILE) + C::kBBytes));
+                        tma_load_2d_pair(smem_u32(sA + s * A_TILE), shrt ? &tmAs : &tmA, fb, kb * BK, rowA);
+                        if constexpr (MODE == kUp) {
+                            tma_load_2d_pair(smem_u32(sB + s * C::kBBytes), &tmB0, fb, kb * BK, rowB0);
+                            tma_load_2d_pair(smem_u32(sB + s * C::kBBytes + C::kBBytes / 2), &tmB1, fb, kb * BK, rowB1);
+                        } else {
+                            tma_load_2d_pair(smem_u32(sB + s * C::kBBytes), &tmB0, fb, kb * BK, rowB0);
+                        }
                     }
                 }
             }
@@ -479,6 +506,13 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
                 if (!wait_bounded_pair(smem_u32(&tempty[acc]), (use & 1u) ^ 1u, abort_flag, p.err, peer_abort)) break;
                 tc_fence_after();
                 const uint32_t d_tmem = tmem_base + acc * BN;
+                uint32_t idesc = C::kIdesc;
+                if constexpr (CG == 2) {
+                    int e, mb, nb;
+                    decode_tile_rows(tile, s_beg, s_end, p.E, p.n_tiles, C::kTileRows, e, mb, nb);
+                    const int start = s_beg[e] + mb * C::kTileRows;
+                    if (short_pair_tile(start, min(s_end[e], start + C::kTileRows))) idesc = C::kIdescShort;
+                }
                 for (int kb = 0; kb < kblocks; ++kb, ++it) {
                     const uint32_t s = it % STG;
                     const uint32_t ph = (it / STG) & 1u;
@@ -493,7 +527,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
                             umma_bf16(d_tmem, adesc + (uint64_t)(kk * 2), bdesc + (uint64_t)(kk * 2), C::kIdesc,
                                       (kb | kk) != 0 ? 1u : 0u);
                         else
-                            umma_bf16_pair(d_tmem, adesc + (uint64_t)(kk * 2), bdesc + (uint64_t)(kk * 2), C::kIdesc,
+                            umma_bf16_pair(d_tmem, adesc + (uint64_t)(kk * 2), bdesc + (uint64_t)(kk * 2), idesc,
                                            (kb | kk) != 0 ? 1u : 0u);
                     }
                     if constexpr (CG == 1) umma_commit(smem_u32(&empty[s])); else umma_commit_pair(smem_u32(&empty[s]));
@@ -507,7 +541,6 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
     } else {
         // ---------------------------------------------------- epilogue (both CTAs)
         const int quad = warp & 3;  // TMEM lanes 32*quad .. 32*quad+31
-        const int r_in = (int)rank * 128 + quad * 32 + lane;
         const uint32_t t_lane = tmem_base + ((uint32_t)(quad * 32) << 16);
         const uint32_t tempty_leader0 = (CG == 2) ? map_to_rank(smem_u32(&tempty[0]), 0) : 0u;
         const uint32_t out_base = smem_u32(sOut) + (uint32_t)quad * 2u * kOutBoxBytes;
@@ -523,8 +556,16 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
             const bool okw = wait_bounded_pair(smem_u32(&tfull[acc]), use & 1u, abort_flag, p.err, peer_abort);
             if (!__all_sync(0xffffffffu, okw)) break;
             tc_fence_after();
-            const int row = s_beg[e] + mb * C::kTileRows + r_in;
-            const int tile_end = min(s_end[e], s_beg[e] + (mb + 1) * C::kTileRows);
+            const int start = s_beg[e] + mb * C::kTileRows;
+            const int tile_end = min(s_end[e], start + C::kTileRows);
+            // Rows and accumulator columns of this warp's TMEM lanes.  Full
+            // tiles: 32 rows, all BN columns.  Short pair tiles: lanes 0-63
+            // hold the CTA's 64 rows for columns 0 .. BN/2-1 and lanes 64-127
+            // the same rows for BN/2 .. BN-1, so quads 0-1 take the first
+            // half of the columns and quads 2-3 the second.
+            const bool shrt = (CG == 2) && short_pair_tile(start, tile_end);
+            const int colhalf = shrt ? (quad >> 1) : 0;
+            const int row = start + (shrt ? (int)rank * 64 + (quad & 1) * 32 : (int)rank * 128 + quad * 32) + lane;
             const bool valid = row < tile_end;
             // rows of this warp: whole box stored by TMA when all 32 are the
             // expert's own; a box straddling the end of the expert's block
@@ -535,8 +576,17 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
             const uint32_t tacc = t_lane + acc * BN;
             if constexpr (MODE == kUp) {
                 __nv_bfloat16* hrow = p.h + (size_t)row * p.n_out;
+                // 64-unit segments: hidden units c64 .. c64+63 of the tile have
+                // a at TMEM columns acol .. acol+63 and b at acol+bdelta ...
+                //   single CTA: a = columns 0 .. BN/2-1, b = BN/2 .. BN-1;
+                //   pair, full: [a 64 | b 64] per CTA half of B, two halves;
+                //   pair, short: one half per lane group, at columns 0-127.
+                const int nseg = (CG == 1) ? BN / 128 : (shrt ? 1 : 2);
+                const int bdelta = (CG == 1) ? BN / 2 : 64;
 #pragma unroll 1
-                for (int c64 = 0; c64 < BN / 2; c64 += 64, ++obox) {
+                for (int seg = 0; seg < nseg; ++seg, ++obox) {
+                    const int c64 = (shrt ? colhalf : seg) * 64;        // hidden offset in the tile
+                    const int acol = (CG == 1) ? seg * 64 : (shrt ? 0 : seg * 128);
                     const uint32_t buf = out_base + (obox & 1u) * kOutBoxBytes;
                     if (box_ok) {
                         if (lane == 0) bulk_wait_read_le1();  // this buffer's previous store has read it
@@ -546,8 +596,8 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
                     for (int half = 0; half < 2; ++half) {
                         const int c = c64 + half * 32;
                         uint32_t a[32], b[32];
-                        tmem_ld32(tacc + c, a);
-                        tmem_ld32(tacc + BN / 2 + c, b);
+                        tmem_ld32(tacc + acol + half * 32, a);
+                        tmem_ld32(tacc + acol + half * 32 + bdelta, b);
                         tmem_wait_ld();
                         uint4 pk[4];
 #pragma unroll
@@ -590,15 +640,20 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
                     wgt = ((unsigned)q < (unsigned)p.rows) ? p.topk_w[q] : 0.f;
                 }
                 float* orow = p.obuf + (size_t)row * p.n_out;
+                // short pair tiles: this warp's lanes hold BN/2 columns,
+                // starting at output column colhalf * BN/2
+                const int ncol = shrt ? BN / 2 : BN;
+                const int cbase = colhalf * (BN / 2);
 #pragma unroll 1
-                for (int c = 0; c < BN; c += 32, ++obox) {
+                for (int cc = 0; cc < ncol; cc += 32, ++obox) {
+                    const int c = cbase + cc;  // tile column
                     const uint32_t buf = out_base + (obox & 1u) * kOutBoxBytes;
                     if (box_ok) {
                         if (lane == 0) bulk_wait_read_le1();
                         __syncwarp();
                     }
                     uint32_t o[32];
-                    tmem_ld32(tacc + c, o);
+                    tmem_ld32(tacc + cc, o);
                     tmem_wait_ld();
                     uint4 v[8];
 #pragma unroll
@@ -685,9 +740,18 @@ bool make_map(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols, ui
 
 // Co-resident persistent grid: CTAs (CG = 1) or CTA pairs (CG = 2) that
 // fit on the device at once, capped by an upper bound on the tile count.
+// Tensor maps of one GEMM: A with 128-, 32- and 64-row boxes (full tiles,
+// decode tiles, short pair tiles); B as single-CTA tiles read it (W1 / W3
+// halves of BN/2 rows, or W2 in 128-row boxes) and as pair tiles read it
+// (64-row W1 / W3 boxes; W2 unchanged); the output in 32-row boxes.
+struct GemmMaps {
+    CUtensorMap A, A32, A64, B0, B1, B0p, B1p, Out;
+};
+
 template <int MODE, int CG, int BN, int RB>
-cudaError_t launch_gemm(const GroupedGemmArgs& a, const CUtensorMap& mA, const CUtensorMap& mB0,
-                        const CUtensorMap& mB1, const CUtensorMap& mOut, const KParams& p, cudaStream_t s) {
+cudaError_t launch_gemm(const GroupedGemmArgs& a, const CUtensorMap& mA, const CUtensorMap& mAs,
+                        const CUtensorMap& mB0, const CUtensorMap& mB1, const CUtensorMap& mOut, const KParams& p,
+                        cudaStream_t s) {
     using C = Cfg<CG, BN, RB>;
     static int units_cache[64] = {0};
     int dev = 0;
@@ -726,10 +790,12 @@ cudaError_t launch_gemm(const GroupedGemmArgs& a, const CUtensorMap& mA, const C
     const int grid_units = (int)(ub < units ? ub : units);
     if (grid_units <= 0) return cudaSuccess;
     cfg.gridDim = dim3(grid_units * CG);
-    return cudaLaunchKernelEx(&cfg, grouped_gemm_kernel<MODE, CG, BN, RB>, mA, mB0, mB1, mOut, p);
+    return cudaLaunchKernelEx(&cfg, grouped_gemm_kernel<MODE, CG, BN, RB>, mA, mAs, mB0, mB1, mOut, p);
 }
 
 // Variant choice: 1 = single-CTA tiles, 2 = CTA-pair tiles, 3 = hybrid.
+// (Pair figures below are from before short pair tiles, when pairs padded
+// every expert to a multiple of 256 rows.)
 // Measured on B200 with Mixtral shapes:
 //  * pairs (M = 256) move a third fewer bytes per MMA from L2 and ran ~10%
 //    faster per row (one-expert 8192-row layer: up 1.34 vs 1.48 ms, down
@@ -786,21 +852,22 @@ int choose_rb(const GroupedGemmArgs& a) {
 }
 
 template <int MODE, int BN>
-cudaError_t launch_variant(const GroupedGemmArgs& a, const CUtensorMap& mA, const CUtensorMap& mA32,
-                           const CUtensorMap& mB0, const CUtensorMap& mB1, const CUtensorMap& mOut, const KParams& p,
-                           cudaStream_t s) {
-    const int cg = choose_cta_group(a, MODE);
-    if (cg == 2) return launch_gemm<MODE, 2, BN, 128>(a, mA, mB0, mB1, mOut, p, s);
-    if (cg == 3) {  // hybrid: pairs on whole 256-row blocks, then single CTAs on the rest (same stream)
-        KParams pf = p, pr = p;
-        pf.row_mode = kFullPairBlocks;
-        pr.row_mode = kPairRemainders;
-        cudaError_t e = launch_gemm<MODE, 2, BN, 128>(a, mA, mB0, mB1, mOut, pf, s);
-        if (e != cudaSuccess) return e;
-        return launch_gemm<MODE, 1, BN, 128>(a, mA, mB0, mB1, mOut, pr, s);
+cudaError_t launch_variant(const GroupedGemmArgs& a, const GemmMaps& m, const KParams& p, cudaStream_t s) {
+    // pairs: 256-column tiles only (the up-projection's interleaved B halves)
+    const int cg = (MODE == kUp && BN != 256) ? 1 : choose_cta_group(a, MODE);
+    if constexpr (MODE == kDown || BN == 256) {
+        if (cg == 2) return launch_gemm<MODE, 2, BN, 128>(a, m.A, m.A64, m.B0p, m.B1p, m.Out, p, s);
+        if (cg == 3) {  // hybrid: pairs on whole 256-row blocks, then single CTAs on the rest (same stream)
+            KParams pf = p, pr = p;
+            pf.row_mode = kFullPairBlocks;
+            pr.row_mode = kPairRemainders;
+            cudaError_t e = launch_gemm<MODE, 2, BN, 128>(a, m.A, m.A64, m.B0p, m.B1p, m.Out, pf, s);
+            if (e != cudaSuccess) return e;
+            return launch_gemm<MODE, 1, BN, 128>(a, m.A, m.A, m.B0, m.B1, m.Out, pr, s);
+        }
     }
-    return choose_rb(a) == 32 ? launch_gemm<MODE, 1, BN, 32>(a, mA32, mB0, mB1, mOut, p, s)
-                              : launch_gemm<MODE, 1, BN, 128>(a, mA, mB0, mB1, mOut, p, s);
+    return choose_rb(a) == 32 ? launch_gemm<MODE, 1, BN, 32>(a, m.A32, m.A32, m.B0, m.B1, m.Out, p, s)
+                              : launch_gemm<MODE, 1, BN, 128>(a, m.A, m.A, m.B0, m.B1, m.Out, p, s);
 }
 
 }  // namespace
@@ -808,37 +875,44 @@ cudaError_t launch_variant(const GroupedGemmArgs& a, const CUtensorMap& mA, cons
 cudaError_t launch_up_swiglu(const GroupedGemmArgs& a, const __nv_bfloat16* x_perm,
                              const __nv_bfloat16* W1, const __nv_bfloat16* W3, __nv_bfloat16* h,
                              cudaStream_t s) {
-    const int bn = choose_up_bn(a);
-    CUtensorMap mA, mA32, mB0, mB1, mOut;
-    if (!make_map(&mA, x_perm, (uint64_t)a.rows, (uint64_t)a.d, BM) ||
-        !make_map(&mA32, x_perm, (uint64_t)a.rows, (uint64_t)a.d, 32) ||
-        !make_map(&mB0, W1, (uint64_t)a.E * a.f, (uint64_t)a.d, bn / 2) ||
-        !make_map(&mB1, W3, (uint64_t)a.E * a.f, (uint64_t)a.d, bn / 2) ||
-        !make_map(&mOut, h, (uint64_t)a.rows, (uint64_t)a.f, 32))
+    // pairs and the hybrid use 256-column tiles whatever MOE_GEMM_BN says
+    const int bn = choose_cta_group(a, kUp) == 1 ? choose_up_bn(a) : 256;
+    GemmMaps m;
+    if (!make_map(&m.A, x_perm, (uint64_t)a.rows, (uint64_t)a.d, BM) ||
+        !make_map(&m.A32, x_perm, (uint64_t)a.rows, (uint64_t)a.d, 32) ||
+        !make_map(&m.A64, x_perm, (uint64_t)a.rows, (uint64_t)a.d, 64) ||
+        !make_map(&m.B0, W1, (uint64_t)a.E * a.f, (uint64_t)a.d, bn / 2) ||
+        !make_map(&m.B1, W3, (uint64_t)a.E * a.f, (uint64_t)a.d, bn / 2) ||
+        !make_map(&m.B0p, W1, (uint64_t)a.E * a.f, (uint64_t)a.d, 64) ||
+        !make_map(&m.B1p, W3, (uint64_t)a.E * a.f, (uint64_t)a.d, 64) ||
+        !make_map(&m.Out, h, (uint64_t)a.rows, (uint64_t)a.f, 32))
         return cudaErrorInvalidValue;
     KParams p{};
     p.offsets = a.offsets; p.E = a.E; p.n_out = a.f; p.Kdim = a.d;
     p.n_tiles = (a.f + bn / 2 - 1) / (bn / 2); p.b_rows_per_expert = a.f; p.h = h; p.rows = a.rows;
     p.err = a.err;
-    return bn == 128 ? launch_variant<kUp, 128>(a, mA, mA32, mB0, mB1, mOut, p, s)
-                     : launch_variant<kUp, 256>(a, mA, mA32, mB0, mB1, mOut, p, s);
+    return bn == 128 ? launch_variant<kUp, 128>(a, m, p, s) : launch_variant<kUp, 256>(a, m, p, s);
 }
 
 cudaError_t launch_down_scaled(const GroupedGemmArgs& a, const __nv_bfloat16* h,
                                const __nv_bfloat16* W2, const int32_t* perm, const float* topk_w,
                                float* obuf, cudaStream_t s) {
-    CUtensorMap mA, mA32, mB, mOut;
-    if (!make_map(&mA, h, (uint64_t)a.rows, (uint64_t)a.f, BM) ||
-        !make_map(&mA32, h, (uint64_t)a.rows, (uint64_t)a.f, 32) ||
-        !make_map(&mB, W2, (uint64_t)a.E * a.d, (uint64_t)a.f, 128) ||
-        !make_map(&mOut, obuf, (uint64_t)a.rows, (uint64_t)a.d, 32, true))
+    GemmMaps m;
+    if (!make_map(&m.A, h, (uint64_t)a.rows, (uint64_t)a.f, BM) ||
+        !make_map(&m.A32, h, (uint64_t)a.rows, (uint64_t)a.f, 32) ||
+        !make_map(&m.A64, h, (uint64_t)a.rows, (uint64_t)a.f, 64) ||
+        !make_map(&m.B0, W2, (uint64_t)a.E * a.d, (uint64_t)a.f, 128) ||
+        !make_map(&m.Out, obuf, (uint64_t)a.rows, (uint64_t)a.d, 32, true))
         return cudaErrorInvalidValue;
+    m.B1 = m.B0;
+    m.B0p = m.B0;
+    m.B1p = m.B0;
     KParams p{};
     p.offsets = a.offsets; p.E = a.E; p.n_out = a.d; p.Kdim = a.f;
     p.n_tiles = (a.d + 255) / 256; p.b_rows_per_expert = a.d;
     p.perm = perm; p.topk_w = topk_w; p.obuf = obuf; p.rows = a.rows;
     p.err = a.err;
-    return launch_variant<kDown, 256>(a, mA, mA32, mB, mB, mOut, p, s);
+    return launch_variant<kDown, 256>(a, m, p, s);
 }
 
 }  // namespace moe

@@ -176,21 +176,51 @@ def test_layer_parity_every_token_f32(shape):
 
 
 GEMM_VARIANTS = [("1", "256", "128"), ("1", "128", "128"), ("1", "256", "32"), ("1", "128", "32"),
-                 ("2", "256", "128"), ("2", "128", "128"), ("h", "256", "128"), ("h", "128", "128")]
+                 ("2", "256", "128"), ("h", "256", "128")]
 
 
 @pytest.mark.parametrize("variant", GEMM_VARIANTS, ids=lambda v: "cg%s-bn%s-rb%s" % v)
 @pytest.mark.parametrize("shape", BF16_SHAPES, ids=lambda s: s.name)
 def test_layer_parity_every_token_bf16(shape, variant, monkeypatch):
     """Every GEMM variant: single-CTA tiles of 128 or 32 token rows, CTA-pair
-    256-row tiles, the hybrid (pairs on whole 256-row blocks, single CTAs on
-    the rest), and 256- or 128-column up-projection tiles."""
+    tiles (256 rows, or 128 for an expert's short last block), the hybrid
+    (pairs on whole 256-row blocks, single CTAs on the rest), and 256- or
+    128-column up-projection tiles (pairs always use 256)."""
     cta_group, bn, rb = variant
     monkeypatch.setenv("MOE_GEMM_CTA_GROUP", cta_group)
     monkeypatch.setenv("MOE_GEMM_BN", bn)
     monkeypatch.setenv("MOE_GEMM_RB", rb)
     rel, _ = full_check(shape)
     assert rel <= 1e-2
+
+
+# Expert block sizes around every tile edge: pair tiles are 256 rows, or 128
+# (an M = 128 pair MMA, 64 rows per CTA) when an expert's last block holds at
+# most 128 rows; single-CTA tiles are 128 rows.
+BLOCK_SIZES = [1, 64, 65, 128, 129, 200, 384, 385]
+
+
+@pytest.mark.parametrize("cta_group", ["1", "2", "h"])
+def test_expert_blocks_at_tile_edges(cta_group, monkeypatch):
+    """moe_expert_ffn on a routing built to give the experts the block sizes
+    above (k = 1, tokens shuffled, arbitrary gate weights), ragged in both
+    output widths (f = 320, d = 384), against the oracle on every token."""
+    monkeypatch.setenv("MOE_GEMM_CTA_GROUP", cta_group)
+    E, d, f = len(BLOCK_SIZES), 384, 320
+    T = sum(BLOCK_SIZES)
+    s = synth.MoEShape("blocks", T, d, f, E, 1, "bf16")
+    t = device_inputs(s, 11)
+    rng = np.random.default_rng(5)
+    idx = rng.permutation(np.repeat(np.arange(E), BLOCK_SIZES)).astype(np.int32).reshape(T, 1)
+    w = rng.uniform(0.25, 1.0, size=(T, 1)).astype(np.float32)
+    idx_d = torch.from_numpy(idx).cuda()
+    w_d = torch.from_numpy(w).cuda()
+    off, perm, inv = moe.moe_permute(idx_d, E)
+    assert np.diff(off.cpu().numpy()).tolist() == BLOCK_SIZES
+    y = moe.moe_expert_ffn(t["x"], t["W1"], t["W3"], t["W2"], off, perm, inv, w_d)
+    h = host_copy(t)
+    y_ref, _, _ = oracle_rows(h, 1, np.arange(T), routing=(idx, w.astype(np.float64)))
+    assert_close(to64(y), y_ref, "bf16")
 
 
 @pytest.mark.parametrize("seed", range(1, 21))
