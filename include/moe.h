@@ -73,7 +73,8 @@ enum {
 /* Bytes of device workspace needed by moe_layer_forward_ex and moe_expert_ffn
  * for this shape (0 for invalid arguments).  Holds the routing result, the
  * permutation, the expert-ordered copy of x, the hidden activations h
- * [T*k, f] and the gate-scaled expert outputs [T*k, d] (fp32). */
+ * [T*k, f], the gate-scaled expert outputs [T*k, d] (fp32) and the expert
+ * GEMMs' tile counters.  No contents need to survive between calls. */
 size_t moe_workspace_size(int T, int d, int f, int E, int k, int dtype);
 
 /* Router and top-k gate ("Mixtral of Experts" §2.1 display 2; Method, steps

@@ -35,7 +35,11 @@
 // Tiles are enumerated per expert from the device-side offsets (no host
 // round trip): expert e owns ceil(M_e / tile rows) row blocks x n_tiles column
 // blocks, numbered with the row block fastest so that the CTAs running at
-// the same time share weight tiles through L2.  Ragged row blocks read the
+// the same time share weight tiles through L2.  Tiles are handed out
+// dynamically: the producer (the even CTA's, for pairs) takes the next tile
+// number from a global counter and passes it to the other roles (and to the
+// odd CTA) through a small shared-memory ring, so short and full tiles
+// balance across the persistent CTAs.  Ragged row blocks read the
 // next expert's rows (or the zero fill past the end) and simply do not
 // store them; ragged column blocks are masked the same way.
 //
@@ -79,6 +83,7 @@ struct KParams {
     int rows;                // T*k
     unsigned int* err;       // device error word (MOE_DEVERR_*)
     int row_mode;            // rows of each expert to cover: kAllRows, kFullPairBlocks or kPairRemainders
+    int* tile_counter;       // next tile to hand out; zero at launch (the row gather zeroes it)
 };
 
 // Row ranges: all rows of each expert; only its whole 256-row blocks; or
@@ -108,6 +113,20 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
     asm volatile(
         "{\n\t.reg .pred p;\n\t"
         "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}\n"
+        : "=r"(ok)
+        : "r"(bar), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+
+// try_wait with cluster-scope acquire: for barriers completed by the other
+// CTA of a pair, whose shared-memory writes must be visible after the wait.
+__device__ __forceinline__ bool mbar_try_wait_cluster(uint32_t bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
         "selp.u32 %0, 1, 0, p;\n\t}\n"
         : "=r"(ok)
         : "r"(bar), "r"(parity)
@@ -348,11 +367,12 @@ __device__ __forceinline__ void decode_tile_rows(int tile, const int* s_beg, con
 // clock are consulted only every 1024 tries, so a phase that completes
 // while the waiter spins is seen within one try (a timer read costs
 // hundreds of cycles, which would delay the next MMA issue).
+template <bool kClusterScope = false>
 __device__ __forceinline__ bool wait_bounded_pair(uint32_t bar, uint32_t parity, volatile int* abort_flag,
                                                   unsigned int* err, uint32_t peer_abort_addr) {
     unsigned long long t0 = 0;
     for (uint32_t i = 1;; ++i) {
-        if (mbar_try_wait(bar, parity)) return true;
+        if (kClusterScope ? mbar_try_wait_cluster(bar, parity) : mbar_try_wait(bar, parity)) return true;
         if ((i & 1023u) == 0) {
             if (*abort_flag) return false;
             const unsigned long long now = globaltimer();
@@ -367,6 +387,18 @@ __device__ __forceinline__ bool wait_bounded_pair(uint32_t bar, uint32_t parity,
         }
     }
 }
+
+// Tile-number ring between the producer that takes tiles from the global
+// counter and the roles that follow it.  Readers of a slot: the MMA thread
+// and the 4 epilogue warps of the CTA, and for pairs also the odd CTA's
+// producer and its 4 epilogue warps (they read the copy the even CTA's
+// producer writes into the odd CTA's ring).  The slot's empty barrier lives
+// in the even CTA.  A tile number of -1 ends the loops.
+constexpr int kSchedSlots = 4;
+template <int CG>
+struct Sched {
+    static constexpr uint32_t kReaders = (CG == 1) ? 5u : 10u;
+};
 
 template <int MODE, int CG, int BN, int RB>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
@@ -387,7 +419,10 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
     uint64_t* empty = bars + STG;
     uint64_t* tfull = bars + 2 * STG;
     uint64_t* tempty = bars + 2 * STG + 2;
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * STG + 4);
+    uint64_t* sfull = bars + 2 * STG + 4;                 // [kSchedSlots] tile number published
+    uint64_t* sempty = sfull + kSchedSlots;               // [kSchedSlots] all readers done (even CTA)
+    volatile int* stile = reinterpret_cast<volatile int*>(sempty + kSchedSlots);  // [kSchedSlots]
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sempty + kSchedSlots) + kSchedSlots;
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
     int* s_beg = reinterpret_cast<int*>(tmem_slot + 2);  // [E] first row of expert e's range
     int* s_end = s_beg + kMaxExperts;                   // [E] end of expert e's range
@@ -405,6 +440,10 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
         for (int a = 0; a < 2; ++a) {
             mbar_init(smem_u32(&tfull[a]), 1);
             mbar_init(smem_u32(&tempty[a]), 4 * CG);  // one arrival per epilogue warp of the tile
+        }
+        for (int q = 0; q < kSchedSlots; ++q) {
+            mbar_init(smem_u32(&sfull[q]), 1);
+            mbar_init(smem_u32(&sempty[q]), Sched<CG>::kReaders);
         }
         *abort_flag = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
@@ -433,15 +472,52 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
 
     const int total = count_tiles_rows(s_beg, s_end, p.E, p.n_tiles, C::kTileRows);
     const int kblocks = (p.Kdim + BK - 1) / BK;
-    const int tile0 = (CG == 2) ? (int)(blockIdx.x >> 1) : (int)blockIdx.x;
-    const int tstep = (CG == 2) ? (int)(gridDim.x >> 1) : (int)gridDim.x;
+    // a reader of tile-ring slot i: wait for the number, read it, release the slot
+    const uint32_t sempty_leader0 = (CG == 2) ? map_to_rank(smem_u32(&sempty[0]), 0) : smem_u32(&sempty[0]);
+    auto read_tile = [&](uint32_t i, bool& ok) -> int {
+        const uint32_t q = i % kSchedSlots, ph = (i / kSchedSlots) & 1u;
+        if (!wait_bounded_pair<CG == 2>(smem_u32(&sfull[q]), ph, abort_flag, p.err, peer_abort)) {
+            ok = false;
+            return -1;
+        }
+        return stile[q];
+    };
+    auto release_tile = [&](uint32_t i) {
+        const uint32_t q = i % kSchedSlots;
+        if constexpr (CG == 2) mbar_arrive_cluster(sempty_leader0 + q * (uint32_t)sizeof(uint64_t));
+        else mbar_arrive(smem_u32(&sempty[q]));
+    };
 
     if (warp == 0) {
         if (lane == 0) {
             // ------------------------------------------------ TMA producer (both CTAs)
             uint32_t it = 0;
             bool ok = true;
-            for (int tile = tile0; tile < total && ok; tile += tstep) {
+            // The next tile's number is taken while the last STG stages of the
+            // current tile are issued, so the atomic's latency is hidden.
+            int next = leader ? atomicAdd(p.tile_counter, 1) : -1;  // the odd CTA of a pair reads the even one's
+            for (uint32_t ti = 0; ok; ++ti) {
+                int tile;
+                if (leader) {
+                    // publish the tile taken (to both CTAs of a pair)
+                    const uint32_t q = ti % kSchedSlots, ph = (ti / kSchedSlots) & 1u;
+                    if (!wait_bounded_pair<CG == 2>(smem_u32(&sempty[q]), ph ^ 1u, abort_flag, p.err, peer_abort)) {
+                        ok = false;
+                        break;
+                    }
+                    tile = next < total ? next : -1;
+                    stile[q] = tile;
+                    if constexpr (CG == 2) {
+                        st_cluster_u32(map_to_rank(smem_u32((const void*)&stile[q]), 1), (uint32_t)tile);
+                        mbar_arrive_cluster(map_to_rank(smem_u32(&sfull[q]), 1));
+                    }
+                    mbar_arrive(smem_u32(&sfull[q]));
+                } else {
+                    tile = read_tile(ti, ok);
+                    if (!ok) break;
+                    release_tile(ti);
+                }
+                if (tile < 0) break;
                 int e, mb, nb;
                 decode_tile_rows(tile, s_beg, s_end, p.E, p.n_tiles, C::kTileRows, e, mb, nb);
                 const int start = s_beg[e] + mb * C::kTileRows;
@@ -459,7 +535,9 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
                     rowB0 = e * p.b_rows_per_expert + nb * BN + (int)rank * (BN / 2);
                     rowB1 = rowB0;
                 }
+                const int kb_next = kblocks > STG ? kblocks - STG : 0;
                 for (int kb = 0; kb < kblocks; ++kb, ++it) {
+                    if (leader && kb == kb_next) next = atomicAdd(p.tile_counter, 1);
                     const uint32_t s = it % STG;
                     const uint32_t ph = (it / STG) & 1u;
                     if (!wait_bounded_pair(smem_u32(&empty[s]), ph ^ 1u, abort_flag, p.err, peer_abort)) { ok = false; break; }
@@ -500,7 +578,11 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
             // ------------------------------------------------ MMA issuer (even CTA)
             uint32_t it = 0, tcount = 0;
             bool ok = true;
-            for (int tile = tile0; tile < total && ok; tile += tstep, ++tcount) {
+            for (;; ++tcount) {
+                const int tile = read_tile(tcount, ok);
+                if (!ok) break;
+                release_tile(tcount);
+                if (tile < 0) break;
                 const uint32_t acc = tcount & 1u;
                 const uint32_t use = tcount >> 1;
                 if (!wait_bounded_pair(smem_u32(&tempty[acc]), (use & 1u) ^ 1u, abort_flag, p.err, peer_abort)) break;
@@ -546,7 +628,13 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
         const uint32_t out_base = smem_u32(sOut) + (uint32_t)quad * 2u * kOutBoxBytes;
         uint32_t obox = 0;  // boxes this warp has staged (selects the buffer)
         uint32_t tcount = 0;
-        for (int tile = tile0; tile < total; tile += tstep, ++tcount) {
+        for (;; ++tcount) {
+            bool got = true;
+            const int tile = read_tile(tcount, got);  // every lane waits and reads
+            __syncwarp();
+            if (!__all_sync(0xffffffffu, got)) break;
+            if (lane == 0) release_tile(tcount);
+            if (tile < 0) break;
             int e, mb, nb;
             decode_tile_rows(tile, s_beg, s_end, p.E, p.n_tiles, C::kTileRows, e, mb, nb);
             const uint32_t acc = tcount & 1u;
@@ -861,6 +949,7 @@ cudaError_t launch_variant(const GroupedGemmArgs& a, const GemmMaps& m, const KP
             KParams pf = p, pr = p;
             pf.row_mode = kFullPairBlocks;
             pr.row_mode = kPairRemainders;
+            pr.tile_counter = p.tile_counter + 1;  // the second launch has its own counter
             cudaError_t e = launch_gemm<MODE, 2, BN, 128>(a, m.A, m.A64, m.B0p, m.B1p, m.Out, pf, s);
             if (e != cudaSuccess) return e;
             return launch_gemm<MODE, 1, BN, 128>(a, m.A, m.A, m.B0, m.B1, m.Out, pr, s);
@@ -891,6 +980,7 @@ cudaError_t launch_up_swiglu(const GroupedGemmArgs& a, const __nv_bfloat16* x_pe
     p.offsets = a.offsets; p.E = a.E; p.n_out = a.f; p.Kdim = a.d;
     p.n_tiles = (a.f + bn / 2 - 1) / (bn / 2); p.b_rows_per_expert = a.f; p.h = h; p.rows = a.rows;
     p.err = a.err;
+    p.tile_counter = a.tile_counters + 0;
     return bn == 128 ? launch_variant<kUp, 128>(a, m, p, s) : launch_variant<kUp, 256>(a, m, p, s);
 }
 
@@ -912,6 +1002,7 @@ cudaError_t launch_down_scaled(const GroupedGemmArgs& a, const __nv_bfloat16* h,
     p.n_tiles = (a.d + 255) / 256; p.b_rows_per_expert = a.d;
     p.perm = perm; p.topk_w = topk_w; p.obuf = obuf; p.rows = a.rows;
     p.err = a.err;
+    p.tile_counter = a.tile_counters + 2;
     return launch_variant<kDown, 256>(a, m, p, s);
 }
 

@@ -98,6 +98,7 @@ Workspace carve_workspace(void* base, int T, int d, int f, int E, int k, bool bf
     w.x_perm = bf16 ? take(n * d * 2) : nullptr;
     w.h = take(n * f * (bf16 ? 2 : 4));
     w.obuf = reinterpret_cast<float*>(take(n * d * 4));
+    w.tile_counters = reinterpret_cast<int32_t*>(take(kTileCounters * 4));
     w.bytes = off;
     return w;
 }
@@ -151,13 +152,13 @@ int run_ffn(const void* x, const void* W1, const void* W3, const void* W2, const
         {
             StageTimer tm(kGather, s);
             e = moe::launch_gather_rows_bf16(static_cast<const __nv_bfloat16*>(x), perm, rows, d, k,
-                                             static_cast<__nv_bfloat16*>(w.x_perm), s);
+                                             static_cast<__nv_bfloat16*>(w.x_perm), w.tile_counters, s);
             tm.done(s);
         }
         if (e != cudaSuccess) return cuda_fail(e, "gather_rows");
         unsigned int* err = moe::device_error_word();
         if (!err) return fail(MOE_ERR_CUDA, "cannot locate the device error word");
-        moe::GroupedGemmArgs a{offsets, E, rows, d, f, num_sms_current(), err};
+        moe::GroupedGemmArgs a{offsets, E, rows, d, f, num_sms_current(), err, w.tile_counters};
         {
             StageTimer tm(kUp, s);
             e = moe::launch_up_swiglu(a, static_cast<const __nv_bfloat16*>(w.x_perm),

@@ -17,6 +17,7 @@ void set_last_error(const char* msg);
 
 constexpr int kMaxExperts = 64;
 constexpr int kMaxTopK = kMaxExperts;  // any k <= E
+constexpr int kTileCounters = 4;        // up, up (second hybrid launch), down, down (second)
 
 // 256-byte aligned carve-up of one workspace blob.
 struct Workspace {
@@ -28,6 +29,7 @@ struct Workspace {
     void* x_perm;       // [T*k, d]  bf16 path only
     void* h;            // [T*k, f]  bf16 or f32
     float* obuf;        // [T*k, d]  gate-scaled expert outputs, fp32
+    int32_t* tile_counters;  // [kTileCounters] GEMM tile schedulers, zeroed by the row gather
     size_t bytes;
 };
 
@@ -38,8 +40,10 @@ cudaError_t launch_router_topk(const void* x, const void* Wg, int T, int d, int 
                                bool bf16, int32_t* idx, float* w, cudaStream_t s);
 cudaError_t launch_permute(const int32_t* idx, int n, int E, int32_t* offsets, int32_t* perm,
                            int32_t* inv, cudaStream_t s);
+// Also zeroes tile_counters[0 .. kTileCounters) for the GEMMs that follow on
+// the same stream.
 cudaError_t launch_gather_rows_bf16(const __nv_bfloat16* x, const int32_t* perm, int rows, int d,
-                                    int k, __nv_bfloat16* x_perm, cudaStream_t s);
+                                    int k, __nv_bfloat16* x_perm, int32_t* tile_counters, cudaStream_t s);
 cudaError_t launch_combine(const float* obuf, const int32_t* inv, const void* residual, int T,
                            int d, int k, bool bf16, void* y, cudaStream_t s);
 
@@ -53,6 +57,7 @@ struct GroupedGemmArgs {
     int d, f;
     int num_sms;
     unsigned int* err;       // device error word
+    int32_t* tile_counters;  // [kTileCounters], zero at the up-projection's launch
 };
 cudaError_t launch_up_swiglu(const GroupedGemmArgs& a, const __nv_bfloat16* x_perm,
                              const __nv_bfloat16* W1, const __nv_bfloat16* W3, __nv_bfloat16* h,

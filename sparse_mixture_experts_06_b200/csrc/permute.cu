@@ -102,7 +102,8 @@ constexpr int kUnroll = 4;
 // x_perm[r, :] = x[perm[r] / k, :]  (a row with an invalid assignment id is zero)
 __global__ void __launch_bounds__(kFlatThreads)
 gather_rows_kernel(const __nv_bfloat16* __restrict__ x, const int32_t* __restrict__ perm, int rows,
-                   int d, int k, __nv_bfloat16* __restrict__ xp) {
+                   int d, int k, __nv_bfloat16* __restrict__ xp, int32_t* __restrict__ tile_counters) {
+    if (blockIdx.x == 0 && threadIdx.x < kTileCounters) tile_counters[threadIdx.x] = 0;
     const int nvec = d / 8;
     for (int r = blockIdx.x; r < rows; r += gridDim.x) {
         const int q = __ldg(perm + r);
@@ -240,8 +241,8 @@ cudaError_t launch_permute(const int32_t* idx, int n, int E, int32_t* offsets, i
 }
 
 cudaError_t launch_gather_rows_bf16(const __nv_bfloat16* x, const int32_t* perm, int rows, int d,
-                                    int k, __nv_bfloat16* x_perm, cudaStream_t s) {
-    gather_rows_kernel<<<flat_grid(rows), kFlatThreads, 0, s>>>(x, perm, rows, d, k, x_perm);
+                                    int k, __nv_bfloat16* x_perm, int32_t* tile_counters, cudaStream_t s) {
+    gather_rows_kernel<<<flat_grid(rows), kFlatThreads, 0, s>>>(x, perm, rows, d, k, x_perm, tile_counters);
     return cudaGetLastError();
 }
 
