@@ -54,6 +54,8 @@ def parse():
                     help="tokens in the oracle's timed CPU-baseline sample (default: the whole prefill batch)")
     ap.add_argument("--ref-sample", type=int, default=128,
                     help="tokens per step of --impl reference (keeps --steps K --warmup W within minutes)")
+    ap.add_argument("--e2e-chunks", type=int, default=2,
+                    help="pieces the end-to-end leg pipelines host copies and compute in")
     ap.add_argument("--gemm-vs-cublas", action="store_true",
                     help="instead of the layer: time the two expert GEMMs against cuBLAS (torch.matmul) "
                          "on the same shapes and print one JSON line")
@@ -367,21 +369,19 @@ def graph_step_ms(r, s, device, steps):
 
 
 def e2e_leg(args, s, t, device, steps):
-    """Same layer through the public entry point moe_layer_forward (library
-    workspace), with the step's tokens copied in from pinned host memory and
-    the output copied back, all inside the timed region."""
+    """Same layer through the public host-buffer entry point
+    moe_layer_forward_host: the step's tokens come from pinned host memory
+    and the output goes back to it, copies pipelined with the compute in
+    args.e2e_chunks pieces, all inside the timed region."""
     import torch
     import sparse_mixture_experts_06_b200 as moe
     x_h = t["x"].cpu().pin_memory()
     y_h = torch.empty_like(x_h).pin_memory()
-    x_d = torch.empty_like(t["x"])
-    y_d = torch.empty_like(t["x"])
     stream = torch.cuda.current_stream(device)
 
     def step():
-        x_d.copy_(x_h, non_blocking=True)
-        moe.moe_layer_forward(x_d, t["Wg"], t["W1"], t["W3"], t["W2"], s.k, y=y_d, stream=stream)
-        y_h.copy_(y_d, non_blocking=True)
+        moe.moe_layer_forward_host(x_h, t["Wg"], t["W1"], t["W3"], t["W2"], s.k, y=y_h, chunks=args.e2e_chunks,
+                                   stream=stream)
 
     for _ in range(3):
         step()
@@ -558,11 +558,16 @@ def main():
     if r["clocks"]:
         line["clocks"] = r["clocks"]
 
+    # every rank runs the host-buffer path on its own tokens; max over ranks
+    if dist is not None:
+        dist.barrier()
+    e_ms, hb, db = e2e_leg(args, s, r["t"], device, max(10, min(K, 100)))
+    e_ms = max_over_ranks(e_ms, dist, device)
     if rank == 0:
-        e_ms, hb, db = e2e_leg(args, s, r["t"], device, max(10, min(K, 100)))
         line["e2e"] = {"value": world * s.T / (e_ms * 1e-3), "unit": "tokens/s", "h2d_bytes_per_step": hb,
-                       "d2h_bytes_per_step": db, "ms_per_step": e_ms,
-                       "path": "pinned host x -> moe_layer_forward (library workspace) -> pinned host y"}
+                       "d2h_bytes_per_step": db, "ms_per_step": e_ms, "chunks": args.e2e_chunks,
+                       "path": "pinned host x -> moe_layer_forward_host (copies pipelined with the layer "
+                               "in %d pieces) -> pinned host y" % args.e2e_chunks}
     del r
     torch.cuda.empty_cache()
 

@@ -39,8 +39,8 @@
  *    are those of the exact logits except within ~1e-13 relative near-ties.
  *  - Thread safety: calls on different streams may run concurrently when
  *    each uses its own workspace (moe_layer_forward_ex); moe_layer_forward
- *    shares one library-owned workspace per device and must not be called
- *    concurrently on two streams of one device.
+ *    and moe_layer_forward_host share one library-owned workspace per device
+ *    and must not be called concurrently on two streams of one device.
  */
 #ifndef MOE_B200_H
 #define MOE_B200_H
@@ -127,6 +127,23 @@ int moe_expert_ffn(const void* x, const void* W1, const void* W3, const void* W2
 int moe_layer_forward(const void* x, const void* Wg, const void* W1, const void* W3,
                       const void* W2, int T, int d, int f, int E, int k, void* y,
                       moe_stream_t stream);
+
+/* The bf16 layer on HOST x and y [T, d] (the serving entry: tokens arrive in
+ * and leave host memory).  The T tokens are processed in `chunks` pieces of
+ * ceil(T / chunks) tokens (chunks >= 1; tokens are independent, so the
+ * result does not depend on the split): while piece c runs on `stream`, the
+ * rows of piece c+1 are copied in and those of piece c-1 copied out on two
+ * library-owned copy streams, ordered with events against `stream`.  The
+ * device staging buffers (2 x and 2 y pieces) share the library workspace
+ * of moe_layer_forward.  Weights are device pointers as elsewhere; x_host
+ * and y_host need no alignment, and copies overlap only if they are
+ * page-locked (cudaHostAlloc / cudaHostRegister).  Asynchronous like the
+ * other calls: y_host is complete once `stream` has been synchronised.
+ * Pipelining of host copies with compute has no counterpart in the pages;
+ * the layer itself is the one moe_layer_forward computes. */
+int moe_layer_forward_host(const void* x_host, const void* Wg, const void* W1, const void* W3,
+                           const void* W2, int T, int d, int f, int E, int k, void* y_host,
+                           int chunks, moe_stream_t stream);
 
 /* As moe_layer_forward with an explicit dtype and a caller-owned workspace.
  * If `residual` is not NULL it must be a [T, d] tensor of the same dtype and

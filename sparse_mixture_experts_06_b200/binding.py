@@ -27,6 +27,7 @@ _SIGS = {
     "moe_expert_ffn": ([_P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _P, _Z, _P, _P], _I),
     "moe_layer_forward": ([_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _P, _P], _I),
     "moe_layer_forward_ex": ([_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _P, _Z, _P, _P], _I),
+    "moe_layer_forward_host": ([_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _P, _I, _P], _I),
     "moe_layer_forward_noalloc": ([_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _P, _P], _I),
     "moe_stack_forward": ([_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _P, _P, _Z, _P, _P], _I),
     "moe_release_workspace": ([_P], _I),
@@ -192,6 +193,25 @@ def moe_layer_forward(x, Wg, W1, W3, W2, k, y=None, stream=None):
     y = torch.empty_like(x) if y is None else y
     _check(lib.moe_layer_forward(_ptr(x), _ptr(Wg), _ptr(W1), _ptr(W3), _ptr(W2), T, d, f, E, k, _ptr(y),
                                  _stream(stream, x)), "moe_layer_forward")
+    return y
+
+
+def moe_layer_forward_host(x, Wg, W1, W3, W2, k, y=None, chunks=2, stream=None):
+    """The bf16 layer on host x / y (CPU tensors; page-locked for overlap),
+    pipelined in `chunks` pieces; returns y (a pinned CPU tensor unless given).
+    Asynchronous: synchronise `stream` (default: the current stream of W1's
+    device) before reading y."""
+    import torch
+    _dev(Wg, W1, W3, W2)
+    if x.is_cuda or not x.is_contiguous() or x.dtype != torch.bfloat16:
+        raise ValueError("x must be a contiguous bfloat16 CPU tensor")
+    T, d = x.shape
+    E, f, _ = W1.shape
+    y = torch.empty((T, d), dtype=torch.bfloat16, pin_memory=True) if y is None else y
+    if y.is_cuda or not y.is_contiguous() or y.dtype != torch.bfloat16 or tuple(y.shape) != (T, d):
+        raise ValueError("y must be a contiguous bfloat16 CPU tensor of shape [T, d]")
+    _check(lib.moe_layer_forward_host(_ptr(x), _ptr(Wg), _ptr(W1), _ptr(W3), _ptr(W2), T, d, f, E, k, _ptr(y),
+                                      chunks, _stream(stream, W1)), "moe_layer_forward_host")
     return y
 
 

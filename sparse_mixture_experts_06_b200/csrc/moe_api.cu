@@ -198,6 +198,56 @@ struct Pool {
 std::mutex g_pool_mu;
 Pool g_pool[64];
 
+// The library-owned workspace of device `dev`, at least `need` bytes:
+// grown (stream-ordered free + malloc on s) when a larger shape arrives.
+int pool_workspace(int dev, size_t need, cudaStream_t s, void** out) {
+    std::lock_guard<std::mutex> lock(g_pool_mu);
+    Pool& p = g_pool[dev];
+    if (p.bytes < need) {
+        if (p.ptr) {
+            cudaError_t e = cudaFreeAsync(p.ptr, s);
+            p.ptr = nullptr;
+            p.bytes = 0;
+            if (e != cudaSuccess) return cuda_fail(e, "cudaFreeAsync(workspace)");
+        }
+        cudaError_t e = cudaMallocAsync(&p.ptr, need, s);
+        if (e != cudaSuccess) {
+            p.ptr = nullptr;
+            return cuda_fail(e, "cudaMallocAsync(workspace)");
+        }
+        p.bytes = need;
+    }
+    *out = p.ptr;
+    return MOE_OK;
+}
+
+// Copy streams and events of moe_layer_forward_host, per device, created on
+// first use and kept for the life of the process.  Buffer b (0 or 1) of the
+// double-buffered x / y staging has: in_done[b] (its x rows have arrived),
+// comp_done[b] (the layer has read x and written y), out_done[b] (y has left).
+struct HostPipe {
+    cudaStream_t h2d = nullptr, d2h = nullptr;
+    cudaEvent_t start = nullptr;
+    cudaEvent_t in_done[2] = {nullptr, nullptr};
+    cudaEvent_t comp_done[2] = {nullptr, nullptr};
+    cudaEvent_t out_done[2] = {nullptr, nullptr};
+    bool ready = false;
+};
+std::mutex g_pipe_mu;
+HostPipe g_pipe[64];
+
+cudaError_t pipe_init(HostPipe& P) {
+    if (P.ready) return cudaSuccess;
+    cudaError_t e = cudaStreamCreateWithFlags(&P.h2d, cudaStreamNonBlocking);
+    if (e == cudaSuccess) e = cudaStreamCreateWithFlags(&P.d2h, cudaStreamNonBlocking);
+    cudaEvent_t* evs[7] = {&P.start, &P.in_done[0], &P.in_done[1], &P.comp_done[0], &P.comp_done[1],
+                           &P.out_done[0], &P.out_done[1]};
+    for (cudaEvent_t* ev : evs)
+        if (e == cudaSuccess) e = cudaEventCreateWithFlags(ev, cudaEventDisableTiming);
+    P.ready = e == cudaSuccess;
+    return e;
+}
+
 }  // namespace
 
 extern "C" {
@@ -356,27 +406,83 @@ int moe_layer_forward(const void* x, const void* Wg, const void* W1, const void*
     if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
     if (dev >= 64) return fail(MOE_ERR_UNSUPPORTED, "device ordinal %d >= 64", dev);
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-    void* ws;
-    {
-        std::lock_guard<std::mutex> lock(g_pool_mu);
-        Pool& p = g_pool[dev];
-        if (p.bytes < need) {
-            if (p.ptr) {
-                e = cudaFreeAsync(p.ptr, s);
-                p.ptr = nullptr;
-                p.bytes = 0;
-                if (e != cudaSuccess) return cuda_fail(e, "cudaFreeAsync(workspace)");
-            }
-            e = cudaMallocAsync(&p.ptr, need, s);
-            if (e != cudaSuccess) {
-                p.ptr = nullptr;
-                return cuda_fail(e, "cudaMallocAsync(workspace)");
-            }
-            p.bytes = need;
-        }
-        ws = p.ptr;
-    }
+    void* ws = nullptr;
+    CHECK(pool_workspace(dev, need, s, &ws));
     return moe_layer_forward_ex(x, Wg, W1, W3, W2, nullptr, T, d, f, E, k, MOE_BF16, ws, need, y, stream);
+}
+
+int moe_layer_forward_host(const void* x_host, const void* Wg, const void* W1, const void* W3,
+                           const void* W2, int T, int d, int f, int E, int k, void* y_host, int chunks,
+                           moe_stream_t stream) {
+    g_last_error.clear();
+    CHECK(check_shape(T, d, f, E, k, MOE_BF16, true));
+    if (T == 0) return MOE_OK;
+    if (!x_host) return fail(MOE_ERR_INVALID_ARG, "x_host is NULL");
+    if (!y_host) return fail(MOE_ERR_INVALID_ARG, "y_host is NULL");
+    CHECK(check_ptr(Wg, "Wg"));
+    CHECK(check_ptr(W1, "W1"));
+    CHECK(check_ptr(W3, "W3"));
+    CHECK(check_ptr(W2, "W2"));
+    if (chunks < 1) return fail(MOE_ERR_INVALID_ARG, "chunks must be >= 1 (got %d)", chunks);
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+    if (dev >= 64) return fail(MOE_ERR_UNSUPPORTED, "device ordinal %d >= 64", dev);
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+
+    const int C = chunks < T ? chunks : T;
+    const int Tc = (T + C - 1) / C;  // tokens per chunk (the last may be shorter)
+    const size_t ws_need = moe_workspace_size(Tc, d, f, E, k, MOE_BF16);
+    const size_t row_bytes = (size_t)d * 2;
+    const size_t buf = align256((size_t)Tc * row_bytes);
+    void* base = nullptr;
+    CHECK(pool_workspace(dev, ws_need + 4 * buf, s, &base));
+    char* xbuf[2] = {static_cast<char*>(base) + ws_need, static_cast<char*>(base) + ws_need + buf};
+    char* ybuf[2] = {xbuf[1] + buf, xbuf[1] + 2 * buf};
+
+    std::lock_guard<std::mutex> lock(g_pipe_mu);
+    HostPipe& P = g_pipe[dev];
+    if ((e = pipe_init(P)) != cudaSuccess) return cuda_fail(e, "creating the copy streams");
+    // the copies follow everything already on s (earlier calls, workspace growth)
+    if ((e = cudaEventRecord(P.start, s)) != cudaSuccess ||
+        (e = cudaStreamWaitEvent(P.h2d, P.start, 0)) != cudaSuccess ||
+        (e = cudaStreamWaitEvent(P.d2h, P.start, 0)) != cudaSuccess)
+        return cuda_fail(e, "ordering the copy streams");
+    const char* xh = static_cast<const char*>(x_host);
+    char* yh = static_cast<char*>(y_host);
+    bool used[2] = {false, false};
+    for (int c = 0; c < C; ++c) {
+        const int t0 = c * Tc;
+        const int tc = T - t0 < Tc ? T - t0 : Tc;
+        if (tc <= 0) break;
+        const int b = c & 1;
+        const size_t off = (size_t)t0 * row_bytes, bytes = (size_t)tc * row_bytes;
+        // x rows in, once the layer two chunks back has finished reading buffer b
+        if (used[b] && (e = cudaStreamWaitEvent(P.h2d, P.comp_done[b], 0)) != cudaSuccess)
+            return cuda_fail(e, "cudaStreamWaitEvent");
+        if ((e = cudaMemcpyAsync(xbuf[b], xh + off, bytes, cudaMemcpyHostToDevice, P.h2d)) != cudaSuccess ||
+            (e = cudaEventRecord(P.in_done[b], P.h2d)) != cudaSuccess)
+            return cuda_fail(e, "copying x to the device");
+        // the layer, once x has arrived and y buffer b has been copied out
+        if ((e = cudaStreamWaitEvent(s, P.in_done[b], 0)) != cudaSuccess ||
+            (used[b] && (e = cudaStreamWaitEvent(s, P.out_done[b], 0)) != cudaSuccess))
+            return cuda_fail(e, "cudaStreamWaitEvent");
+        CHECK(moe_layer_forward_ex(xbuf[b], Wg, W1, W3, W2, nullptr, tc, d, f, E, k, MOE_BF16, base, ws_need,
+                                   ybuf[b], stream));
+        if ((e = cudaEventRecord(P.comp_done[b], s)) != cudaSuccess)
+            return cuda_fail(e, "cudaEventRecord");
+        // y rows out
+        if ((e = cudaStreamWaitEvent(P.d2h, P.comp_done[b], 0)) != cudaSuccess ||
+            (e = cudaMemcpyAsync(yh + off, ybuf[b], bytes, cudaMemcpyDeviceToHost, P.d2h)) != cudaSuccess ||
+            (e = cudaEventRecord(P.out_done[b], P.d2h)) != cudaSuccess)
+            return cuda_fail(e, "copying y to the host");
+        used[b] = true;
+    }
+    // work later enqueued on s (and a synchronize of s) also covers the copies out
+    for (int b = 0; b < 2; ++b)
+        if (used[b] && (e = cudaStreamWaitEvent(s, P.out_done[b], 0)) != cudaSuccess)
+            return cuda_fail(e, "cudaStreamWaitEvent");
+    return MOE_OK;
 }
 
 int moe_release_workspace(moe_stream_t stream) {

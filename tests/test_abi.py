@@ -126,6 +126,26 @@ def test_layer_rejects_invalid_arguments():
                P(512), None) == 1   # offsets NULL
 
 
+def test_host_layer_rejects_invalid_arguments():
+    """moe_layer_forward_host: argument errors are reported before any CUDA
+    call (fake pointers; the valid list itself is never called)."""
+    P = ctypes.c_void_p
+    f = moe.lib.moe_layer_forward_host
+    args = [P(8)] + [P(16)] * 4 + [16, 64, 128, 8, 2, P(8), 2, None]
+    bad = list(args); bad[0] = None                            # x_host NULL
+    assert f(*bad) == 1 and "x_host" in moe.moe_last_error_string()
+    bad = list(args); bad[10] = None                           # y_host NULL
+    assert f(*bad) == 1 and "y_host" in moe.moe_last_error_string()
+    bad = list(args); bad[11] = 0                              # no chunks
+    assert f(*bad) == 1 and "chunks" in moe.moe_last_error_string()
+    bad = list(args); bad[2] = P(24)                           # W1 not 16-byte aligned
+    assert f(*bad) == 1 and "aligned" in moe.moe_last_error_string()
+    bad = list(args); bad[9] = 9                               # k > E
+    assert f(*bad) == 1
+    bad = list(args); bad[5] = 0; bad[0] = None; bad[10] = None  # T = 0: a no-op
+    assert f(*bad) == 0
+
+
 def test_stack_rejects_invalid_arguments():
     P = ctypes.c_void_p
     arr = (ctypes.c_void_p * 2)(16, 16)
