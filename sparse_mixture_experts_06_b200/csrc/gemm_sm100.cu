@@ -7,30 +7,36 @@
 //   down (second half and the gate weighting of §2.1 display 3):
 //         obuf_r = topk_w[perm[r]] * (W2_e h_r), fp32.
 //
-// Both are one persistent, warp-specialised kernel over output tiles of
-// 128 permuted rows:
+// Both are one persistent, warp-specialised kernel (192 threads per CTA):
 //   warp 0      TMA producer: 2-D tiled bulk copies (128-byte swizzle) of the
-//               A tile (128 rows x 64 k) and the B tile (256 rows x 64 k)
-//               into a 4-stage shared-memory ring, signalled on mbarriers;
+//               A tile (token rows x 64 k) and the B tile (weight rows x 64 k)
+//               into a shared-memory ring of stages, signalled on mbarriers;
 //   warp 1      MMA issuer: one thread issues tcgen05.mma (bf16 x bf16 ->
-//               fp32, M = 128, N = 256, K = 16) into a tensor-memory (TMEM)
-//               accumulator and releases ring stages with tcgen05.commit;
+//               fp32, K = 16) into a tensor-memory (TMEM) accumulator and
+//               releases ring stages with tcgen05.commit;
 //   warps 2-5   epilogue: tcgen05.ld of the accumulator (each warp owns the
-//               32 TMEM lanes = tile rows of its quadrant), fused SiLU(a)*b
-//               or gate scaling, and the stores.
-// TMEM holds two 256-column accumulators, so the epilogue of one tile
-// overlaps the main loop of the next.
+//               32 TMEM lanes of its quadrant), fused SiLU(a)*b or gate
+//               scaling, and the stores.
+// Tile shapes (template variants; the host picks one per launch):
+//   single CTA   128 (or 32) rows x 256 columns, M = 128 N = 256 MMAs; two
+//                TMEM accumulators, so a tile's epilogue overlaps the next
+//                tile's main loop;
+//   CTA pair     256 rows x 512 columns (default) or 256 x 256: cta_group::2
+//                M = 256 MMAs issued by the even CTA, each CTA holding 128
+//                rows of A and half of each MMA's B.  The 512-column tile
+//                issues two N = 256 MMAs per k step on the same A and fills
+//                all of TMEM (one accumulator buffer).
 //
 // Up tiles: B = 128 rows of W1_e stacked on the same 128 rows of W3_e, so
 // one N = 256 MMA produces a (columns 0-127) and b (128-255) for 128
-// hidden units.  Down tiles: B = 256 rows of W2_e.
+// hidden units.  Down tiles: B = 256 rows of W2_e per MMA.
 //
-// CTA pairs (cta_group::2) run 256-row tiles as M = 256 MMAs; the last row
-// block of an expert that holds at most 128 rows runs as an M = 128 pair
-// MMA instead (each CTA loads 64 rows of A), so pairs pad an expert to a
-// multiple of 128 rows, not 256.  In a pair up tile each CTA's half of B is
-// 64 rows of W1 followed by the same 64 rows of W3, so that a and b of one
-// hidden unit sit in the same TMEM lane for both MMA shapes.
+// In a pair, the last row block of an expert that holds at most 128 rows
+// runs as an M = 128 pair MMA (each CTA loads 64 rows of A), so pairs pad
+// an expert to a multiple of 128 rows, not 256.  In a pair up tile each
+// CTA's part of B is 64 rows of W1 followed by the same 64 rows of W3, so
+// that a and b of one hidden unit sit in the same TMEM lane for both MMA
+// shapes.
 //
 // Tiles are enumerated per expert from the device-side offsets (no host
 // round trip): expert e owns ceil(M_e / tile rows) row blocks x n_tiles column
@@ -304,13 +310,20 @@ constexpr int kOutBytes = 4 * 2 * kOutBoxBytes;
 // occupies TMEM lanes 0-63 for columns 0 .. BN/2-1 and lanes 64-127 for
 // columns BN/2 .. BN-1, both at column offsets 0 .. BN/2-1 (the 2x2
 // datapath layout of the 2-SM M = 128 shape).
+// NH (pairs only): MMAs of N = BN per tile along N.  NH = 2 makes a 256 x 2BN
+// tile: both MMAs of a k step share the A tile, so each CTA loads A once per
+// 2 BN columns (a quarter fewer bytes per MMA than NH = 1), and each CTA's
+// B stage holds NH parts of BN/2 rows, part h feeding MMA h.  The two
+// accumulators then fill all 512 TMEM columns, so there is one accumulator
+// buffer and the epilogue of a tile is not overlapped with the next tile's
+// MMAs (NH = 1 keeps two buffers and overlaps them).
 // The stage ring fills 192 KiB of shared memory.
 //
 // Instruction descriptor (kind::f16): D fp32 (bits 4-5 = 1), A and B bf16
 // (bits 7-9 = 1, 10-12 = 1), both K-major (bits 15, 16 = 0), N >> 3 in
 // bits 17-22, M >> 4 in bits 24-28.
 
-template <int CG, int BN, int RB>
+template <int CG, int BN, int RB, int NH = 1>
 struct Cfg {
     // RB (single CTA only): token rows loaded per tile, 128 or 32.  With 32
     // the TMA fills only the first 32 rows of the 128-row A buffer; the MMA
@@ -318,11 +331,14 @@ struct Cfg {
     // accumulator rows that are never stored: row i of the product depends
     // on row i of A alone.  For decode, where experts hold a few rows each.
     static_assert(CG == 1 || RB == 128, "pairs load 128 rows per CTA");
+    static_assert(NH == 1 || CG == 2, "two MMAs per tile along N: pairs only");
     static constexpr int kTileRows = (CG == 1) ? RB : 256;   // rows of one tile (pair)
     static constexpr int kABytes = ((CG == 1) ? RB : 128) * BK * 2;  // A bytes loaded per stage
-    static constexpr int kBRows = (CG == 1) ? BN : BN / 2;   // B rows held by one CTA
-    static constexpr int kBHalf = (BN / 2) * BK * 2;         // bytes of BN/2 rows of B
+    static constexpr int kBRows = (CG == 1) ? BN : NH * BN / 2;   // B rows held by one CTA
+    static constexpr int kBHalf = (BN / 2) * BK * 2;         // bytes of BN/2 rows of B (one part, pairs)
     static constexpr int kBBytes = kBRows * BK * 2;
+    static constexpr int kNAcc = (NH == 1) ? 2 : 1;          // accumulator buffers in TMEM
+    static constexpr int kTileN = NH * BN;                   // accumulator columns of a tile
     static constexpr int kStageBytes = A_TILE + kBBytes;     // per CTA (A buffer always 128 rows)
     static constexpr int kStages = (196608 / kStageBytes) > 8 ? 8 : (196608 / kStageBytes);
     static constexpr int kSmem = 1024 + kStages * kStageBytes + kOutBytes + 1024;
@@ -400,12 +416,12 @@ struct Sched {
     static constexpr uint32_t kReaders = (CG == 1) ? 5u : 10u;
 };
 
-template <int MODE, int CG, int BN, int RB>
+template <int MODE, int CG, int BN, int RB, int NH>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
 grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmAs,
                     const __grid_constant__ CUtensorMap tmB0, const __grid_constant__ CUtensorMap tmB1,
                     const __grid_constant__ CUtensorMap tmOut, const KParams p) {
-    using C = Cfg<CG, BN, RB>;
+    using C = Cfg<CG, BN, RB, NH>;
     // pair up tiles interleave 64 rows of W1 and of W3 per CTA (N = 256)
     static_assert(!(CG == 2 && MODE == kUp) || BN == 256, "pair up-projection tiles are 256 columns wide");
     constexpr int STG = C::kStages;
@@ -528,11 +544,13 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
                     rowB0 = e * p.b_rows_per_expert + nb * (MODE == kUp ? BN / 2 : BN);
                     rowB1 = (MODE == kUp) ? rowB0 : rowB0 + BN / 2;
                 } else if constexpr (MODE == kUp) {
-                    // this CTA's 64 hidden units: W1 rows, then the same W3 rows
-                    rowB0 = e * p.b_rows_per_expert + nb * (BN / 2) + (int)rank * (BN / 4);
+                    // part h: this CTA's 64 hidden units of MMA h, W1 rows then
+                    // the same W3 rows (rowB0 + h * BN / 2 for part h)
+                    rowB0 = e * p.b_rows_per_expert + nb * (NH * BN / 2) + (int)rank * (BN / 4);
                     rowB1 = rowB0;
                 } else {
-                    rowB0 = e * p.b_rows_per_expert + nb * BN + (int)rank * (BN / 2);
+                    // part h: rows rowB0 + h * BN of W2
+                    rowB0 = e * p.b_rows_per_expert + nb * (NH * BN) + (int)rank * (BN / 2);
                     rowB1 = rowB0;
                 }
                 const int kb_next = kblocks > STG ? kblocks - STG : 0;
@@ -551,11 +569,15 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
                         // both CTAs' bytes are counted on the even CTA's barrier
                         if (leader) mbar_arrive_expect_tx(fb, 2 * ((shrt ? C::kAShortBytes : A_TILE) + C::kBBytes));
                         tma_load_2d_pair(smem_u32(sA + s * A_TILE), shrt ? &tmAs : &tmA, fb, kb * BK, rowA);
-                        if constexpr (MODE == kUp) {
-                            tma_load_2d_pair(smem_u32(sB + s * C::kBBytes), &tmB0, fb, kb * BK, rowB0);
-                            tma_load_2d_pair(smem_u32(sB + s * C::kBBytes + C::kBBytes / 2), &tmB1, fb, kb * BK, rowB1);
-                        } else {
-                            tma_load_2d_pair(smem_u32(sB + s * C::kBBytes), &tmB0, fb, kb * BK, rowB0);
+#pragma unroll
+                        for (int h = 0; h < NH; ++h) {
+                            const uint32_t part = smem_u32(sB + s * C::kBBytes + h * C::kBHalf);
+                            if constexpr (MODE == kUp) {
+                                tma_load_2d_pair(part, &tmB0, fb, kb * BK, rowB0 + h * (BN / 2));
+                                tma_load_2d_pair(part + C::kBHalf / 2, &tmB1, fb, kb * BK, rowB1 + h * (BN / 2));
+                            } else {
+                                tma_load_2d_pair(part, &tmB0, fb, kb * BK, rowB0 + h * BN);
+                            }
                         }
                     }
                 }
@@ -583,11 +605,11 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
                 if (!ok) break;
                 release_tile(tcount);
                 if (tile < 0) break;
-                const uint32_t acc = tcount & 1u;
-                const uint32_t use = tcount >> 1;
+                const uint32_t acc = tcount % C::kNAcc;
+                const uint32_t use = tcount / C::kNAcc;
                 if (!wait_bounded_pair(smem_u32(&tempty[acc]), (use & 1u) ^ 1u, abort_flag, p.err, peer_abort)) break;
                 tc_fence_after();
-                const uint32_t d_tmem = tmem_base + acc * BN;
+                const uint32_t d_tmem = tmem_base + acc * C::kTileN;
                 uint32_t idesc = C::kIdesc;
                 if constexpr (CG == 2) {
                     int e, mb, nb;
@@ -605,12 +627,16 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
 #pragma unroll
                     for (int kk = 0; kk < BK / UMMA_K; ++kk) {
                         // advance 16 bf16 = 32 bytes along K inside the swizzle row
-                        if constexpr (CG == 1)
+                        if constexpr (CG == 1) {
                             umma_bf16(d_tmem, adesc + (uint64_t)(kk * 2), bdesc + (uint64_t)(kk * 2), C::kIdesc,
                                       (kb | kk) != 0 ? 1u : 0u);
-                        else
-                            umma_bf16_pair(d_tmem, adesc + (uint64_t)(kk * 2), bdesc + (uint64_t)(kk * 2), idesc,
-                                           (kb | kk) != 0 ? 1u : 0u);
+                        } else {
+#pragma unroll
+                            for (int h = 0; h < NH; ++h)  // part h of B (kBHalf bytes = kBHalf >> 4 descriptor units)
+                                umma_bf16_pair(d_tmem + h * BN, adesc + (uint64_t)(kk * 2),
+                                               bdesc + (uint64_t)(h * (C::kBHalf >> 4) + kk * 2), idesc,
+                                               (kb | kk) != 0 ? 1u : 0u);
+                        }
                     }
                     if constexpr (CG == 1) umma_commit(smem_u32(&empty[s])); else umma_commit_pair(smem_u32(&empty[s]));
                 }
@@ -637,8 +663,8 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
             if (tile < 0) break;
             int e, mb, nb;
             decode_tile_rows(tile, s_beg, s_end, p.E, p.n_tiles, C::kTileRows, e, mb, nb);
-            const uint32_t acc = tcount & 1u;
-            const uint32_t use = tcount >> 1;
+            const uint32_t acc = tcount % C::kNAcc;
+            const uint32_t use = tcount / C::kNAcc;
             // every lane waits; the decision to stop is warp-uniform so the
             // .sync.aligned TMEM loads below always run on a converged warp
             const bool okw = wait_bounded_pair(smem_u32(&tfull[acc]), use & 1u, abort_flag, p.err, peer_abort);
@@ -661,110 +687,119 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
             // expert's rows)
             const int wrow0 = row - lane;
             const bool box_ok = wrow0 + 32 <= tile_end;
-            const uint32_t tacc = t_lane + acc * BN;
-            if constexpr (MODE == kUp) {
-                __nv_bfloat16* hrow = p.h + (size_t)row * p.n_out;
-                // 64-unit segments: hidden units c64 .. c64+63 of the tile have
-                // a at TMEM columns acol .. acol+63 and b at acol+bdelta ...
-                //   single CTA: a = columns 0 .. BN/2-1, b = BN/2 .. BN-1;
-                //   pair, full: [a 64 | b 64] per CTA half of B, two halves;
-                //   pair, short: one half per lane group, at columns 0-127.
-                const int nseg = (CG == 1) ? BN / 128 : (shrt ? 1 : 2);
-                const int bdelta = (CG == 1) ? BN / 2 : 64;
+            // MMA h of the tile: accumulator columns h * BN .. h * BN + BN-1,
+            // output columns from hb (hidden units, up) or ob (down)
 #pragma unroll 1
-                for (int seg = 0; seg < nseg; ++seg, ++obox) {
-                    const int c64 = (shrt ? colhalf : seg) * 64;        // hidden offset in the tile
-                    const int acol = (CG == 1) ? seg * 64 : (shrt ? 0 : seg * 128);
-                    const uint32_t buf = out_base + (obox & 1u) * kOutBoxBytes;
-                    if (box_ok) {
-                        if (lane == 0) bulk_wait_read_le1();  // this buffer's previous store has read it
-                        __syncwarp();
-                    }
-#pragma unroll 1
-                    for (int half = 0; half < 2; ++half) {
-                        const int c = c64 + half * 32;
-                        uint32_t a[32], b[32];
-                        tmem_ld32(tacc + acol + half * 32, a);
-                        tmem_ld32(tacc + acol + half * 32 + bdelta, b);
-                        tmem_wait_ld();
-                        uint4 pk[4];
-#pragma unroll
-                        for (int g = 0; g < 4; ++g) {
-                            pk[g].x = pack_bf16x2(silu_mul(__uint_as_float(a[g * 8 + 0]), __uint_as_float(b[g * 8 + 0])),
-                                                  silu_mul(__uint_as_float(a[g * 8 + 1]), __uint_as_float(b[g * 8 + 1])));
-                            pk[g].y = pack_bf16x2(silu_mul(__uint_as_float(a[g * 8 + 2]), __uint_as_float(b[g * 8 + 2])),
-                                                  silu_mul(__uint_as_float(a[g * 8 + 3]), __uint_as_float(b[g * 8 + 3])));
-                            pk[g].z = pack_bf16x2(silu_mul(__uint_as_float(a[g * 8 + 4]), __uint_as_float(b[g * 8 + 4])),
-                                                  silu_mul(__uint_as_float(a[g * 8 + 5]), __uint_as_float(b[g * 8 + 5])));
-                            pk[g].w = pack_bf16x2(silu_mul(__uint_as_float(a[g * 8 + 6]), __uint_as_float(b[g * 8 + 6])),
-                                                  silu_mul(__uint_as_float(a[g * 8 + 7]), __uint_as_float(b[g * 8 + 7])));
+            for (int h = 0; h < NH; ++h) {
+                const uint32_t tacc = t_lane + acc * C::kTileN + h * BN;
+                const int hb = nb * (NH * BN / 2) + h * (BN / 2);
+                const int ob = nb * (NH * BN) + h * BN;
+                (void)hb;
+                (void)ob;
+                if constexpr (MODE == kUp) {
+                    __nv_bfloat16* hrow = p.h + (size_t)row * p.n_out;
+                    // 64-unit segments: hidden units c64 .. c64+63 of the tile have
+                    // a at TMEM columns acol .. acol+63 and b at acol+bdelta ...
+                    //   single CTA: a = columns 0 .. BN/2-1, b = BN/2 .. BN-1;
+                    //   pair, full: [a 64 | b 64] per CTA half of B, two halves;
+                    //   pair, short: one half per lane group, at columns 0-127.
+                    const int nseg = (CG == 1) ? BN / 128 : (shrt ? 1 : 2);
+                    const int bdelta = (CG == 1) ? BN / 2 : 64;
+    #pragma unroll 1
+                    for (int seg = 0; seg < nseg; ++seg, ++obox) {
+                        const int c64 = (shrt ? colhalf : seg) * 64;        // hidden offset in the tile
+                        const int acol = (CG == 1) ? seg * 64 : (shrt ? 0 : seg * 128);
+                        const uint32_t buf = out_base + (obox & 1u) * kOutBoxBytes;
+                        if (box_ok) {
+                            if (lane == 0) bulk_wait_read_le1();  // this buffer's previous store has read it
+                            __syncwarp();
+                        }
+    #pragma unroll 1
+                        for (int half = 0; half < 2; ++half) {
+                            const int c = c64 + half * 32;
+                            uint32_t a[32], b[32];
+                            tmem_ld32(tacc + acol + half * 32, a);
+                            tmem_ld32(tacc + acol + half * 32 + bdelta, b);
+                            tmem_wait_ld();
+                            uint4 pk[4];
+    #pragma unroll
+                            for (int g = 0; g < 4; ++g) {
+                                pk[g].x = pack_bf16x2(silu_mul(__uint_as_float(a[g * 8 + 0]), __uint_as_float(b[g * 8 + 0])),
+                                                      silu_mul(__uint_as_float(a[g * 8 + 1]), __uint_as_float(b[g * 8 + 1])));
+                                pk[g].y = pack_bf16x2(silu_mul(__uint_as_float(a[g * 8 + 2]), __uint_as_float(b[g * 8 + 2])),
+                                                      silu_mul(__uint_as_float(a[g * 8 + 3]), __uint_as_float(b[g * 8 + 3])));
+                                pk[g].z = pack_bf16x2(silu_mul(__uint_as_float(a[g * 8 + 4]), __uint_as_float(b[g * 8 + 4])),
+                                                      silu_mul(__uint_as_float(a[g * 8 + 5]), __uint_as_float(b[g * 8 + 5])));
+                                pk[g].w = pack_bf16x2(silu_mul(__uint_as_float(a[g * 8 + 6]), __uint_as_float(b[g * 8 + 6])),
+                                                      silu_mul(__uint_as_float(a[g * 8 + 7]), __uint_as_float(b[g * 8 + 7])));
+                            }
+                            if (box_ok) {
+    #pragma unroll
+                                for (int g = 0; g < 4; ++g)
+                                    st_shared_v4(buf + lane * 128 + ((((half * 4 + g) ^ (lane & 7))) << 4), pk[g]);
+                            } else if (valid) {
+                                const int col0 = hb + c;
+    #pragma unroll
+                                for (int g = 0; g < 4; ++g)
+                                    if (col0 + g * 8 < p.n_out) *reinterpret_cast<uint4*>(hrow + col0 + g * 8) = pk[g];
+                            }
                         }
                         if (box_ok) {
-#pragma unroll
-                            for (int g = 0; g < 4; ++g)
-                                st_shared_v4(buf + lane * 128 + ((((half * 4 + g) ^ (lane & 7))) << 4), pk[g]);
+                            fence_proxy_async_smem();
+                            __syncwarp();
+                            if (lane == 0) {
+                                // a box wholly past the last column is not stored; the
+                                // (empty) group keeps one group per staged box
+                                if (hb + c64 < p.n_out) tma_store_2d(&tmOut, buf, hb + c64, wrow0);
+                                bulk_commit();
+                            }
+                        }
+                    }
+                } else {
+                    float wgt = 0.f;
+                    if (valid) {
+                        const int q = p.perm[row];
+                        wgt = ((unsigned)q < (unsigned)p.rows) ? p.topk_w[q] : 0.f;
+                    }
+                    float* orow = p.obuf + (size_t)row * p.n_out;
+                    // short pair tiles: this warp's lanes hold BN/2 columns,
+                    // starting at output column colhalf * BN/2
+                    const int ncol = shrt ? BN / 2 : BN;
+                    const int cbase = colhalf * (BN / 2);
+    #pragma unroll 1
+                    for (int cc = 0; cc < ncol; cc += 32, ++obox) {
+                        const int c = cbase + cc;  // tile column
+                        const uint32_t buf = out_base + (obox & 1u) * kOutBoxBytes;
+                        if (box_ok) {
+                            if (lane == 0) bulk_wait_read_le1();
+                            __syncwarp();
+                        }
+                        uint32_t o[32];
+                        tmem_ld32(tacc + cc, o);
+                        tmem_wait_ld();
+                        uint4 v[8];
+    #pragma unroll
+                        for (int g = 0; g < 8; ++g) {
+                            v[g].x = __float_as_uint(wgt * __uint_as_float(o[g * 4 + 0]));
+                            v[g].y = __float_as_uint(wgt * __uint_as_float(o[g * 4 + 1]));
+                            v[g].z = __float_as_uint(wgt * __uint_as_float(o[g * 4 + 2]));
+                            v[g].w = __float_as_uint(wgt * __uint_as_float(o[g * 4 + 3]));
+                        }
+                        if (box_ok) {
+    #pragma unroll
+                            for (int g = 0; g < 8; ++g) st_shared_v4(buf + lane * 128 + ((g ^ (lane & 7)) << 4), v[g]);
+                            fence_proxy_async_smem();
+                            __syncwarp();
+                            if (lane == 0) {
+                                if (ob + c < p.n_out) tma_store_2d(&tmOut, buf, ob + c, wrow0);
+                                bulk_commit();
+                            }
                         } else if (valid) {
-                            const int col0 = nb * (BN / 2) + c;
-#pragma unroll
-                            for (int g = 0; g < 4; ++g)
-                                if (col0 + g * 8 < p.n_out) *reinterpret_cast<uint4*>(hrow + col0 + g * 8) = pk[g];
+                            const int col0 = ob + c;
+    #pragma unroll
+                            for (int g = 0; g < 8; ++g)
+                                if (col0 + g * 4 < p.n_out) *reinterpret_cast<uint4*>(orow + col0 + g * 4) = v[g];
                         }
-                    }
-                    if (box_ok) {
-                        fence_proxy_async_smem();
-                        __syncwarp();
-                        if (lane == 0) {
-                            // a box wholly past the last column is not stored; the
-                            // (empty) group keeps one group per staged box
-                            if (nb * (BN / 2) + c64 < p.n_out) tma_store_2d(&tmOut, buf, nb * (BN / 2) + c64, wrow0);
-                            bulk_commit();
-                        }
-                    }
-                }
-            } else {
-                float wgt = 0.f;
-                if (valid) {
-                    const int q = p.perm[row];
-                    wgt = ((unsigned)q < (unsigned)p.rows) ? p.topk_w[q] : 0.f;
-                }
-                float* orow = p.obuf + (size_t)row * p.n_out;
-                // short pair tiles: this warp's lanes hold BN/2 columns,
-                // starting at output column colhalf * BN/2
-                const int ncol = shrt ? BN / 2 : BN;
-                const int cbase = colhalf * (BN / 2);
-#pragma unroll 1
-                for (int cc = 0; cc < ncol; cc += 32, ++obox) {
-                    const int c = cbase + cc;  // tile column
-                    const uint32_t buf = out_base + (obox & 1u) * kOutBoxBytes;
-                    if (box_ok) {
-                        if (lane == 0) bulk_wait_read_le1();
-                        __syncwarp();
-                    }
-                    uint32_t o[32];
-                    tmem_ld32(tacc + cc, o);
-                    tmem_wait_ld();
-                    uint4 v[8];
-#pragma unroll
-                    for (int g = 0; g < 8; ++g) {
-                        v[g].x = __float_as_uint(wgt * __uint_as_float(o[g * 4 + 0]));
-                        v[g].y = __float_as_uint(wgt * __uint_as_float(o[g * 4 + 1]));
-                        v[g].z = __float_as_uint(wgt * __uint_as_float(o[g * 4 + 2]));
-                        v[g].w = __float_as_uint(wgt * __uint_as_float(o[g * 4 + 3]));
-                    }
-                    if (box_ok) {
-#pragma unroll
-                        for (int g = 0; g < 8; ++g) st_shared_v4(buf + lane * 128 + ((g ^ (lane & 7)) << 4), v[g]);
-                        fence_proxy_async_smem();
-                        __syncwarp();
-                        if (lane == 0) {
-                            if (nb * BN + c < p.n_out) tma_store_2d(&tmOut, buf, nb * BN + c, wrow0);
-                            bulk_commit();
-                        }
-                    } else if (valid) {
-                        const int col0 = nb * BN + c;
-#pragma unroll
-                        for (int g = 0; g < 8; ++g)
-                            if (col0 + g * 4 < p.n_out) *reinterpret_cast<uint4*>(orow + col0 + g * 4) = v[g];
                     }
                 }
             }
@@ -836,11 +871,11 @@ struct GemmMaps {
     CUtensorMap A, A32, A64, B0, B1, B0p, B1p, Out;
 };
 
-template <int MODE, int CG, int BN, int RB>
+template <int MODE, int CG, int BN, int RB, int NH = 1>
 cudaError_t launch_gemm(const GroupedGemmArgs& a, const CUtensorMap& mA, const CUtensorMap& mAs,
                         const CUtensorMap& mB0, const CUtensorMap& mB1, const CUtensorMap& mOut, const KParams& p,
                         cudaStream_t s) {
-    using C = Cfg<CG, BN, RB>;
+    using C = Cfg<CG, BN, RB, NH>;
     static int units_cache[64] = {0};
     int dev = 0;
     cudaGetDevice(&dev);
@@ -860,14 +895,14 @@ cudaError_t launch_gemm(const GroupedGemmArgs& a, const CUtensorMap& mA, const C
         cfg.numAttrs = 1;
     }
     if (!units) {
-        cudaError_t e = cudaFuncSetAttribute(grouped_gemm_kernel<MODE, CG, BN, RB>,
+        cudaError_t e = cudaFuncSetAttribute(grouped_gemm_kernel<MODE, CG, BN, RB, NH>,
                                              cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmem);
         if (e != cudaSuccess) return e;
         units = a.num_sms / CG;
         if (CG == 2) {
             int clusters = 0;
             cfg.gridDim = dim3(2 * units);
-            if (cudaOccupancyMaxActiveClusters(&clusters, grouped_gemm_kernel<MODE, CG, BN, RB>, &cfg) == cudaSuccess &&
+            if (cudaOccupancyMaxActiveClusters(&clusters, grouped_gemm_kernel<MODE, CG, BN, RB, NH>, &cfg) == cudaSuccess &&
                 clusters > 0 && clusters < units)
                 units = clusters;
             cudaGetLastError();  // an unsupported query is not an error for the launch
@@ -878,33 +913,31 @@ cudaError_t launch_gemm(const GroupedGemmArgs& a, const CUtensorMap& mA, const C
     const int grid_units = (int)(ub < units ? ub : units);
     if (grid_units <= 0) return cudaSuccess;
     cfg.gridDim = dim3(grid_units * CG);
-    return cudaLaunchKernelEx(&cfg, grouped_gemm_kernel<MODE, CG, BN, RB>, mA, mAs, mB0, mB1, mOut, p);
+    return cudaLaunchKernelEx(&cfg, grouped_gemm_kernel<MODE, CG, BN, RB, NH>, mA, mAs, mB0, mB1, mOut, p);
 }
 
 // Variant choice: 1 = single-CTA tiles, 2 = CTA-pair tiles, 3 = hybrid.
-// (Pair figures below are from before short pair tiles, when pairs padded
-// every expert to a multiple of 256 rows.)
-// Measured on B200 with Mixtral shapes:
-//  * pairs (M = 256) move a third fewer bytes per MMA from L2 and ran ~10%
-//    faster per row (one-expert 8192-row layer: up 1.34 vs 1.48 ms, down
-//    0.66 vs 0.77 ms), but pad every expert to a multiple of 256 rows;
-//  * grouped prefill (T = 4096, ~1000 rows per expert): single-CTA tiles are
-//    best for the up-projection (K = d), pairs for the down-projection
-//    (K = f): 1.55 + 0.77 ms;
-//  * the hybrid (pairs on each expert's whole 256-row blocks, then a
-//    single-CTA launch on the remaining rows) was slower (1.62 + 0.93 ms):
-//    the second launch has only 1-2 row tiles per weight tile and streams
-//    every expert's weights from HBM again;
-//  * decode (a few rows per expert): single-CTA tiles.
-// MOE_GEMM_CTA_GROUP = 1, 2 or h forces a variant (all exact; the tests run
-// each).
+// Measured on B200 with Mixtral shapes (d = 4096, f = 14336, E = 8):
+//  * pairs need a third fewer bytes per MMA from L2 than single-CTA tiles,
+//    and 256 x 512 pair tiles (two MMAs sharing each A tile, see NH) a
+//    quarter fewer again.  Prefill (T = 4096, ~1000 rows per expert), both
+//    GEMMs: single up + 256 x 256 pair down 2.50-2.54 ms per layer, pairs
+//    256 x 256 for both 2.50 ms, pairs 256 x 512 for both 2.38-2.42 ms;
+//    skewed (T = 16384): 10.2, 10.1 and 9.3 ms;
+//  * the hybrid (pairs on whole 256-row blocks, then a single-CTA launch on
+//    the remaining rows) was slower: the second launch has only 1-2 row
+//    tiles per weight tile and streams every expert's weights again;
+//  * decode (a few rows per expert): single-CTA tiles of 32 token rows.
+// Pairs are used once experts average 512 rows; MOE_GEMM_CTA_GROUP = 1, 2 or
+// h forces a variant (all exact; the tests run each).
 int choose_cta_group(const GroupedGemmArgs& a, int mode) {
     if (const char* env = getenv("MOE_GEMM_CTA_GROUP")) {
         if (env[0] == '1') return 1;
         if (env[0] == '2') return 2;
         if (env[0] == 'h') return 3;
     }
-    return (mode == kDown && a.rows >= 512 * a.E) ? 2 : 1;
+    (void)mode;
+    return a.rows >= 512 * a.E ? 2 : 1;
 }
 
 }  // namespace
@@ -939,11 +972,26 @@ int choose_rb(const GroupedGemmArgs& a) {
     return a.rows <= 16 * a.E ? 32 : 128;
 }
 
+// Pair tiles of 256 x 512 (two N = 256 MMAs sharing each A tile; default)
+// or 256 x 256 (two TMEM accumulator buffers, epilogue overlapped).
+// MOE_GEMM_WIDE = 1 or 0 forces one.
+bool choose_wide(const GroupedGemmArgs&) {
+    if (const char* env = getenv("MOE_GEMM_WIDE")) return env[0] == '1';
+    return true;
+}
+
 template <int MODE, int BN>
 cudaError_t launch_variant(const GroupedGemmArgs& a, const GemmMaps& m, const KParams& p, cudaStream_t s) {
     // pairs: 256-column tiles only (the up-projection's interleaved B halves)
     const int cg = (MODE == kUp && BN != 256) ? 1 : choose_cta_group(a, MODE);
     if constexpr (MODE == kDown || BN == 256) {
+        if (cg == 2 && choose_wide(a)) {
+            // 256 x 512 pair tiles: twice the columns per tile
+            KParams pw = p;
+            const int cols = (MODE == kUp) ? BN : 2 * BN;  // output columns of a wide tile
+            pw.n_tiles = (p.n_out + cols - 1) / cols;
+            return launch_gemm<MODE, 2, BN, 128, 2>(a, m.A, m.A64, m.B0p, m.B1p, m.Out, pw, s);
+        }
         if (cg == 2) return launch_gemm<MODE, 2, BN, 128>(a, m.A, m.A64, m.B0p, m.B1p, m.Out, p, s);
         if (cg == 3) {  // hybrid: pairs on whole 256-row blocks, then single CTAs on the rest (same stream)
             KParams pf = p, pr = p;

@@ -175,21 +175,24 @@ def test_layer_parity_every_token_f32(shape):
     assert rel <= 1e-5
 
 
-GEMM_VARIANTS = [("1", "256", "128"), ("1", "128", "128"), ("1", "256", "32"), ("1", "128", "32"),
-                 ("2", "256", "128"), ("h", "256", "128")]
+GEMM_VARIANTS = [("1", "256", "128", "0"), ("1", "128", "128", "0"), ("1", "256", "32", "0"),
+                 ("1", "128", "32", "0"), ("2", "256", "128", "0"), ("2", "256", "128", "1"),
+                 ("h", "256", "128", "0")]
 
 
-@pytest.mark.parametrize("variant", GEMM_VARIANTS, ids=lambda v: "cg%s-bn%s-rb%s" % v)
+@pytest.mark.parametrize("variant", GEMM_VARIANTS, ids=lambda v: "cg%s-bn%s-rb%s-wide%s" % v)
 @pytest.mark.parametrize("shape", BF16_SHAPES, ids=lambda s: s.name)
 def test_layer_parity_every_token_bf16(shape, variant, monkeypatch):
     """Every GEMM variant: single-CTA tiles of 128 or 32 token rows, CTA-pair
-    tiles (256 rows, or 128 for an expert's short last block), the hybrid
-    (pairs on whole 256-row blocks, single CTAs on the rest), and 256- or
-    128-column up-projection tiles (pairs always use 256)."""
-    cta_group, bn, rb = variant
+    tiles (256 rows, or 128 for an expert's short last block) 256 or 512
+    columns wide, the hybrid (pairs on whole 256-row blocks, single CTAs on
+    the rest), and 256- or 128-column up-projection tiles (pairs always use
+    256-column MMAs)."""
+    cta_group, bn, rb, wide = variant
     monkeypatch.setenv("MOE_GEMM_CTA_GROUP", cta_group)
     monkeypatch.setenv("MOE_GEMM_BN", bn)
     monkeypatch.setenv("MOE_GEMM_RB", rb)
+    monkeypatch.setenv("MOE_GEMM_WIDE", wide)
     rel, _ = full_check(shape)
     assert rel <= 1e-2
 
@@ -200,12 +203,13 @@ def test_layer_parity_every_token_bf16(shape, variant, monkeypatch):
 BLOCK_SIZES = [1, 64, 65, 128, 129, 200, 384, 385]
 
 
-@pytest.mark.parametrize("cta_group", ["1", "2", "h"])
-def test_expert_blocks_at_tile_edges(cta_group, monkeypatch):
+@pytest.mark.parametrize("cta_group,wide", [("1", "0"), ("2", "0"), ("2", "1"), ("h", "0")])
+def test_expert_blocks_at_tile_edges(cta_group, wide, monkeypatch):
     """moe_expert_ffn on a routing built to give the experts the block sizes
     above (k = 1, tokens shuffled, arbitrary gate weights), ragged in both
     output widths (f = 320, d = 384), against the oracle on every token."""
     monkeypatch.setenv("MOE_GEMM_CTA_GROUP", cta_group)
+    monkeypatch.setenv("MOE_GEMM_WIDE", wide)
     E, d, f = len(BLOCK_SIZES), 384, 320
     T = sum(BLOCK_SIZES)
     s = synth.MoEShape("blocks", T, d, f, E, 1, "bf16")
@@ -368,15 +372,17 @@ def test_prefill_full_shape(mixtral_weights):
     big_check("prefill", mixtral_weights, 256)
 
 
-@pytest.mark.parametrize("name,cta_group,bn,rb", [("decode", "2", "256", "128"), ("decode", "1", "256", "128"),
-                                                  ("decode", "h", "256", "128"),
-                                                  ("prefill", "1", "128", "128"), ("prefill", "2", "256", "128"),
-                                                  ("prefill", "1", "256", "128"), ("prefill", "1", "256", "32")])
-def test_full_shapes_other_gemm_variant(name, cta_group, bn, rb, mixtral_weights, monkeypatch):
+@pytest.mark.parametrize("name,cta_group,bn,rb,wide", [
+    ("decode", "2", "256", "128", "0"), ("decode", "2", "256", "128", "1"), ("decode", "1", "256", "128", "0"),
+    ("decode", "h", "256", "128", "0"),
+    ("prefill", "1", "128", "128", "0"), ("prefill", "2", "256", "128", "0"), ("prefill", "2", "256", "128", "1"),
+    ("prefill", "1", "256", "128", "0"), ("prefill", "1", "256", "32", "0")])
+def test_full_shapes_other_gemm_variant(name, cta_group, bn, rb, wide, mixtral_weights, monkeypatch):
     """Variants the size heuristics do not pick, at the full shapes."""
     monkeypatch.setenv("MOE_GEMM_CTA_GROUP", cta_group)
     monkeypatch.setenv("MOE_GEMM_BN", bn)
     monkeypatch.setenv("MOE_GEMM_RB", rb)
+    monkeypatch.setenv("MOE_GEMM_WIDE", wide)
     big_check(name, mixtral_weights, None if name == "decode" else 256)
 
 
