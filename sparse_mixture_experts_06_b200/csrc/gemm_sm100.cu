@@ -7,16 +7,16 @@
 //   down (second half and the gate weighting of §2.1 display 3):
 //         obuf_r = topk_w[perm[r]] * (W2_e h_r), fp32.
 //
-// Both are one persistent, warp-specialised kernel (192 threads per CTA):
+// Both are one persistent, warp-specialised kernel (320 threads per CTA):
 //   warp 0      TMA producer: 2-D tiled bulk copies (128-byte swizzle) of the
 //               A tile (token rows x 64 k) and the B tile (weight rows x 64 k)
 //               into a shared-memory ring of stages, signalled on mbarriers;
 //   warp 1      MMA issuer: one thread issues tcgen05.mma (bf16 x bf16 ->
 //               fp32, K = 16) into a tensor-memory (TMEM) accumulator and
 //               releases ring stages with tcgen05.commit;
-//   warps 2-5   epilogue: tcgen05.ld of the accumulator (each warp owns the
-//               32 TMEM lanes of its quadrant), fused SiLU(a)*b or gate
-//               scaling, and the stores.
+//   warps 2-9   epilogue: tcgen05.ld of the accumulator (two warps per
+//               quadrant of 32 TMEM lanes, splitting the tile's columns),
+//               fused SiLU(a)*b or gate scaling, and the stores.
 // Tile shapes (template variants; the host picks one per launch):
 //   single CTA   128 (or 32) rows x 256 columns, M = 128 N = 256 MMAs; two
 //                TMEM accumulators, so a tile's epilogue overlaps the next
@@ -68,7 +68,8 @@ constexpr int BM = 128;            // tile rows (permuted tokens)
 constexpr int BK = 64;             // k per stage: 64 bf16 = one 128-byte swizzle row
 constexpr int UMMA_K = 16;         // k per tcgen05.mma (kind::f16)
 constexpr int A_TILE = BM * BK * 2;            // 16 KiB: 128 rows x 64 k
-constexpr int NUM_THREADS = 192;
+constexpr int kEpiWarps = 8;                  // two per TMEM lane quadrant
+constexpr int NUM_THREADS = 64 + 32 * kEpiWarps;
 constexpr int TMEM_COLS = 512;                 // 2 accumulators x 256 fp32 columns
 constexpr unsigned long long kTimeoutNs = 4000000000ull;
 
@@ -281,7 +282,7 @@ __device__ __forceinline__ void tma_store_2d(const CUtensorMap* map, uint32_t sr
                  : "memory");
 }
 __device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
-__device__ __forceinline__ void bulk_wait_read_le1() { asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory"); }
+__device__ __forceinline__ void bulk_wait_read_all() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
 __device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
 __device__ __forceinline__ void fence_proxy_async_smem() {
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
@@ -291,13 +292,13 @@ __device__ __forceinline__ void st_shared_v4(uint32_t addr, uint4 v) {
                  : "memory");
 }
 
-// Epilogue staging: each of the 4 epilogue warps owns two 4 KiB buffers
-// (double buffering) holding one 32-row x 128-byte output box in the
-// 128-byte swizzled layout the store's tensor map expects: 16-byte chunk j
-// of row r sits at r * 128 + ((j ^ (r & 7)) << 4), which also makes the 32
-// lanes' shared-memory writes conflict-free.
+// Epilogue staging: each of the 8 epilogue warps owns a 4 KiB buffer
+// holding one 32-row x 128-byte output box in the 128-byte swizzled layout
+// the store's tensor map expects: 16-byte chunk j of row r sits at
+// r * 128 + ((j ^ (r & 7)) << 4), which also makes the 32 lanes'
+// shared-memory writes conflict-free.
 constexpr int kOutBoxBytes = 32 * 128;
-constexpr int kOutBytes = 4 * 2 * kOutBoxBytes;
+constexpr int kOutBytes = kEpiWarps * kOutBoxBytes;
 
 // ---------------------------------------------------------------------------
 // Per-variant constants.  BN = accumulator columns of a tile (the MMA's N):
@@ -406,14 +407,14 @@ __device__ __forceinline__ bool wait_bounded_pair(uint32_t bar, uint32_t parity,
 
 // Tile-number ring between the producer that takes tiles from the global
 // counter and the roles that follow it.  Readers of a slot: the MMA thread
-// and the 4 epilogue warps of the CTA, and for pairs also the odd CTA's
-// producer and its 4 epilogue warps (they read the copy the even CTA's
+// and the kEpiWarps epilogue warps of the CTA, and for pairs also the odd
+// CTA's producer and its epilogue warps (they read the copy the even CTA's
 // producer writes into the odd CTA's ring).  The slot's empty barrier lives
 // in the even CTA.  A tile number of -1 ends the loops.
 constexpr int kSchedSlots = 4;
 template <int CG>
 struct Sched {
-    static constexpr uint32_t kReaders = (CG == 1) ? 5u : 10u;
+    static constexpr uint32_t kReaders = (CG == 1) ? 1u + kEpiWarps : 2u * (1u + kEpiWarps);
 };
 
 template <int MODE, int CG, int BN, int RB, int NH>
@@ -455,7 +456,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
         }
         for (int a = 0; a < 2; ++a) {
             mbar_init(smem_u32(&tfull[a]), 1);
-            mbar_init(smem_u32(&tempty[a]), 4 * CG);  // one arrival per epilogue warp of the tile
+            mbar_init(smem_u32(&tempty[a]), kEpiWarps * CG);  // one arrival per epilogue warp of the tile
         }
         for (int q = 0; q < kSchedSlots; ++q) {
             mbar_init(smem_u32(&sfull[q]), 1);
@@ -648,11 +649,15 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
         __syncwarp();
     } else {
         // ---------------------------------------------------- epilogue (both CTAs)
+        // Two warps per TMEM lane quadrant (warp % 4 selects the lanes a warp
+        // may read); of the tile's output units (64-hidden-unit segments of
+        // the up-projection, 32-column boxes of the down-projection, over all
+        // MMA parts) warp sub = 0 takes the even ones and sub = 1 the odd ones.
         const int quad = warp & 3;  // TMEM lanes 32*quad .. 32*quad+31
+        const int sub = (warp - 2) >> 2;
         const uint32_t t_lane = tmem_base + ((uint32_t)(quad * 32) << 16);
         const uint32_t tempty_leader0 = (CG == 2) ? map_to_rank(smem_u32(&tempty[0]), 0) : 0u;
-        const uint32_t out_base = smem_u32(sOut) + (uint32_t)quad * 2u * kOutBoxBytes;
-        uint32_t obox = 0;  // boxes this warp has staged (selects the buffer)
+        const uint32_t buf = smem_u32(sOut) + (uint32_t)(warp - 2) * kOutBoxBytes;
         uint32_t tcount = 0;
         for (;; ++tcount) {
             bool got = true;
@@ -687,6 +692,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
             // expert's rows)
             const int wrow0 = row - lane;
             const bool box_ok = wrow0 + 32 <= tile_end;
+            int unit = 0;  // output units of the tile so far (this warp takes unit % 2 == sub)
             // MMA h of the tile: accumulator columns h * BN .. h * BN + BN-1,
             // output columns from hb (hidden units, up) or ob (down)
 #pragma unroll 1
@@ -706,12 +712,12 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
                     const int nseg = (CG == 1) ? BN / 128 : (shrt ? 1 : 2);
                     const int bdelta = (CG == 1) ? BN / 2 : 64;
     #pragma unroll 1
-                    for (int seg = 0; seg < nseg; ++seg, ++obox) {
+                    for (int seg = 0; seg < nseg; ++seg) {
+                        if ((unit++ & 1) != sub) continue;
                         const int c64 = (shrt ? colhalf : seg) * 64;        // hidden offset in the tile
                         const int acol = (CG == 1) ? seg * 64 : (shrt ? 0 : seg * 128);
-                        const uint32_t buf = out_base + (obox & 1u) * kOutBoxBytes;
                         if (box_ok) {
-                            if (lane == 0) bulk_wait_read_le1();  // this buffer's previous store has read it
+                            if (lane == 0) bulk_wait_read_all();  // the buffer's previous store has read it
                             __syncwarp();
                         }
     #pragma unroll 1
@@ -767,11 +773,11 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
                     const int ncol = shrt ? BN / 2 : BN;
                     const int cbase = colhalf * (BN / 2);
     #pragma unroll 1
-                    for (int cc = 0; cc < ncol; cc += 32, ++obox) {
+                    for (int cc = 0; cc < ncol; cc += 32) {
+                        if ((unit++ & 1) != sub) continue;
                         const int c = cbase + cc;  // tile column
-                        const uint32_t buf = out_base + (obox & 1u) * kOutBoxBytes;
                         if (box_ok) {
-                            if (lane == 0) bulk_wait_read_le1();
+                            if (lane == 0) bulk_wait_read_all();  // the buffer's previous store has read it
                             __syncwarp();
                         }
                         uint32_t o[32];
