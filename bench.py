@@ -54,7 +54,7 @@ def parse():
                     help="tokens in the oracle's timed CPU-baseline sample (default: the whole prefill batch)")
     ap.add_argument("--ref-sample", type=int, default=128,
                     help="tokens per step of --impl reference (keeps --steps K --warmup W within minutes)")
-    ap.add_argument("--e2e-chunks", type=int, default=2,
+    ap.add_argument("--e2e-chunks", type=int, default=1,
                     help="pieces the end-to-end leg pipelines host copies and compute in")
     ap.add_argument("--gemm-vs-cublas", action="store_true",
                     help="instead of the layer: time the two expert GEMMs against cuBLAS (torch.matmul) "
@@ -370,9 +370,12 @@ def graph_step_ms(r, s, device, steps):
 
 def e2e_leg(args, s, t, device, steps):
     """Same layer through the public host-buffer entry point
-    moe_layer_forward_host: the step's tokens come from pinned host memory
-    and the output goes back to it, copies pipelined with the compute in
-    args.e2e_chunks pieces, all inside the timed region."""
+    moe_layer_forward_host, as a server calls it back to back: every step
+    copies its tokens in from pinned host memory and its output back, inside
+    the timed region; the library pipelines those copies with the compute of
+    the neighbouring pieces (args.e2e_chunks per step, staging alternating
+    across steps; x_ready, since the host tokens are ready at each call, and
+    y_async, with one moe_layer_forward_host_wait before the end event)."""
     import torch
     import sparse_mixture_experts_06_b200 as moe
     x_h = t["x"].cpu().pin_memory()
@@ -381,7 +384,7 @@ def e2e_leg(args, s, t, device, steps):
 
     def step():
         moe.moe_layer_forward_host(x_h, t["Wg"], t["W1"], t["W3"], t["W2"], s.k, y=y_h, chunks=args.e2e_chunks,
-                                   stream=stream)
+                                   x_ready=True, y_async=True, stream=stream)
 
     for _ in range(3):
         step()
@@ -390,6 +393,7 @@ def e2e_leg(args, s, t, device, steps):
     a.record(stream)
     for _ in range(steps):
         step()
+    moe.moe_layer_forward_host_wait(stream)  # the end event follows the last step's copy out
     b.record(stream)
     torch.cuda.synchronize(device)
     ms = a.elapsed_time(b) / steps
@@ -566,8 +570,9 @@ def main():
     if rank == 0:
         line["e2e"] = {"value": world * s.T / (e_ms * 1e-3), "unit": "tokens/s", "h2d_bytes_per_step": hb,
                        "d2h_bytes_per_step": db, "ms_per_step": e_ms, "chunks": args.e2e_chunks,
-                       "path": "pinned host x -> moe_layer_forward_host (copies pipelined with the layer "
-                               "in %d pieces) -> pinned host y" % args.e2e_chunks}
+                       "path": "pinned host x -> moe_layer_forward_host (x_ready, y_async; each step's "
+                               "copies pipelined with the compute of neighbouring pieces, %d per step) -> "
+                               "pinned host y" % args.e2e_chunks}
     del r
     torch.cuda.empty_cache()
 

@@ -64,6 +64,14 @@ enum {
     MOE_ERR_CUDA = 4         /* a CUDA call failed; see moe_last_error_string()     */
 };
 
+/* Flags of moe_layer_forward_host. */
+enum {
+    MOE_HOST_X_READY = 1, /* x_host holds its values at the call (no work still queued on the
+                             stream writes it), so its copies may start before that work ends */
+    MOE_HOST_Y_ASYNC = 2  /* later work on the stream is not ordered after this call's copies
+                             out; moe_layer_forward_host_wait() orders it (before reading y) */
+};
+
 /* Device-side flags reported by moe_device_errors(). */
 enum {
     MOE_DEVERR_PIPELINE_TIMEOUT = 1u, /* a GEMM pipeline wait gave up (kernel returned early)  */
@@ -131,19 +139,35 @@ int moe_layer_forward(const void* x, const void* Wg, const void* W1, const void*
 /* The bf16 layer on HOST x and y [T, d] (the serving entry: tokens arrive in
  * and leave host memory).  The T tokens are processed in `chunks` pieces of
  * ceil(T / chunks) tokens (chunks >= 1; tokens are independent, so the
- * result does not depend on the split): while piece c runs on `stream`, the
- * rows of piece c+1 are copied in and those of piece c-1 copied out on two
- * library-owned copy streams, ordered with events against `stream`.  The
- * device staging buffers (2 x and 2 y pieces) share the library workspace
- * of moe_layer_forward.  Weights are device pointers as elsewhere; x_host
- * and y_host need no alignment, and copies overlap only if they are
- * page-locked (cudaHostAlloc / cudaHostRegister).  Asynchronous like the
- * other calls: y_host is complete once `stream` has been synchronised.
- * Pipelining of host copies with compute has no counterpart in the pages;
- * the layer itself is the one moe_layer_forward computes. */
+ * result does not depend on the split).  Each piece's x rows are copied in
+ * on a library-owned copy stream, the layer runs on `stream`, and its y
+ * rows are copied out on a second copy stream, all ordered with events.
+ * Pieces alternate between two device staging buffers, counted across
+ * calls, so the copies of one piece overlap the compute of the neighbouring
+ * pieces, including the last piece of the previous call and the first of
+ * the next one.  Without MOE_HOST_X_READY in `flags` the first copy in waits
+ * for all work already on `stream`; with it, copies in wait only for their
+ * staging buffer to be free (use it when x_host is not produced by work
+ * still queued on `stream`).  The layer uses the workspace of
+ * moe_layer_forward; the staging (2 x and 2 y pieces) is a separate
+ * library allocation.  Weights are device pointers as elsewhere; x_host and
+ * y_host need no alignment, and copies overlap only if they are page-locked
+ * (cudaHostAlloc / cudaHostRegister).  Asynchronous like the other calls:
+ * y_host is complete once `stream` has been synchronised.  Pipelining of
+ * host copies with compute has no counterpart in the pages; the layer
+ * itself is the one moe_layer_forward computes.  Unknown flags:
+ * MOE_ERR_INVALID_ARG.  Without MOE_HOST_Y_ASYNC, `stream` waits for the
+ * call's copies out, so synchronising `stream` completes y_host; with it,
+ * the next call's compute may overlap this call's copies out (a server's
+ * steady state), and moe_layer_forward_host_wait(stream) must be called
+ * before y_host is read. */
 int moe_layer_forward_host(const void* x_host, const void* Wg, const void* W1, const void* W3,
                            const void* W2, int T, int d, int f, int E, int k, void* y_host,
-                           int chunks, moe_stream_t stream);
+                           int chunks, int flags, moe_stream_t stream);
+
+/* Makes `stream` wait for every copy out that moe_layer_forward_host has
+ * enqueued on the current device (needed after MOE_HOST_Y_ASYNC calls). */
+int moe_layer_forward_host_wait(moe_stream_t stream);
 
 /* As moe_layer_forward with an explicit dtype and a caller-owned workspace.
  * If `residual` is not NULL it must be a [T, d] tensor of the same dtype and
@@ -187,8 +211,9 @@ int moe_layer_forward_noalloc(const void* x, const void* Wg, const void* W1, con
                               const void* W2, int T, int d, int f, int E, int k, void* y,
                               moe_stream_t stream);
 
-/* Frees the workspace moe_layer_forward keeps for the current device
- * (stream-ordered on `stream`). */
+/* Frees the workspace moe_layer_forward keeps for the current device and
+ * the staging of moe_layer_forward_host (stream-ordered on `stream`, after
+ * the copies that use it). */
 int moe_release_workspace(moe_stream_t stream);
 
 /* Synchronises the current device, returns the device-side flags

@@ -7,7 +7,8 @@ ABI of include/moe.h); this package is the thin Python binding over it.
 from .binding import (  # noqa: F401
     MOE_BF16, MOE_F32, MoEError, lib, lib_path,
     moe_workspace_size, moe_router_topk, moe_permute, moe_routing_stats, moe_expert_ffn,
-    moe_layer_forward, moe_layer_forward_ex, moe_layer_forward_host, moe_layer_forward_noalloc,
+    moe_layer_forward, moe_layer_forward_ex, moe_layer_forward_host, moe_layer_forward_host_wait,
+    moe_layer_forward_noalloc,
     moe_stack_forward,
     moe_release_workspace,
     moe_device_errors, moe_last_error_string, moe_version,

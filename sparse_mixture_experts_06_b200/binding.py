@@ -9,6 +9,7 @@ import ctypes
 import os
 
 MOE_BF16, MOE_F32 = 0, 1
+MOE_HOST_X_READY, MOE_HOST_Y_ASYNC = 1, 2
 _STATUS = {0: "MOE_OK", 1: "MOE_ERR_INVALID_ARG", 2: "MOE_ERR_UNSUPPORTED", 3: "MOE_ERR_WORKSPACE",
            4: "MOE_ERR_CUDA"}
 
@@ -27,7 +28,8 @@ _SIGS = {
     "moe_expert_ffn": ([_P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _P, _Z, _P, _P], _I),
     "moe_layer_forward": ([_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _P, _P], _I),
     "moe_layer_forward_ex": ([_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _P, _Z, _P, _P], _I),
-    "moe_layer_forward_host": ([_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _P, _I, _P], _I),
+    "moe_layer_forward_host": ([_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _P, _I, _I, _P], _I),
+    "moe_layer_forward_host_wait": ([_P], _I),
     "moe_layer_forward_noalloc": ([_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _P, _P], _I),
     "moe_stack_forward": ([_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _P, _P, _Z, _P, _P], _I),
     "moe_release_workspace": ([_P], _I),
@@ -196,11 +198,14 @@ def moe_layer_forward(x, Wg, W1, W3, W2, k, y=None, stream=None):
     return y
 
 
-def moe_layer_forward_host(x, Wg, W1, W3, W2, k, y=None, chunks=2, stream=None):
+def moe_layer_forward_host(x, Wg, W1, W3, W2, k, y=None, chunks=2, x_ready=False, y_async=False, stream=None):
     """The bf16 layer on host x / y (CPU tensors; page-locked for overlap),
     pipelined in `chunks` pieces; returns y (a pinned CPU tensor unless given).
-    Asynchronous: synchronise `stream` (default: the current stream of W1's
-    device) before reading y."""
+    x_ready=True passes MOE_HOST_X_READY (x's copies may start before work
+    already queued on the stream ends); y_async=True passes MOE_HOST_Y_ASYNC
+    (call moe_layer_forward_host_wait before reading y).  Asynchronous:
+    synchronise `stream` (default: the current stream of W1's device) before
+    reading y."""
     import torch
     _dev(Wg, W1, W3, W2)
     if x.is_cuda or not x.is_contiguous() or x.dtype != torch.bfloat16:
@@ -211,8 +216,15 @@ def moe_layer_forward_host(x, Wg, W1, W3, W2, k, y=None, chunks=2, stream=None):
     if y.is_cuda or not y.is_contiguous() or y.dtype != torch.bfloat16 or tuple(y.shape) != (T, d):
         raise ValueError("y must be a contiguous bfloat16 CPU tensor of shape [T, d]")
     _check(lib.moe_layer_forward_host(_ptr(x), _ptr(Wg), _ptr(W1), _ptr(W3), _ptr(W2), T, d, f, E, k, _ptr(y),
-                                      chunks, _stream(stream, W1)), "moe_layer_forward_host")
+                                      chunks, (MOE_HOST_X_READY if x_ready else 0) | (MOE_HOST_Y_ASYNC if y_async else 0),
+                                      _stream(stream, W1)), "moe_layer_forward_host")
     return y
+
+
+def moe_layer_forward_host_wait(stream=None):
+    """Orders `stream` (default: the current stream) after every copy out of
+    earlier moe_layer_forward_host calls on the current device."""
+    _check(lib.moe_layer_forward_host_wait(_stream(stream)), "moe_layer_forward_host_wait")
 
 
 def moe_layer_forward_noalloc(x, Wg, W1, W3, W2, k, y, stream=None):

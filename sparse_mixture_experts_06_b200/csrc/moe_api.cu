@@ -221,16 +221,24 @@ int pool_workspace(int dev, size_t need, cudaStream_t s, void** out) {
     return MOE_OK;
 }
 
-// Copy streams and events of moe_layer_forward_host, per device, created on
-// first use and kept for the life of the process.  Buffer b (0 or 1) of the
-// double-buffered x / y staging has: in_done[b] (its x rows have arrived),
-// comp_done[b] (the layer has read x and written y), out_done[b] (y has left).
+// Copy streams, events and staging memory of moe_layer_forward_host, per
+// device, created on first use and kept for the life of the process.  The
+// staging holds two x pieces and two y pieces; piece number n (counted
+// across calls) uses buffer n & 1, so consecutive pieces, also those of
+// consecutive calls, alternate.  Buffer b has: in_done[b] (its x rows have
+// arrived), comp_done[b] (the layer has read x and written y), out_done[b]
+// (y has left).  The staging is separate from the layer workspace, so work
+// that other calls put on the stream never touches it.
 struct HostPipe {
     cudaStream_t h2d = nullptr, d2h = nullptr;
     cudaEvent_t start = nullptr;
     cudaEvent_t in_done[2] = {nullptr, nullptr};
     cudaEvent_t comp_done[2] = {nullptr, nullptr};
     cudaEvent_t out_done[2] = {nullptr, nullptr};
+    void* stage = nullptr;
+    size_t stage_bytes = 0;
+    size_t piece_bytes = 0;   // staging piece size of the last call (the buffers' layout)
+    unsigned long long next_piece = 0;
     bool ready = false;
 };
 std::mutex g_pipe_mu;
@@ -246,6 +254,34 @@ cudaError_t pipe_init(HostPipe& P) {
         if (e == cudaSuccess) e = cudaEventCreateWithFlags(ev, cudaEventDisableTiming);
     P.ready = e == cudaSuccess;
     return e;
+}
+
+// Staging of at least `need` bytes.  Growing it frees the old buffers on s
+// after every copy and layer that used them (stream-ordered), then
+// allocates on s; *grown tells the caller that the copy streams must wait
+// for s before touching the new buffers.
+cudaError_t pipe_stage(HostPipe& P, size_t need, cudaStream_t s, bool* grown) {
+    *grown = false;
+    if (P.stage_bytes >= need) return cudaSuccess;
+    cudaError_t e = cudaSuccess;
+    if (P.stage) {
+        for (int b = 0; b < 2 && e == cudaSuccess; ++b) {
+            e = cudaStreamWaitEvent(s, P.in_done[b], 0);
+            if (e == cudaSuccess) e = cudaStreamWaitEvent(s, P.out_done[b], 0);
+        }
+        if (e == cudaSuccess) e = cudaFreeAsync(P.stage, s);
+        P.stage = nullptr;
+        P.stage_bytes = 0;
+        if (e != cudaSuccess) return e;
+    }
+    e = cudaMallocAsync(&P.stage, need, s);
+    if (e != cudaSuccess) {
+        P.stage = nullptr;
+        return e;
+    }
+    P.stage_bytes = need;
+    *grown = true;
+    return cudaSuccess;
 }
 
 }  // namespace
@@ -413,7 +449,7 @@ int moe_layer_forward(const void* x, const void* Wg, const void* W1, const void*
 
 int moe_layer_forward_host(const void* x_host, const void* Wg, const void* W1, const void* W3,
                            const void* W2, int T, int d, int f, int E, int k, void* y_host, int chunks,
-                           moe_stream_t stream) {
+                           int flags, moe_stream_t stream) {
     g_last_error.clear();
     CHECK(check_shape(T, d, f, E, k, MOE_BF16, true));
     if (T == 0) return MOE_OK;
@@ -424,6 +460,7 @@ int moe_layer_forward_host(const void* x_host, const void* Wg, const void* W1, c
     CHECK(check_ptr(W3, "W3"));
     CHECK(check_ptr(W2, "W2"));
     if (chunks < 1) return fail(MOE_ERR_INVALID_ARG, "chunks must be >= 1 (got %d)", chunks);
+    if (flags & ~(MOE_HOST_X_READY | MOE_HOST_Y_ASYNC)) return fail(MOE_ERR_INVALID_ARG, "unknown flags 0x%x", flags);
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
@@ -431,23 +468,33 @@ int moe_layer_forward_host(const void* x_host, const void* Wg, const void* W1, c
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
 
     const int C = chunks < T ? chunks : T;
-    const int Tc = (T + C - 1) / C;  // tokens per chunk (the last may be shorter)
+    const int Tc = (T + C - 1) / C;  // tokens per piece (the last may be shorter)
     const size_t ws_need = moe_workspace_size(Tc, d, f, E, k, MOE_BF16);
     const size_t row_bytes = (size_t)d * 2;
     const size_t buf = align256((size_t)Tc * row_bytes);
-    void* base = nullptr;
-    CHECK(pool_workspace(dev, ws_need + 4 * buf, s, &base));
-    char* xbuf[2] = {static_cast<char*>(base) + ws_need, static_cast<char*>(base) + ws_need + buf};
-    char* ybuf[2] = {xbuf[1] + buf, xbuf[1] + 2 * buf};
+    void* ws = nullptr;
+    CHECK(pool_workspace(dev, ws_need, s, &ws));
 
     std::lock_guard<std::mutex> lock(g_pipe_mu);
     HostPipe& P = g_pipe[dev];
     if ((e = pipe_init(P)) != cudaSuccess) return cuda_fail(e, "creating the copy streams");
-    // the copies follow everything already on s (earlier calls, workspace growth)
-    if ((e = cudaEventRecord(P.start, s)) != cudaSuccess ||
-        (e = cudaStreamWaitEvent(P.h2d, P.start, 0)) != cudaSuccess ||
-        (e = cudaStreamWaitEvent(P.d2h, P.start, 0)) != cudaSuccess)
-        return cuda_fail(e, "ordering the copy streams");
+    bool grown = false;
+    if ((e = pipe_stage(P, 4 * buf, s, &grown)) != cudaSuccess) return cuda_fail(e, "allocating the staging");
+    char* xbuf[2] = {static_cast<char*>(P.stage), static_cast<char*>(P.stage) + buf};
+    char* ybuf[2] = {xbuf[1] + buf, xbuf[1] + 2 * buf};
+    // The copies in wait for everything already on s (x_host may be written
+    // by it), unless the caller says x_host is ready now; either way they
+    // wait for s after a staging (re)allocation or a change of piece size
+    // (the buffers then overlap differently: the events of the previous
+    // pieces no longer describe them; s itself follows every earlier copy).
+    const bool relayout = P.piece_bytes != buf;
+    P.piece_bytes = buf;
+    if (grown || relayout || !(flags & MOE_HOST_X_READY)) {
+        if ((e = cudaEventRecord(P.start, s)) != cudaSuccess ||
+            (e = cudaStreamWaitEvent(P.h2d, P.start, 0)) != cudaSuccess ||
+            (e = cudaStreamWaitEvent(P.d2h, P.start, 0)) != cudaSuccess)
+            return cuda_fail(e, "ordering the copy streams");
+    }
     const char* xh = static_cast<const char*>(x_host);
     char* yh = static_cast<char*>(y_host);
     bool used[2] = {false, false};
@@ -455,19 +502,19 @@ int moe_layer_forward_host(const void* x_host, const void* Wg, const void* W1, c
         const int t0 = c * Tc;
         const int tc = T - t0 < Tc ? T - t0 : Tc;
         if (tc <= 0) break;
-        const int b = c & 1;
+        const int b = (int)(P.next_piece++ & 1ull);
         const size_t off = (size_t)t0 * row_bytes, bytes = (size_t)tc * row_bytes;
-        // x rows in, once the layer two chunks back has finished reading buffer b
-        if (used[b] && (e = cudaStreamWaitEvent(P.h2d, P.comp_done[b], 0)) != cudaSuccess)
-            return cuda_fail(e, "cudaStreamWaitEvent");
-        if ((e = cudaMemcpyAsync(xbuf[b], xh + off, bytes, cudaMemcpyHostToDevice, P.h2d)) != cudaSuccess ||
+        // x rows in, once the layer that last used buffer b has read it (a
+        // never-recorded event is already complete)
+        if ((e = cudaStreamWaitEvent(P.h2d, P.comp_done[b], 0)) != cudaSuccess ||
+            (e = cudaMemcpyAsync(xbuf[b], xh + off, bytes, cudaMemcpyHostToDevice, P.h2d)) != cudaSuccess ||
             (e = cudaEventRecord(P.in_done[b], P.h2d)) != cudaSuccess)
             return cuda_fail(e, "copying x to the device");
         // the layer, once x has arrived and y buffer b has been copied out
         if ((e = cudaStreamWaitEvent(s, P.in_done[b], 0)) != cudaSuccess ||
-            (used[b] && (e = cudaStreamWaitEvent(s, P.out_done[b], 0)) != cudaSuccess))
+            (e = cudaStreamWaitEvent(s, P.out_done[b], 0)) != cudaSuccess)
             return cuda_fail(e, "cudaStreamWaitEvent");
-        CHECK(moe_layer_forward_ex(xbuf[b], Wg, W1, W3, W2, nullptr, tc, d, f, E, k, MOE_BF16, base, ws_need,
+        CHECK(moe_layer_forward_ex(xbuf[b], Wg, W1, W3, W2, nullptr, tc, d, f, E, k, MOE_BF16, ws, ws_need,
                                    ybuf[b], stream));
         if ((e = cudaEventRecord(P.comp_done[b], s)) != cudaSuccess)
             return cuda_fail(e, "cudaEventRecord");
@@ -478,9 +525,28 @@ int moe_layer_forward_host(const void* x_host, const void* Wg, const void* W1, c
             return cuda_fail(e, "copying y to the host");
         used[b] = true;
     }
-    // work later enqueued on s (and a synchronize of s) also covers the copies out
+    // work later enqueued on s (and a synchronize of s) also covers the
+    // copies out, unless the caller orders them later (moe_layer_forward_host_wait)
+    if (!(flags & MOE_HOST_Y_ASYNC))
+        for (int b = 0; b < 2; ++b)
+            if (used[b] && (e = cudaStreamWaitEvent(s, P.out_done[b], 0)) != cudaSuccess)
+                return cuda_fail(e, "cudaStreamWaitEvent");
+    return MOE_OK;
+}
+
+int moe_layer_forward_host_wait(moe_stream_t stream) {
+    g_last_error.clear();
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+    if (dev >= 64) return MOE_OK;
+    std::lock_guard<std::mutex> lock(g_pipe_mu);
+    HostPipe& P = g_pipe[dev];
+    if (!P.ready) return MOE_OK;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    // the copy-out stream is serial: its latest event covers every earlier copy
     for (int b = 0; b < 2; ++b)
-        if (used[b] && (e = cudaStreamWaitEvent(s, P.out_done[b], 0)) != cudaSuccess)
+        if ((e = cudaStreamWaitEvent(s, P.out_done[b], 0)) != cudaSuccess)
             return cuda_fail(e, "cudaStreamWaitEvent");
     return MOE_OK;
 }
@@ -491,13 +557,28 @@ int moe_release_workspace(moe_stream_t stream) {
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
     if (dev >= 64) return MOE_OK;
-    std::lock_guard<std::mutex> lock(g_pool_mu);
-    Pool& p = g_pool[dev];
-    if (p.ptr) {
-        e = cudaFreeAsync(p.ptr, reinterpret_cast<cudaStream_t>(stream));
-        p.ptr = nullptr;
-        p.bytes = 0;
-        if (e != cudaSuccess) return cuda_fail(e, "cudaFreeAsync(workspace)");
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    {
+        std::lock_guard<std::mutex> lock(g_pool_mu);
+        Pool& p = g_pool[dev];
+        if (p.ptr) {
+            e = cudaFreeAsync(p.ptr, s);
+            p.ptr = nullptr;
+            p.bytes = 0;
+            if (e != cudaSuccess) return cuda_fail(e, "cudaFreeAsync(workspace)");
+        }
+    }
+    std::lock_guard<std::mutex> lock(g_pipe_mu);
+    HostPipe& P = g_pipe[dev];
+    if (P.stage) {
+        for (int b = 0; b < 2 && e == cudaSuccess; ++b) {
+            e = cudaStreamWaitEvent(s, P.in_done[b], 0);
+            if (e == cudaSuccess) e = cudaStreamWaitEvent(s, P.out_done[b], 0);
+        }
+        if (e == cudaSuccess) e = cudaFreeAsync(P.stage, s);
+        P.stage = nullptr;
+        P.stage_bytes = 0;
+        if (e != cudaSuccess) return cuda_fail(e, "cudaFreeAsync(staging)");
     }
     return MOE_OK;
 }

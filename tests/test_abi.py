@@ -131,7 +131,7 @@ def test_host_layer_rejects_invalid_arguments():
     call (fake pointers; the valid list itself is never called)."""
     P = ctypes.c_void_p
     f = moe.lib.moe_layer_forward_host
-    args = [P(8)] + [P(16)] * 4 + [16, 64, 128, 8, 2, P(8), 2, None]
+    args = [P(8)] + [P(16)] * 4 + [16, 64, 128, 8, 2, P(8), 2, 0, None]
     bad = list(args); bad[0] = None                            # x_host NULL
     assert f(*bad) == 1 and "x_host" in moe.moe_last_error_string()
     bad = list(args); bad[10] = None                           # y_host NULL
@@ -142,6 +142,8 @@ def test_host_layer_rejects_invalid_arguments():
     assert f(*bad) == 1 and "aligned" in moe.moe_last_error_string()
     bad = list(args); bad[9] = 9                               # k > E
     assert f(*bad) == 1
+    bad = list(args); bad[12] = 6                              # unknown flag bits
+    assert f(*bad) == 1 and "flags" in moe.moe_last_error_string()
     bad = list(args); bad[5] = 0; bad[0] = None; bad[10] = None  # T = 0: a no-op
     assert f(*bad) == 0
 

@@ -71,6 +71,50 @@ def test_host_layer_more_chunks_than_tokens_and_repeat_calls():
         assert_close(y.float().double().numpy(), y_ref, "bf16")
 
 
+@pytest.mark.parametrize("x_ready,y_async", [(False, False), (True, False), (True, True)])
+def test_host_layer_back_to_back_calls_alternate_buffers(x_ready, y_async):
+    """Many calls in a row without a host synchronisation, piece sizes
+    changing between calls (the staging layout changes) and host inputs
+    that differ per call: every call's y matches the device path on its own
+    x.  With x_ready the copies of a call may start while the previous call
+    still computes; with y_async its copies out may overlap the next call,
+    and moe_layer_forward_host_wait orders the stream after them."""
+    s = synth.MoEShape("host-b2b", 600, 128, 256, 8, 2, "bf16")
+    t = device_inputs(s, 23)
+    xs = [(t["x"] * (1.0 + 0.25 * i)).to(torch.bfloat16) for i in range(6)]
+    xs_h = [x.cpu().pin_memory() for x in xs]
+    plan = [1, 1, 2, 2, 3, 1]
+    ys = [moe.moe_layer_forward_host(xh, t["Wg"], t["W1"], t["W3"], t["W2"], 2, chunks=c, x_ready=x_ready,
+                                     y_async=y_async)
+          for xh, c in zip(xs_h, plan)]
+    if y_async:
+        moe.moe_layer_forward_host_wait()
+    torch.cuda.current_stream().synchronize()
+    for x, c, y in zip(xs, plan, ys):
+        tt = dict(t, x=x)
+        ref = piecewise_device(tt, 2, c).cpu()
+        assert torch.equal(y.view(torch.int16), ref.view(torch.int16))
+
+
+def test_host_layer_chained_through_host_memory():
+    """Without x_ready, a call whose x_host is the y_host of the call before
+    (written by that call's copy out, still queued on the stream) reads the
+    finished values: two layers chained through pinned host memory equal two
+    device layers."""
+    s = synth.MoEShape("host-chain", 300, 128, 256, 8, 2, "bf16")
+    t = device_inputs(s, 24)
+    x_h = t["x"].cpu().pin_memory()
+    mid = torch.empty_like(x_h).pin_memory()
+    out = torch.empty_like(x_h).pin_memory()
+    moe.moe_layer_forward_host(x_h, t["Wg"], t["W1"], t["W3"], t["W2"], 2, y=mid, chunks=2)
+    moe.moe_layer_forward_host(mid, t["Wg"], t["W1"], t["W3"], t["W2"], 2, y=out, chunks=3)
+    torch.cuda.current_stream().synchronize()
+    ref1 = piecewise_device(t, 2, 2)
+    assert torch.equal(mid.view(torch.int16), ref1.cpu().view(torch.int16))
+    y2 = piecewise_device(dict(t, x=ref1), 2, 3)
+    assert torch.equal(out.view(torch.int16), y2.cpu().view(torch.int16))
+
+
 def test_host_layer_prefill_shape_two_chunks():
     s = synth.CONFIGS["prefill"]
     t = device_inputs(s, 0)
