@@ -200,7 +200,7 @@ int moe_stack_forward(const void* x, const void* const* Wg, const void* const* W
  * counterpart in the paper: it is a deployment convenience of this library.
  * Instead of allocating, it uses a 32 MiB scratch array compiled into the
  * library (kept by every GPU that loads it until the process exits), which
- * covers T*k*(2d + 2f + 4d) bytes plus routing buffers: up to 316 tokens at
+ * covers T*k*(2d + 2f + 4d) bytes plus routing buffers: up to 314 tokens at
  * the Mixtral-8x7B dimensions.  Larger shapes return MOE_ERR_WORKSPACE with a
  * message naming the bytes needed.  The first call on each device looks up
  * the array's device address (cudaGetSymbolAddress) with that device

@@ -12,7 +12,7 @@
 //
 // The scratch is a file-scope device array of kStaticScratchBytes (32 MiB),
 // enough for T*k*(2d + 2f + 4d) bytes plus small routing buffers: at the
-// Mixtral-8x7B dimensions (d = 4096, f = 14336, k = 2) that is up to 316
+// Mixtral-8x7B dimensions (d = 4096, f = 14336, k = 2) that is up to 314
 // tokens per call.  Every GPU that loads this part of the library keeps the
 // 32 MiB until the process exits.  In host code the array's name is only a
 // stand-in, so its device address is looked up with cudaGetSymbolAddress on

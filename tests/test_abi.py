@@ -164,3 +164,12 @@ def test_stack_rejects_invalid_arguments():
     assert f(*bad) == 1                                   # scratch aliases y
     bad = list(base); bad[14] = 100
     assert f(*bad) == 1 or f(*bad) == 3                   # never launched: fails before or at the workspace check
+
+
+def test_noalloc_token_limit_matches_its_documentation():
+    """The static scratch of moe_layer_forward_noalloc (32 MiB) holds the
+    workspace of up to 314 tokens at the Mixtral-8x7B dimensions, as its
+    declaration says; 315 does not fit."""
+    cap = 32 << 20
+    assert moe.moe_workspace_size(314, 4096, 14336, 8, 2, 0) <= cap
+    assert moe.moe_workspace_size(315, 4096, 14336, 8, 2, 0) > cap
