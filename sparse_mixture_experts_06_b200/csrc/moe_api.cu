@@ -99,6 +99,7 @@ Workspace carve_workspace(void* base, int T, int d, int f, int E, int k, bool bf
     w.h = take(n * f * (bf16 ? 2 : 4));
     w.obuf = reinterpret_cast<float*>(take(n * d * 4));
     w.tile_counters = reinterpret_cast<int32_t*>(take(kTileCounters * 4));
+    w.chunk_base = reinterpret_cast<int32_t*>(take((size_t)E * ((n + kChunkA - 1) / kChunkA) * 4));
     w.bytes = off;
     return w;
 }
@@ -140,22 +141,24 @@ struct StageTimer {
     }
 };
 
-// Experts + combine on carved workspace `w` (routing fields supplied by the caller).
+// Experts + combine on carved workspace `w` (routing fields supplied by the
+// caller).  x_gathered: w.x_perm already holds the permuted rows of x and the
+// tile counters are zero (the chunked permutation did both).
 int run_ffn(const void* x, const void* W1, const void* W3, const void* W2, const int32_t* offsets,
             const int32_t* perm, const int32_t* inv, const float* topk_w, const void* residual,
             int T, int d, int f, int E, int k, bool bf16, const moe::Workspace& w, void* y,
-            cudaStream_t s) {
+            cudaStream_t s, bool x_gathered = false) {
     const int rows = T * k;
     cudaError_t e;
     if (bf16) {
         if (const char* msg = moe::gemm_init_error()) return fail(MOE_ERR_CUDA, "%s", msg);
-        {
+        if (!x_gathered) {
             StageTimer tm(kGather, s);
             e = moe::launch_gather_rows_bf16(static_cast<const __nv_bfloat16*>(x), perm, rows, d, k,
                                              static_cast<__nv_bfloat16*>(w.x_perm), w.tile_counters, s);
             tm.done(s);
+            if (e != cudaSuccess) return cuda_fail(e, "gather_rows");
         }
-        if (e != cudaSuccess) return cuda_fail(e, "gather_rows");
         unsigned int* err = moe::device_error_word();
         if (!err) return fail(MOE_ERR_CUDA, "cannot locate the device error word");
         moe::GroupedGemmArgs a{offsets, E, rows, d, f, num_sms_current(), err, w.tile_counters};
@@ -390,14 +393,26 @@ int moe_layer_forward_ex(const void* x, const void* Wg, const void* W1, const vo
         tm.done(s);
     }
     if (e != cudaSuccess) return cuda_fail(e, "router_topk");
+    // chunked permutation: counts and scan ("permute" stage), then the
+    // stable scatter with the x row copies ("gather_rows" stage)
+    const bool chunked = moe::chunked_permute_fits(T * k, E);
     {
         StageTimer tm(kPermute, s);
-        e = moe::launch_permute(w.topk_idx, T * k, E, w.offsets, w.perm, w.inv, s);
+        e = chunked ? moe::launch_chunk_count_scan(w.topk_idx, T * k, E, w.chunk_base, w.offsets, s)
+                    : moe::launch_permute(w.topk_idx, T * k, E, w.offsets, w.perm, w.inv, s);
         tm.done(s);
     }
     if (e != cudaSuccess) return cuda_fail(e, "permute");
+    if (chunked) {
+        StageTimer tm(kGather, s);
+        e = moe::launch_chunk_scatter(w.topk_idx, T * k, E, k, w.chunk_base, w.perm, w.inv,
+                                      bf16 ? static_cast<const __nv_bfloat16*>(x) : nullptr, d,
+                                      bf16 ? static_cast<__nv_bfloat16*>(w.x_perm) : nullptr, w.tile_counters, s);
+        tm.done(s);
+        if (e != cudaSuccess) return cuda_fail(e, "permutation scatter");
+    }
     return run_ffn(x, W1, W3, W2, w.offsets, w.perm, w.inv, w.topk_w, residual, T, d, f, E, k, bf16, w,
-                   y, s);
+                   y, s, chunked);
 }
 
 int moe_stack_forward(const void* x, const void* const* Wg, const void* const* W1, const void* const* W3,

@@ -18,6 +18,8 @@ void set_last_error(const char* msg);
 constexpr int kMaxExperts = 64;
 constexpr int kMaxTopK = kMaxExperts;  // any k <= E
 constexpr int kTileCounters = 4;        // up, up (second hybrid launch), down, down (second)
+constexpr int kChunkA = 64;             // assignments per chunk of the layer's permutation
+constexpr int kChunkScanMaxCells = 48 * 1024;  // E x chunks counted in shared memory (192 KiB)
 
 // 256-byte aligned carve-up of one workspace blob.
 struct Workspace {
@@ -30,6 +32,7 @@ struct Workspace {
     void* h;            // [T*k, f]  bf16 or f32
     float* obuf;        // [T*k, d]  gate-scaled expert outputs, fp32
     int32_t* tile_counters;  // [kTileCounters] GEMM tile schedulers, zeroed by the row gather
+    int32_t* chunk_base;     // [E * ceil(T*k / kChunkA)] first row of each (expert, chunk)
     size_t bytes;
 };
 
@@ -40,6 +43,18 @@ cudaError_t launch_router_topk(const void* x, const void* Wg, int T, int d, int 
                                bool bf16, int32_t* idx, float* w, cudaStream_t s);
 cudaError_t launch_permute(const int32_t* idx, int n, int E, int32_t* offsets, int32_t* perm,
                            int32_t* inv, cudaStream_t s);
+// The layer's permutation in two launches: count_scan (one block: per-chunk
+// expert counts, their scan into chunk_base and offsets), then scatter (one
+// block per chunk: ranks, writes perm / inv and, if x_perm is not null,
+// copies the x rows).  Same results as launch_permute followed by
+// launch_gather_rows_bf16, whose work it replaces, including the zeroing of
+// tile_counters (may be null).  Only when chunked_permute_fits(n, E).
+bool chunked_permute_fits(int n, int E);
+cudaError_t launch_chunk_count_scan(const int32_t* idx, int n, int E, int32_t* chunk_base, int32_t* offsets,
+                                    cudaStream_t s);
+cudaError_t launch_chunk_scatter(const int32_t* idx, int n, int E, int k, const int32_t* chunk_base,
+                                 int32_t* perm, int32_t* inv, const __nv_bfloat16* x, int d,
+                                 __nv_bfloat16* x_perm, int32_t* tile_counters, cudaStream_t s);
 // Also zeroes tile_counters[0 .. kTileCounters) for the GEMMs that follow on
 // the same stream.
 cudaError_t launch_gather_rows_bf16(const __nv_bfloat16* x, const int32_t* perm, int rows, int d,

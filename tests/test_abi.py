@@ -47,9 +47,10 @@ def _sz(T, d, f, E, k, dt):
     n = T * k
     a = lambda b: (b + 255) // 256 * 256  # noqa: E731
     esz = 2 if dt == moe.MOE_BF16 else 4
-    # idx, w, perm, inv; offsets; x_perm (bf16); h; obuf; 4 GEMM tile counters
+    # idx, w, perm, inv; offsets; x_perm (bf16); h; obuf; 4 GEMM tile counters; chunk bases of the
+    # permutation (E per 64 assignments)
     return (a(4 * n) * 4 + a(4 * (E + 1)) + (a(n * d * 2) if dt == moe.MOE_BF16 else 0)
-            + a(n * f * esz) + a(n * d * 4) + a(4 * 4))
+            + a(n * f * esz) + a(n * d * 4) + a(4 * 4) + a(4 * E * ((n + 63) // 64)))
 
 
 @pytest.mark.parametrize("shape", [(4096, 4096, 14336, 8, 2), (32, 4096, 14336, 8, 2), (16, 64, 128, 8, 2),

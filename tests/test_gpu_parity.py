@@ -149,6 +149,48 @@ def test_routing_stats_of_the_synthetic_router():
     assert abs(st[9] / n - 13 / 28) < 4 * math.sqrt(13 / 28 * 15 / 28 / n)
 
 
+# ---------------------------------------------------------------- the layer's own permutation
+
+def workspace_routing_views(ws, T, E, k):
+    """offsets, perm, inv as the layer leaves them in its workspace (the
+    carve order of the C library: topk_idx, topk_w, offsets, perm, inv, each
+    at a 256-byte boundary)."""
+    n = T * k
+    a = lambda b: (b + 255) // 256 * 256  # noqa: E731
+    o_off = 2 * a(4 * n)
+    p_off = o_off + a(4 * (E + 1))
+    i_off = p_off + a(4 * n)
+    as_i32 = lambda off, cnt: ws[off: off + 4 * cnt].view(torch.int32)  # noqa: E731
+    return as_i32(o_off, E + 1), as_i32(p_off, n), as_i32(i_off, n)
+
+
+@pytest.mark.parametrize("shape", [
+    synth.MoEShape("perm-decode", 32, 256, 256, 8, 2, "bf16"),      # one-block permutation (few assignments)
+    synth.MoEShape("perm-ragged", 1100, 128, 128, 8, 2, "bf16"),     # 2200 assignments: ragged last chunk
+    synth.MoEShape("perm-4100", 4100, 128, 128, 8, 2, "bf16"),
+    synth.MoEShape("perm-E64k8", 300, 128, 128, 64, 8, "bf16"),
+    synth.MoEShape("perm-f32", 1200, 64, 128, 8, 2, "f32"),
+    synth.MoEShape("perm-fallback", 50000, 64, 64, 64, 1, "bf16"),  # E x chunks above the scan's shared memory
+], ids=lambda s: s.name)
+def test_layer_permutation_matches_the_stable_sort(shape):
+    """The permutation the layer builds for itself (chunked count/scan +
+    scatter, or the one-block kernel when E x chunks is too large) equals
+    the oracle's stable counting sort of the router's choices, bit for bit,
+    and the layer's output on sampled tokens matches the oracle."""
+    t = device_inputs(shape, 31)
+    ws = torch.empty(moe.moe_workspace_size(shape.T, shape.d, shape.f, shape.E, shape.k,
+                                            0 if shape.dtype == "bf16" else 1), dtype=torch.uint8, device="cuda")
+    y = moe.moe_layer_forward_ex(t["x"], t["Wg"], t["W1"], t["W3"], t["W2"], shape.k, workspace=ws)
+    idx, _ = moe.moe_router_topk(t["x"], t["Wg"], shape.k)
+    off, perm, inv = workspace_routing_views(ws, shape.T, shape.E, shape.k)
+    torch.cuda.synchronize()
+    check_permutation(off.cpu().numpy(), perm.cpu().numpy(), inv.cpu().numpy(), idx.cpu().numpy(), shape.E)
+    h = host_copy(t)
+    toks = np.random.default_rng(1).choice(shape.T, size=min(shape.T, 64), replace=False)
+    y_ref, _, _ = oracle_rows(h, shape.k, np.sort(toks), routing=None)
+    assert_close(to64(y)[np.sort(toks)], y_ref, shape.dtype)
+
+
 # ---------------------------------------------------------------- whole layer, every token
 
 F32_SHAPES = [
