@@ -235,6 +235,13 @@ int moe_profile_enable(int on);
 int moe_profile_read(double* total_ms, int* launches, int n);
 const char* moe_profile_stage_name(int stage);
 
+/* Restricts the recording to the stages whose bit (1 << stage) is set in
+ * stage_mask (initially all).  The events between two kernels order them
+ * fully, so every recorded stage also removes the overlap of that kernel's
+ * launch with its predecessor's tail; measure the layer's time with as few
+ * stages recorded as needed. */
+int moe_profile_select(unsigned int stage_mask);
+
 /* Text of the last error returned on this host thread ("" if none). */
 const char* moe_last_error_string(void);
 

@@ -37,6 +37,7 @@ _SIGS = {
     "moe_profile_enable": ([_I], _I),
     "moe_profile_read": ([_P, _P, _I], _I),
     "moe_profile_stage_name": ([_I], ctypes.c_char_p),
+    "moe_profile_select": ([ctypes.c_uint], _I),
     "moe_last_error_string": ([], ctypes.c_char_p),
     "moe_version": ([], ctypes.c_char_p),
 }
@@ -115,6 +116,17 @@ def moe_profile_read() -> dict:
 
 def moe_profile_stage_name(i: int) -> str:
     return lib.moe_profile_stage_name(i).decode()
+
+
+def moe_profile_select(stages=None):
+    """Record only the named stages (None: all)."""
+    mask = 0xFFFFFFFF
+    if stages is not None:
+        names = [moe_profile_stage_name(i) for i in range(MOE_PROFILE_STAGES)]
+        mask = 0
+        for st in stages:
+            mask |= 1 << names.index(st)
+    _check(lib.moe_profile_select(mask), "moe_profile_select")
 
 
 def moe_workspace_size(T, d, f, E, k, dtype=MOE_BF16) -> int:

@@ -465,12 +465,6 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
         *abort_flag = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
-    if (threadIdx.x < p.E) {
-        const int o0 = p.offsets[threadIdx.x], o1 = p.offsets[threadIdx.x + 1];
-        const int split = o0 + ((o1 - o0) / 256) * 256;  // end of the whole 256-row blocks
-        s_beg[threadIdx.x] = (p.row_mode == kPairRemainders) ? split : o0;
-        s_end[threadIdx.x] = (p.row_mode == kFullPairBlocks) ? split : o1;
-    }
     if (warp == 1) {
         if constexpr (CG == 1) {
             asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_slot)),
@@ -481,6 +475,16 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
                          "r"(TMEM_COLS) : "memory");
             asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
         }
+    }
+    // the set-up above overlaps the previous kernel's tail; offsets, the A
+    // rows and the tile counter are earlier kernels' outputs
+    pdl_wait();
+    pdl_trigger();
+    if (threadIdx.x < p.E) {
+        const int o0 = p.offsets[threadIdx.x], o1 = p.offsets[threadIdx.x + 1];
+        const int split = o0 + ((o1 - o0) / 256) * 256;  // end of the whole 256-row blocks
+        s_beg[threadIdx.x] = (p.row_mode == kPairRemainders) ? split : o0;
+        s_end[threadIdx.x] = (p.row_mode == kFullPairBlocks) ? split : o1;
     }
     tc_fence_before();
     if constexpr (CG == 2) cluster_sync_all(); else __syncthreads();
@@ -887,7 +891,7 @@ cudaError_t launch_gemm(const GroupedGemmArgs& a, const CUtensorMap& mA, const C
     cudaGetDevice(&dev);
     int units = (dev < 64) ? units_cache[dev] : 0;
     cudaLaunchConfig_t cfg = {};
-    cudaLaunchAttribute attr[1];
+    cudaLaunchAttribute attr[2];
     cfg.blockDim = dim3(NUM_THREADS);
     cfg.dynamicSmemBytes = C::kSmem;
     cfg.stream = s;
@@ -919,6 +923,7 @@ cudaError_t launch_gemm(const GroupedGemmArgs& a, const CUtensorMap& mA, const C
     const int grid_units = (int)(ub < units ? ub : units);
     if (grid_units <= 0) return cudaSuccess;
     cfg.gridDim = dim3(grid_units * CG);
+    set_pdl(attr[cfg.numAttrs++]);  // after the occupancy query, which takes the cluster attribute only
     return cudaLaunchKernelEx(&cfg, grouped_gemm_kernel<MODE, CG, BN, RB, NH>, mA, mAs, mB0, mB1, mOut, p);
 }
 

@@ -116,6 +116,7 @@ constexpr int kMaxProfiled = 8192;
 struct Prof {
     std::mutex mu;
     bool on = false;
+    unsigned mask = ~0u;            // stages that record events (bit = stage)
     int device = -1;
     std::vector<cudaEvent_t> pool;  // 2 per launch
     std::vector<int> stage;
@@ -130,7 +131,7 @@ struct StageTimer {
         std::lock_guard<std::mutex> lock(g_prof.mu);
         int dev = -1;
         cudaGetDevice(&dev);
-        if (!g_prof.on || dev != g_prof.device || g_prof.used >= kMaxProfiled) return;
+        if (!g_prof.on || dev != g_prof.device || g_prof.used >= kMaxProfiled || !((g_prof.mask >> st) & 1u)) return;
         slot = g_prof.used++;
         g_prof.stage[slot] = st;
         cudaEventRecord(g_prof.pool[2 * slot], s);
@@ -662,6 +663,13 @@ int moe_profile_read(double* total_ms, int* launches, int n) {
         if (launches) launches[i] = cnt[i];
     }
     return kNumStages;
+}
+
+int moe_profile_select(unsigned int stage_mask) {
+    g_last_error.clear();
+    std::lock_guard<std::mutex> lock(g_prof.mu);
+    g_prof.mask = stage_mask;
+    return MOE_OK;
 }
 
 const char* moe_profile_stage_name(int stage) {

@@ -12,6 +12,20 @@ namespace moe {
 unsigned int* device_error_word();                 // nullptr if the lookup fails
 cudaError_t read_clear_device_errors(unsigned int* out);
 
+// Programmatic dependent launch.  The layer's kernels are launched with
+// programmatic stream serialisation, so a kernel may start (launch, set up)
+// while its predecessor on the stream finishes; each one calls pdl_wait()
+// before it reads anything an earlier kernel wrote (the wait returns once
+// the predecessor grid has completed and its writes are visible; it returns
+// at once for a kernel launched without the attribute) and pdl_trigger()
+// to let its own successor launch early.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+inline void set_pdl(cudaLaunchAttribute& a) {
+    a.id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    a.val.programmaticStreamSerializationAllowed = 1;
+}
+
 // Sets the text moe_last_error_string() returns on this host thread.
 void set_last_error(const char* msg);
 

@@ -33,6 +33,8 @@ constexpr int kPermThreads = 1024;
 __global__ void __launch_bounds__(kPermThreads)
 permute_kernel(const int32_t* __restrict__ idx, int n, int E, int32_t* __restrict__ offsets,
                int32_t* __restrict__ perm, int32_t* __restrict__ inv) {
+    pdl_wait();
+    pdl_trigger();
     __shared__ int s_cnt[kMaxExperts];
     __shared__ int s_base[kMaxExperts];
     __shared__ int s_tile[kMaxExperts];
@@ -118,6 +120,8 @@ chunk_count_scan_kernel(const int32_t* __restrict__ idx, int n, int E, int nch, 
     extern __shared__ int s_cnt[];  // [E * nch], expert-major
     __shared__ int s_wsum[32];
     __shared__ int s_carry;
+    pdl_wait();
+    pdl_trigger();
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int m = E * nch;
     for (int i = tid; i < m; i += kScanThreads) s_cnt[i] = 0;
@@ -201,6 +205,8 @@ chunk_scatter_kernel(const int32_t* __restrict__ idx, int n, int E, int nch, int
     __shared__ int s_tok[kChunkA];
     const int c = blockIdx.x / parts, part = blockIdx.x - c * parts;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    pdl_wait();
+    pdl_trigger();
     if (blockIdx.x == 0 && tile_counters && tid < kTileCounters) tile_counters[tid] = 0;
     for (int i = tid; i < kRankWarps * kMaxExperts; i += kScatThreads) (&s_wcnt[0][0])[i] = 0;
     __syncthreads();
@@ -265,6 +271,8 @@ chunk_scatter_kernel(const int32_t* __restrict__ idx, int n, int E, int nch, int
 __global__ void __launch_bounds__(kFlatThreads)
 gather_rows_kernel(const __nv_bfloat16* __restrict__ x, const int32_t* __restrict__ perm, int rows,
                    int d, int k, __nv_bfloat16* __restrict__ xp, int32_t* __restrict__ tile_counters) {
+    pdl_wait();
+    pdl_trigger();
     if (blockIdx.x == 0 && threadIdx.x < kTileCounters) tile_counters[threadIdx.x] = 0;
     const int nvec = d / 8;
     for (int r = blockIdx.x; r < rows; r += gridDim.x) {
@@ -324,6 +332,8 @@ template <bool BF16>
 __global__ void __launch_bounds__(kFlatThreads)
 combine_kernel(const float* __restrict__ obuf, const int32_t* __restrict__ inv,
                const void* __restrict__ residual, int T, int d, int k, void* __restrict__ y) {
+    pdl_wait();
+    pdl_trigger();
     const int nvec = d / 4;
     const unsigned n = (unsigned)(T * k);
     for (int t = blockIdx.x; t < T; t += gridDim.x) {
@@ -357,6 +367,21 @@ combine_kernel(const float* __restrict__ obuf, const int32_t* __restrict__ inv,
             }
         }
     }
+}
+
+// Launch with programmatic stream serialisation (see pdl_wait / pdl_trigger).
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kernel)(KArgs...), int grid, int block, size_t smem, cudaStream_t s, Args... args) {
+    cudaLaunchConfig_t cfg = {};
+    cudaLaunchAttribute attr[1];
+    set_pdl(attr[0]);
+    cfg.gridDim = dim3(grid);
+    cfg.blockDim = dim3(block);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kernel, static_cast<KArgs>(args)...);
 }
 
 // Grid for a row kernel over `items` rows: one block per row, capped at 8
@@ -398,8 +423,7 @@ cudaError_t read_clear_device_errors(unsigned int* out) {
 
 cudaError_t launch_permute(const int32_t* idx, int n, int E, int32_t* offsets, int32_t* perm,
                            int32_t* inv, cudaStream_t s) {
-    permute_kernel<<<1, kPermThreads, 0, s>>>(idx, n, E, offsets, perm, inv);
-    return cudaGetLastError();
+    return launch_pdl(permute_kernel, 1, kPermThreads, 0, s, idx, n, E, offsets, perm, inv);
 }
 
 // Below 2048 assignments the one-block permutation and the row gather are
@@ -423,9 +447,8 @@ cudaError_t launch_chunk_count_scan(const int32_t* idx, int n, int E, int32_t* c
         attr_done[dev] = true;
     }
     const int nch = (n + kChunkA - 1) / kChunkA;
-    chunk_count_scan_kernel<<<1, kScanThreads, (size_t)E * nch * sizeof(int), s>>>(idx, n, E, nch, chunk_base,
-                                                                                    offsets);
-    return cudaGetLastError();
+    return launch_pdl(chunk_count_scan_kernel, 1, kScanThreads, (size_t)E * nch * sizeof(int), s, idx, n, E, nch,
+                      chunk_base, offsets);
 }
 
 cudaError_t launch_chunk_scatter(const int32_t* idx, int n, int E, int k, const int32_t* chunk_base,
@@ -437,24 +460,20 @@ cudaError_t launch_chunk_scatter(const int32_t* idx, int n, int E, int k, const 
     int parts = (want + nch - 1) / nch;
     parts = parts < 1 ? 1 : (parts > 8 ? 8 : parts);
     if (!x_perm) parts = 1;
-    chunk_scatter_kernel<<<nch * parts, kScatThreads, 0, s>>>(idx, n, E, nch, k, parts, chunk_base, perm, inv, x, d,
-                                                               x_perm, tile_counters);
-    return cudaGetLastError();
+    return launch_pdl(chunk_scatter_kernel, nch * parts, kScatThreads, 0, s, idx, n, E, nch, k, parts, chunk_base,
+                      perm, inv, x, d, x_perm, tile_counters);
 }
 
 cudaError_t launch_gather_rows_bf16(const __nv_bfloat16* x, const int32_t* perm, int rows, int d,
                                     int k, __nv_bfloat16* x_perm, int32_t* tile_counters, cudaStream_t s) {
-    gather_rows_kernel<<<flat_grid(rows), kFlatThreads, 0, s>>>(x, perm, rows, d, k, x_perm, tile_counters);
-    return cudaGetLastError();
+    return launch_pdl(gather_rows_kernel, flat_grid(rows), kFlatThreads, 0, s, x, perm, rows, d, k, x_perm,
+                      tile_counters);
 }
 
 cudaError_t launch_combine(const float* obuf, const int32_t* inv, const void* residual, int T,
                            int d, int k, bool bf16, void* y, cudaStream_t s) {
-    if (bf16)
-        combine_kernel<true><<<flat_grid(T), kFlatThreads, 0, s>>>(obuf, inv, residual, T, d, k, y);
-    else
-        combine_kernel<false><<<flat_grid(T), kFlatThreads, 0, s>>>(obuf, inv, residual, T, d, k, y);
-    return cudaGetLastError();
+    if (bf16) return launch_pdl(combine_kernel<true>, flat_grid(T), kFlatThreads, 0, s, obuf, inv, residual, T, d, k, y);
+    return launch_pdl(combine_kernel<false>, flat_grid(T), kFlatThreads, 0, s, obuf, inv, residual, T, d, k, y);
 }
 
 }  // namespace moe

@@ -108,6 +108,8 @@ __global__ void __launch_bounds__(kWarps * 32, BF16 ? 4 : 2)  // bf16: 64 regist
 router_topk_kernel(const void* __restrict__ x, const void* __restrict__ Wg, int T, int d, int E, int k,
                    int32_t* __restrict__ idx_out, float* __restrict__ w_out) {
     extern __shared__ __align__(16) unsigned char smem_raw[];
+    pdl_wait();     // x may be the previous kernel's output (a layer stack)
+    pdl_trigger();
     double* wfrag = reinterpret_cast<double*>(smem_raw);  // [kChunks][8][32]
     double* part = wfrag + kFragDoubles;                  // [kTokBlock][E]
     cg::cluster_group cluster = cg::this_cluster();
@@ -242,17 +244,18 @@ cudaError_t launch_impl(const void* x, const void* Wg, int T, int d, int E, int 
     }
     const int blocks = (T + kTokBlock - 1) / kTokBlock;
     cudaLaunchConfig_t cfg = {};
-    cudaLaunchAttribute attr[1];
+    cudaLaunchAttribute attr[2];
     attr[0].id = cudaLaunchAttributeClusterDimension;
     attr[0].val.clusterDim.x = kCluster;
     attr[0].val.clusterDim.y = 1;
     attr[0].val.clusterDim.z = 1;
+    set_pdl(attr[1]);
     cfg.gridDim = dim3(kCluster * blocks);
     cfg.blockDim = dim3(kWarps * 32);
     cfg.dynamicSmemBytes = router_smem_bytes(E);
     cfg.stream = s;
     cfg.attrs = attr;
-    cfg.numAttrs = 1;
+    cfg.numAttrs = 2;
     return cudaLaunchKernelEx(&cfg, router_topk_kernel<BF16>, x, Wg, T, d, E, k, idx, w);
 }
 
