@@ -210,7 +210,7 @@ def moe_layer_forward(x, Wg, W1, W3, W2, k, y=None, stream=None):
     return y
 
 
-def moe_layer_forward_host(x, Wg, W1, W3, W2, k, y=None, chunks=2, x_ready=False, y_async=False, stream=None):
+def moe_layer_forward_host(x, Wg, W1, W3, W2, k, y=None, chunks=1, x_ready=False, y_async=False, stream=None):
     """The bf16 layer on host x / y (CPU tensors; page-locked for overlap),
     pipelined in `chunks` pieces; returns y (a pinned CPU tensor unless given).
     x_ready=True passes MOE_HOST_X_READY (x's copies may start before work
