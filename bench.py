@@ -469,10 +469,8 @@ def gemm_vs_cublas(args, device):
                                 "down_ms": round(dng, 4), "down": tf(2.0 * M * d * f, dng)}
     del xs, hs, W13e
 
-    def ours(shape, tt, key, env=None):
-        old = os.environ.get("MOE_GEMM_CTA_GROUP")
-        if env is not None:
-            os.environ["MOE_GEMM_CTA_GROUP"] = env
+    def ours(shape, tt, key, cta_group=0):
+        moe.moe_set_gemm_variant(cta_group)
         try:
             y = torch.empty_like(tt["x"])
             ws = torch.empty(moe.moe_workspace_size(shape.T, d, f, shape.E, shape.k, 0), dtype=torch.uint8,
@@ -489,19 +487,15 @@ def gemm_vs_cublas(args, device):
             p = moe.moe_profile_read()
             moe.moe_profile_enable(False)
         finally:
-            if env is not None:
-                if old is None:
-                    os.environ.pop("MOE_GEMM_CTA_GROUP", None)
-                else:
-                    os.environ["MOE_GEMM_CTA_GROUP"] = old
-        u, w = p["up_swiglu_gemm"][0] / 20, p["down_scaled_gemm"][0] / 20
+            moe.moe_set_gemm_variant()
+        u, w = p["up_swiglu_gemm"][0] / 20, p["down_combine_gemm"][0] / 20
         out[key] = {"up_ms": round(u, 4), "up": tf(4.0 * M * d * f, u), "down_ms": round(w, 4),
                     "down": tf(2.0 * M * d * f, w)}
 
     one = synth.MoEShape("one-expert", M, d, f, 1, 1, "bf16")
     t1 = device_inputs(one, 0, device=device)
-    for cg in ("1", "2"):
-        ours(one, t1, "ours_one_expert_cta_group_%s" % cg, env=cg)
+    for cg in (1, 2):
+        ours(one, t1, "ours_one_expert_cta_group_%d" % cg, cta_group=cg)
     del t1
     ours(s, t, "ours_grouped_prefill")
     print(json.dumps(out))
@@ -606,7 +600,7 @@ def main():
         counts = None
         wbytes = 3.0 * d.E * d.d * d.f * 2  # all 8 experts are touched at T=32 with near-uniform routing
         ups, upn = rd["prof_up"]["up_swiglu_gemm"]
-        dns, dnn = p["down_scaled_gemm"]
+        dns, dnn = p["down_combine_gemm"]
         gms = graph_step_ms(rd, d, device, dargs.steps)
         line["decode"] = {"workload": workload_desc(d, world)["workload"], "ms_per_step": dms,
                           "ms_per_step_cuda_graph": gms,

@@ -39,8 +39,12 @@
  *    are those of the exact logits except within ~1e-13 relative near-ties.
  *  - Thread safety: calls on different streams may run concurrently when
  *    each uses its own workspace (moe_layer_forward_ex); moe_layer_forward
- *    and moe_layer_forward_host share one library-owned workspace per device
- *    and must not be called concurrently on two streams of one device.
+ *    and moe_layer_forward_host share one library-owned workspace per device,
+ *    so their calls on one device must not overlap on the GPU (use one
+ *    stream, or order the streams with events).
+ *  - cudaDeviceReset() discards the library's per-device state (the cached
+ *    workspace, copy streams and symbol addresses); do not call the library
+ *    on a device after resetting it in the same process.
  */
 #ifndef MOE_B200_H
 #define MOE_B200_H
@@ -81,8 +85,10 @@ enum {
 /* Bytes of device workspace needed by moe_layer_forward_ex and moe_expert_ffn
  * for this shape (0 for invalid arguments).  Holds the routing result, the
  * permutation, the expert-ordered copy of x, the hidden activations h
- * [T*k, f], the gate-scaled expert outputs [T*k, d] (fp32) and the expert
- * GEMMs' tile counters.  No contents need to survive between calls. */
+ * [T*k, f], the gate-scaled expert outputs [T*k, d] (fp32), the expert
+ * GEMMs' tile counters and the combine's arrival counters (one per token
+ * and 128 output columns).  No contents need to survive between calls: the
+ * calls clear the counters themselves. */
 size_t moe_workspace_size(int T, int d, int f, int E, int k, int dtype);
 
 /* Router and top-k gate ("Mixtral of Experts" §2.1 display 2; Method, steps
@@ -120,8 +126,12 @@ int moe_routing_stats(const int32_t* topk_idx, int T, int E, int k, int seq_len,
  * step 4; SwiGLU expert).  For every permuted row r of expert e with
  * assignment q = perm[r] = t*k + j:  h_r = SiLU(W1_e x_t) * (W3_e x_t)
  * (rounded to bf16 on the bf16 path), o_r = topk_w[q] * (W2_e h_r) in fp32,
- * and y[t] = sum_j o_{inv[t*k+j]} in slot order, rounded once to y's dtype.
- * offsets/perm/inv/topk_w are as produced by moe_permute / moe_router_topk.
+ * and y[t] = sum_j o_{inv[t*k+j]} in slot order, rounded once to y's dtype
+ * (slots whose inv entry is out of range add nothing).  On the bf16 path the
+ * gate weighting and this sum run in the down-projection GEMM's epilogue.
+ * offsets/perm/inv/topk_w are as produced by moe_permute / moe_router_topk:
+ * perm and inv must be inverse permutations over the routed assignments
+ * (otherwise y is unspecified, though every access stays in bounds).
  * workspace: device memory of at least moe_workspace_size() bytes. */
 int moe_expert_ffn(const void* x, const void* W1, const void* W3, const void* W2,
                    const int32_t* offsets, const int32_t* perm, const int32_t* inv,
@@ -131,7 +141,11 @@ int moe_expert_ffn(const void* x, const void* W1, const void* W3, const void* W2
 /* The whole layer in bf16: router, permutation, experts, combine.  The
  * workspace comes from a library-owned, stream-ordered allocation per device
  * (grown with cudaMallocAsync on `stream` when a larger shape arrives and
- * kept until moe_release_workspace()). */
+ * kept until moe_release_workspace()).  Calls on one device share that
+ * workspace: serialise them (one stream, or events between streams); callers
+ * that run layers concurrently give each stream its own workspace through
+ * moe_layer_forward_ex.  Growing the workspace frees the old one only after
+ * the work already enqueued with it (on any stream) has finished. */
 int moe_layer_forward(const void* x, const void* Wg, const void* W1, const void* W3,
                       const void* W2, int T, int d, int f, int E, int k, void* y,
                       moe_stream_t stream);
@@ -180,8 +194,8 @@ int moe_layer_forward_ex(const void* x, const void* Wg, const void* W1, const vo
 
 /* A stack of L layers with the residual stream between them (Method, step 5;
  * tab. 1: 32 layers): x_{l+1} = x_l + MoE_l(x_l) for l = 0 .. L-1, y = x_L.
- * The residual is added in the combine kernel of each layer (no extra
- * pass).  Wg, W1, W3, W2 are HOST arrays of L device pointers (layer l's
+ * The residual is added in each layer's combine (the down-projection
+ * GEMM's epilogue on the bf16 path; no extra pass).  Wg, W1, W3, W2 are HOST arrays of L device pointers (layer l's
  * weights, layouts as above).  scratch: a caller [T, d] device buffer of the
  * activation dtype (the layers ping-pong between y and scratch; unused when
  * L = 1); x is left untouched; x, y and scratch must be distinct.
@@ -200,7 +214,7 @@ int moe_stack_forward(const void* x, const void* const* Wg, const void* const* W
  * counterpart in the paper: it is a deployment convenience of this library.
  * Instead of allocating, it uses a 32 MiB scratch array compiled into the
  * library (kept by every GPU that loads it until the process exits), which
- * covers T*k*(2d + 2f + 4d) bytes plus routing buffers: up to 314 tokens at
+ * covers T*k*(2d + 2f + 4d) bytes plus routing buffers and counters: up to 314 tokens at
  * the Mixtral-8x7B dimensions.  Larger shapes return MOE_ERR_WORKSPACE with a
  * message naming the bytes needed.  The first call on each device looks up
  * the array's device address (cudaGetSymbolAddress) with that device
@@ -213,7 +227,7 @@ int moe_layer_forward_noalloc(const void* x, const void* Wg, const void* W1, con
 
 /* Frees the workspace moe_layer_forward keeps for the current device and
  * the staging of moe_layer_forward_host (stream-ordered on `stream`, after
- * the copies that use it). */
+ * the work and the copies that used them). */
 int moe_release_workspace(moe_stream_t stream);
 
 /* Synchronises the current device, returns the device-side flags
@@ -224,8 +238,8 @@ unsigned int moe_device_errors(void);
  * library launches on the current device is bracketed by a pair of CUDA
  * events recorded on the launching stream (no synchronisation is added).
  * Stages: 0 router_topk, 1 permute, 2 gather, 3 up-projection GEMM (SwiGLU
- * epilogue), 4 down-projection GEMM (gate scaling), 5 combine, 6 fp32 expert
- * kernels.  moe_profile_enable(1) clears and starts recording (up to 8192
+ * epilogue), 4 down-projection GEMM (gate scaling and, on the bf16 path, the
+ * combine), 5 combine (fp32 path), 6 fp32 expert kernels.  moe_profile_enable(1) clears and starts recording (up to 8192
  * launches), moe_profile_enable(0) stops.  moe_profile_read() waits for the
  * recorded events, writes per-stage total milliseconds and launch counts
  * for the first n stages, clears the record, and returns the number of
@@ -241,6 +255,30 @@ const char* moe_profile_stage_name(int stage);
  * launch with its predecessor's tail; measure the layer's time with as few
  * stages recorded as needed. */
 int moe_profile_select(unsigned int stage_mask);
+
+/* Test and measurement hooks.  Process-wide settings, read by every GEMM
+ * launch that follows on any thread; never needed in normal use.
+ *
+ * moe_set_gemm_variant forces the expert GEMMs' tile variant (every variant
+ * computes the same result; the automatic choice is the measured fastest):
+ *   cta_group   0 automatic, 1 single-CTA tiles, 2 CTA-pair tiles, 3 pairs on
+ *               each expert's whole 256-row blocks then single CTAs on the rest
+ *   up_bn       0 automatic, 128 or 256: width of single-CTA up-projection tiles
+ *   token_rows  0 automatic, 32 or 128: token rows of single-CTA tiles
+ *   pair_cols   0 automatic, 256 or 512: columns of CTA-pair tiles
+ * Any other value: MOE_ERR_INVALID_ARG, nothing changed.
+ *
+ * moe_set_wait_test serves failure-detection tests.  Every wait of the GEMM
+ * pipelines (a stage, an accumulator, a tile number) gives up after
+ * wait_limit_ns of waiting (0 restores the default, 4 s): the kernel then
+ * raises MOE_DEVERR_PIPELINE_TIMEOUT, stops the other roles of its CTA (and
+ * of its CTA pair), lets the work it already issued finish, frees its tensor
+ * memory and returns, leaving its outputs incomplete.  With stall_epilogue
+ * != 0 the epilogue of every GEMM waits on a barrier that nothing completes,
+ * so that this path runs; the context stays usable, and the next calls with
+ * stall_epilogue = 0 compute normally. */
+int moe_set_gemm_variant(int cta_group, int up_bn, int token_rows, int pair_cols);
+int moe_set_wait_test(unsigned long long wait_limit_ns, int stall_epilogue);
 
 /* Text of the last error returned on this host thread ("" if none). */
 const char* moe_last_error_string(void);

@@ -13,4 +13,5 @@ from .binding import (  # noqa: F401
     moe_release_workspace,
     moe_device_errors, moe_last_error_string, moe_version,
     moe_profile_enable, moe_profile_read, moe_profile_stage_name, moe_profile_select,
+    moe_set_gemm_variant, moe_set_wait_test,
 )

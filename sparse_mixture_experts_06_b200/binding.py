@@ -38,6 +38,8 @@ _SIGS = {
     "moe_profile_read": ([_P, _P, _I], _I),
     "moe_profile_stage_name": ([_I], ctypes.c_char_p),
     "moe_profile_select": ([ctypes.c_uint], _I),
+    "moe_set_gemm_variant": ([_I, _I, _I, _I], _I),
+    "moe_set_wait_test": ([ctypes.c_ulonglong, _I], _I),
     "moe_last_error_string": ([], ctypes.c_char_p),
     "moe_version": ([], ctypes.c_char_p),
 }
@@ -127,6 +129,17 @@ def moe_profile_select(stages=None):
         for st in stages:
             mask |= 1 << names.index(st)
     _check(lib.moe_profile_select(mask), "moe_profile_select")
+
+
+def moe_set_gemm_variant(cta_group=0, up_bn=0, token_rows=0, pair_cols=0):
+    """Force the expert GEMMs' tile variant (0 = automatic); test and measurement hook."""
+    _check(lib.moe_set_gemm_variant(cta_group, up_bn, token_rows, pair_cols), "moe_set_gemm_variant")
+
+
+def moe_set_wait_test(wait_limit_ns=0, stall_epilogue=False):
+    """Bound of the GEMM pipeline waits (0 = default 4 s) and the epilogue stall
+    of the failure-detection test."""
+    _check(lib.moe_set_wait_test(int(wait_limit_ns), 1 if stall_epilogue else 0), "moe_set_wait_test")
 
 
 def moe_workspace_size(T, d, f, E, k, dtype=MOE_BF16) -> int:

@@ -56,6 +56,7 @@
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
+#include <atomic>
 #include <cstdlib>
 #include <mutex>
 
@@ -71,7 +72,9 @@ constexpr int A_TILE = BM * BK * 2;            // 16 KiB: 128 rows x 64 k
 constexpr int kEpiWarps = 8;                  // two per TMEM lane quadrant
 constexpr int NUM_THREADS = 64 + 32 * kEpiWarps;
 constexpr int TMEM_COLS = 512;                 // 2 accumulators x 256 fp32 columns
-constexpr unsigned long long kTimeoutNs = 4000000000ull;
+constexpr unsigned long long kWaitLimitNs = 4000000000ull;  // default bound of a pipeline wait
+constexpr unsigned long long kDrainLimitNs = 1000000000ull;  // bound of the exit drain of issued MMAs
+constexpr unsigned long long kQuiesceNs = 100000ull;         // after an abort: copies in flight land
 
 
 enum Mode { kUp = 0, kDown = 1 };
@@ -85,12 +88,19 @@ struct KParams {
     int b_rows_per_expert;   // f (up) or d (down): expert stride in the 2-D weight view
     __nv_bfloat16* h;        // up output [rows, f]
     const int32_t* perm;     // down: assignment of each permuted row
+    const int32_t* inv;      // down: permuted row of each assignment [T*k]
     const float* topk_w;     // down: gate weights [T*k]
-    float* obuf;             // down output [rows, d]
+    float* obuf;             // down: parked gate-scaled rows [rows, d] (fp32)
+    unsigned int* arrivals;  // down: [T, ceil(d / 128)] slot arrival counters, zero at launch
+    __nv_bfloat16* y;        // down: layer output [T, d]
+    const __nv_bfloat16* residual;  // down: added to y after the slot sum, or null
+    int k;                   // experts per token
     int rows;                // T*k
     unsigned int* err;       // device error word (MOE_DEVERR_*)
     int row_mode;            // rows of each expert to cover: kAllRows, kFullPairBlocks or kPairRemainders
     int* tile_counter;       // next tile to hand out; zero at launch (the row gather zeroes it)
+    unsigned long long wait_limit_ns;  // bound of every pipeline wait
+    int stall_test;          // failure-detection test: the epilogue waits on a barrier nothing completes
 };
 
 // Row ranges: all rows of each expert; only its whole 256-row blocks; or
@@ -285,6 +295,12 @@ __device__ __forceinline__ void umma_commit_pair(uint32_t bar) {
         : "memory");
 }
 
+// Arrive-one on this CTA's own mbarrier when the pair MMAs this thread issued
+// complete.
+__device__ __forceinline__ void umma_commit_pair_own(uint32_t bar) {
+    asm volatile("tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar) : "memory");
+}
+
 // Bulk tensor store of a 32-row box from this CTA's shared memory (async
 // proxy); completion is tracked per thread with bulk groups.
 __device__ __forceinline__ void tma_store_2d(const CUtensorMap* map, uint32_t src, int c0, int c1) {
@@ -298,6 +314,9 @@ __device__ __forceinline__ void bulk_wait_read_all() { asm volatile("cp.async.bu
 __device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
 __device__ __forceinline__ void fence_proxy_async_smem() {
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+__device__ __forceinline__ void fence_proxy_async_global() {
+    asm volatile("fence.proxy.async.global;" ::: "memory");
 }
 __device__ __forceinline__ void st_shared_v4(uint32_t addr, uint4 v) {
     asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w)
@@ -398,7 +417,8 @@ __device__ __forceinline__ void decode_tile_rows(int tile, const int* s_beg, con
 // hundreds of cycles, which would delay the next MMA issue).
 template <bool kClusterScope = false>
 __device__ __forceinline__ bool wait_bounded_pair(uint32_t bar, uint32_t parity, volatile int* abort_flag,
-                                                  unsigned int* err, uint32_t peer_abort_addr) {
+                                                  unsigned int* err, uint32_t peer_abort_addr,
+                                                  unsigned long long limit_ns) {
     unsigned long long t0 = 0;
     for (uint32_t i = 1;; ++i) {
         if (kClusterScope ? mbar_try_wait_cluster(bar, parity) : mbar_try_wait(bar, parity)) return true;
@@ -407,7 +427,7 @@ __device__ __forceinline__ bool wait_bounded_pair(uint32_t bar, uint32_t parity,
             const unsigned long long now = globaltimer();
             if (t0 == 0) {
                 t0 = now;
-            } else if (now - t0 > kTimeoutNs) {
+            } else if (now - t0 > limit_ns) {
                 *abort_flag = 1;
                 if (peer_abort_addr) st_cluster_u32(peer_abort_addr, 1u);
                 atomicOr(err, 1u);
@@ -415,6 +435,36 @@ __device__ __forceinline__ bool wait_bounded_pair(uint32_t bar, uint32_t parity,
             }
         }
     }
+}
+
+// Exit-path wait for work this thread has already issued (the MMAs, which
+// need nothing more from any other role to complete): bounded by
+// kDrainLimitNs and blind to the abort flag; on expiry it raises the error
+// flag and gives up.
+__device__ __forceinline__ bool wait_drain(uint32_t bar, uint32_t parity, unsigned int* err) {
+    unsigned long long t0 = 0;
+    for (uint32_t i = 1;; ++i) {
+        if (mbar_try_wait(bar, parity)) return true;
+        if ((i & 1023u) == 0) {
+            const unsigned long long now = globaltimer();
+            if (t0 == 0) {
+                t0 = now;
+            } else if (now - t0 > kDrainLimitNs) {
+                atomicOr(err, 1u);
+                return false;
+            }
+        }
+    }
+}
+
+// After an abort, bulk copies a producer issued may still be landing in
+// shared memory, and some complete on barrier phases that will never finish
+// (the other CTA of the pair stopped issuing first), so they cannot be
+// waited for one by one: the producer waits kQuiesceNs, many times the
+// latency of a copy, before the CTA frees its resources.
+__device__ __forceinline__ void quiesce_copies() {
+    const unsigned long long t0 = globaltimer();
+    while (globaltimer() - t0 < kQuiesceNs) __nanosleep(1000);
 }
 
 // Tile-number ring between the producer that takes tiles from the global
@@ -428,6 +478,99 @@ template <int CG>
 struct Sched {
     static constexpr uint32_t kReaders = (CG == 1) ? 1u + kEpiWarps : 2u * (1u + kEpiWarps);
 };
+
+// ---------------------------------------------------------------------------
+// The combine, fused into the down-projection's epilogue (§2.1 display 3:
+// y[t] = sum_j w[t, j] * SwiGLU_{idx[t, j]}(x[t]); Method: the expert results
+// are scattered back to the token order).
+//
+// Every permuted row r (assignment q = perm[r] = t*k + j) first parks its
+// gate-scaled fp32 row in obuf[r] with the tile's bulk stores, and the warp
+// releases the accumulator.  Then, per group of 128 output columns, each
+// lane adds one to the counter of (its token, the group); the arrival that
+// brings the counter to the token's number of routed slots is the last one.
+// Every other slot parked its row before it counted (bulk-store completion,
+// proxy fence, release fence, atomic), so the last arrival reads the k rows
+// back, adds them in slot order j = 0, 1, ... (then the residual, if any),
+// rounds once to bf16 and stores y[t].  The sum is the same whichever tile
+// finishes last, nothing waits on another CTA, and all of it overlaps the
+// next tile's main loop.  Counters start at zero (the permutation kernels
+// clear them before the GEMMs run).
+
+__device__ __forceinline__ float4 ldcg_f4(const float* a) { return __ldcg(reinterpret_cast<const float4*>(a)); }
+
+// a = v for the first routed slot, a += v after it (slot order)
+__device__ __forceinline__ void add_slot(float4& a, const float4& v, bool& first) {
+    if (first) {
+        a = v;
+        first = false;
+    } else {
+        a.x += v.x; a.y += v.y; a.z += v.z; a.w += v.w;
+    }
+}
+
+// Rows `m` (a warp-uniform lane mask) are last arrivals of the 128-column
+// group that starts at output column c0; lane l sums columns c0 + 4l .. +3
+// of each such row's token (t, and the token's slot rows rr0 / rr1 for
+// j = 0 / 1, are held by the row's lane).  Eight rows at a time, all their
+// loads issued before the sums.
+__device__ __forceinline__ void combine_group(unsigned m, int t, int rr0, int rr1, int c0, const KParams& p,
+                                           int lane) {
+    constexpr int B = 8;
+    const int d = p.n_out;
+    const unsigned nrows = (unsigned)p.rows;
+    const int c = c0 + 4 * lane;
+    const bool colok = c < d;  // d is a multiple of 8: four columns are all in or all out
+    const float4 zero = make_float4(0.f, 0.f, 0.f, 0.f);
+    while (m) {
+        int src[B], tb[B], r0[B], r1[B];
+#pragma unroll
+        for (int b = 0; b < B; ++b) {
+            src[b] = m ? __ffs(m) - 1 : -1;
+            m = m ? (m & (m - 1)) : 0u;
+        }
+#pragma unroll
+        for (int b = 0; b < B; ++b) {
+            const int s = src[b] < 0 ? 0 : src[b];
+            tb[b] = __shfl_sync(0xffffffffu, t, s);
+            r0[b] = __shfl_sync(0xffffffffu, rr0, s);
+            r1[b] = __shfl_sync(0xffffffffu, rr1, s);
+        }
+        float4 v0[B], v1[B];
+        uint2 rs[B];
+#pragma unroll
+        for (int b = 0; b < B; ++b) {
+            const bool live = src[b] >= 0 && colok;
+            v0[b] = (live && (unsigned)r0[b] < nrows) ? ldcg_f4(p.obuf + (size_t)r0[b] * d + c) : zero;
+            v1[b] = (live && (unsigned)r1[b] < nrows) ? ldcg_f4(p.obuf + (size_t)r1[b] * d + c) : zero;
+            rs[b] = (live && p.residual)
+                        ? __ldg(reinterpret_cast<const uint2*>(p.residual + (size_t)tb[b] * d + c))
+                        : make_uint2(0u, 0u);
+        }
+#pragma unroll
+        for (int b = 0; b < B; ++b) {
+            if (src[b] < 0 || !colok) continue;
+            float4 a = zero;
+            bool first = true;
+            if ((unsigned)r0[b] < nrows) add_slot(a, v0[b], first);
+            if ((unsigned)r1[b] < nrows) add_slot(a, v1[b], first);
+            for (int j = 2; j < p.k; ++j) {  // slots beyond the first two (general top-k)
+                const int r = __ldg(p.inv + (size_t)tb[b] * p.k + j);
+                if ((unsigned)r < nrows) add_slot(a, ldcg_f4(p.obuf + (size_t)r * d + c), first);
+            }
+            if (p.residual) {
+                a.x = __uint_as_float(rs[b].x << 16) + a.x;
+                a.y = __uint_as_float(rs[b].x & 0xFFFF0000u) + a.y;
+                a.z = __uint_as_float(rs[b].y << 16) + a.z;
+                a.w = __uint_as_float(rs[b].y & 0xFFFF0000u) + a.w;
+            }
+            uint2 out;
+            out.x = pack_bf16x2(a.x, a.y);
+            out.y = pack_bf16x2(a.z, a.w);
+            *reinterpret_cast<uint2*>(p.y + (size_t)tb[b] * d + c) = out;
+        }
+    }
+}
 
 template <int MODE, int CG, int BN, int RB, int NH>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
@@ -450,8 +593,10 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
     uint64_t* tempty = bars + 2 * STG + 2;
     uint64_t* sfull = bars + 2 * STG + 4;                 // [kSchedSlots] tile number published
     uint64_t* sempty = sfull + kSchedSlots;               // [kSchedSlots] all readers done (even CTA)
-    volatile int* stile = reinterpret_cast<volatile int*>(sempty + kSchedSlots);  // [kSchedSlots]
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sempty + kSchedSlots) + kSchedSlots;
+    uint64_t* mma_done = sempty + kSchedSlots;            // the MMA issuer's exit drain
+    uint64_t* stall_bar = mma_done + 1;                   // failure-detection test: never completed
+    volatile int* stile = reinterpret_cast<volatile int*>(stall_bar + 1);  // [kSchedSlots]
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(stall_bar + 1) + kSchedSlots;
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
     int* s_beg = reinterpret_cast<int*>(tmem_slot + 2);  // [E] first row of expert e's range
     int* s_end = s_beg + kMaxExperts;                   // [E] end of expert e's range
@@ -474,6 +619,8 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
             mbar_init(smem_u32(&sfull[q]), 1);
             mbar_init(smem_u32(&sempty[q]), Sched<CG>::kReaders);
         }
+        mbar_init(smem_u32(mma_done), 1);
+        mbar_init(smem_u32(stall_bar), 1);
         *abort_flag = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
@@ -509,7 +656,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
     const uint32_t sempty_leader0 = (CG == 2) ? map_to_rank(smem_u32(&sempty[0]), 0) : smem_u32(&sempty[0]);
     auto read_tile = [&](uint32_t i, bool& ok) -> int {
         const uint32_t q = i % kSchedSlots, ph = (i / kSchedSlots) & 1u;
-        if (!wait_bounded_pair<CG == 2>(smem_u32(&sfull[q]), ph, abort_flag, p.err, peer_abort)) {
+        if (!wait_bounded_pair<CG == 2>(smem_u32(&sfull[q]), ph, abort_flag, p.err, peer_abort, p.wait_limit_ns)) {
             ok = false;
             return -1;
         }
@@ -534,7 +681,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
                 if (leader) {
                     // publish the tile taken (to both CTAs of a pair)
                     const uint32_t q = ti % kSchedSlots, ph = (ti / kSchedSlots) & 1u;
-                    if (!wait_bounded_pair<CG == 2>(smem_u32(&sempty[q]), ph ^ 1u, abort_flag, p.err, peer_abort)) {
+                    if (!wait_bounded_pair<CG == 2>(smem_u32(&sempty[q]), ph ^ 1u, abort_flag, p.err, peer_abort, p.wait_limit_ns)) {
                         ok = false;
                         break;
                     }
@@ -575,7 +722,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
                     if (leader && kb == kb_next) next = atomicAdd(p.tile_counter, 1);
                     const uint32_t s = it % STG;
                     const uint32_t ph = (it / STG) & 1u;
-                    if (!wait_bounded_pair(smem_u32(&empty[s]), ph ^ 1u, abort_flag, p.err, peer_abort)) { ok = false; break; }
+                    if (!wait_bounded_pair(smem_u32(&empty[s]), ph ^ 1u, abort_flag, p.err, peer_abort, p.wait_limit_ns)) { ok = false; break; }
                     const uint32_t fb = smem_u32(&full[s]);
                     if constexpr (CG == 1) {
                         mbar_arrive_expect_tx(fb, C::kABytes + C::kBBytes);
@@ -603,13 +750,18 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
             // issued stages (use j of a stage completes phase j / STG of its
             // empty barrier), so no arrival from the pair's commits is still
             // on its way when the CTA exits.
+            bool drained = ok;
             if (ok) {
                 const uint32_t first = it > (uint32_t)STG ? it - (uint32_t)STG : 0u;
                 for (uint32_t j = first; j < it; ++j) {
-                    if (!wait_bounded_pair(smem_u32(&empty[j % STG]), (j / STG) & 1u, abort_flag, p.err, peer_abort))
+                    if (!wait_bounded_pair(smem_u32(&empty[j % STG]), (j / STG) & 1u, abort_flag, p.err, peer_abort,
+                                           p.wait_limit_ns)) {
+                        drained = false;
                         break;
+                    }
                 }
             }
+            if (!drained) quiesce_copies();
         }
         __syncwarp();
     } else if (warp == 1) {
@@ -624,7 +776,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
                 if (tile < 0) break;
                 const uint32_t acc = tcount % C::kNAcc;
                 const uint32_t use = tcount / C::kNAcc;
-                if (!wait_bounded_pair(smem_u32(&tempty[acc]), (use & 1u) ^ 1u, abort_flag, p.err, peer_abort)) break;
+                if (!wait_bounded_pair(smem_u32(&tempty[acc]), (use & 1u) ^ 1u, abort_flag, p.err, peer_abort, p.wait_limit_ns)) break;
                 tc_fence_after();
                 const uint32_t d_tmem = tmem_base + acc * C::kTileN;
                 uint32_t idesc = C::kIdesc;
@@ -637,7 +789,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
                 for (int kb = 0; kb < kblocks; ++kb, ++it) {
                     const uint32_t s = it % STG;
                     const uint32_t ph = (it / STG) & 1u;
-                    if (!wait_bounded_pair(smem_u32(&full[s]), ph, abort_flag, p.err, peer_abort)) { ok = false; break; }
+                    if (!wait_bounded_pair(smem_u32(&full[s]), ph, abort_flag, p.err, peer_abort, p.wait_limit_ns)) { ok = false; break; }
                     tc_fence_after();
                     const uint64_t adesc = sw128_desc(smem_u32(sA + s * A_TILE));
                     const uint64_t bdesc = sw128_desc(smem_u32(sB + s * C::kBBytes));
@@ -661,19 +813,30 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
                     if constexpr (CG == 1) umma_commit(smem_u32(&tfull[acc])); else umma_commit_pair(smem_u32(&tfull[acc]));
                 }
             }
+            // Exit drain: every MMA issued here has completed before the block
+            // frees its tensor memory and its peer's shared memory goes away
+            // (after an abort some were never waited for).
+            if (it > 0) {
+                if constexpr (CG == 1) umma_commit(smem_u32(mma_done)); else umma_commit_pair_own(smem_u32(mma_done));
+                wait_drain(smem_u32(mma_done), 0u, p.err);
+            }
         }
         __syncwarp();
     } else {
         // ---------------------------------------------------- epilogue (both CTAs)
         // Two warps per TMEM lane quadrant (warp % 4 selects the lanes a warp
-        // may read); of the tile's output units (64-hidden-unit segments of
-        // the up-projection, 32-column boxes of the down-projection, over all
-        // MMA parts) warp sub = 0 takes the even ones and sub = 1 the odd ones.
+        // may read).  Up: of the tile's 64-hidden-unit segments (over all MMA
+        // parts) warp sub = 0 takes the even ones and sub = 1 the odd ones.
+        // Down: the quadrant's columns in groups of 128 (four 32-column
+        // boxes; the unit of the combine's arrival counters), sub = 0 taking
+        // the first half of the groups and sub = 1 the rest.
         const int quad = warp & 3;  // TMEM lanes 32*quad .. 32*quad+31
         const int sub = (warp - 2) >> 2;
         const uint32_t t_lane = tmem_base + ((uint32_t)(quad * 32) << 16);
         const uint32_t tempty_leader0 = (CG == 2) ? map_to_rank(smem_u32(&tempty[0]), 0) : 0u;
         const uint32_t buf = smem_u32(sOut) + (uint32_t)(warp - 2) * kOutBoxBytes;
+        const unsigned nrows = (unsigned)p.rows;
+        const int ngrp = (p.n_out + kCombineCols - 1) / kCombineCols;  // down: arrival counters per token
         uint32_t tcount = 0;
         for (;; ++tcount) {
             bool got = true;
@@ -686,11 +849,6 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
             decode_tile_rows(tile, s_beg, s_end, p.E, p.n_tiles, C::kTileRows, e, mb, nb);
             const uint32_t acc = tcount % C::kNAcc;
             const uint32_t use = tcount / C::kNAcc;
-            // every lane waits; the decision to stop is warp-uniform so the
-            // .sync.aligned TMEM loads below always run on a converged warp
-            const bool okw = wait_bounded_pair(smem_u32(&tfull[acc]), use & 1u, abort_flag, p.err, peer_abort);
-            if (!__all_sync(0xffffffffu, okw)) break;
-            tc_fence_after();
             const int start = s_beg[e] + mb * C::kTileRows;
             const int tile_end = min(s_end[e], start + C::kTileRows);
             // Rows and accumulator columns of this warp's TMEM lanes.  Full
@@ -708,17 +866,51 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
             // expert's rows)
             const int wrow0 = row - lane;
             const bool box_ok = wrow0 + 32 <= tile_end;
-            int unit = 0;  // output units of the tile so far (this warp takes unit % 2 == sub)
-            // MMA h of the tile: accumulator columns h * BN .. h * BN + BN-1,
-            // output columns from hb (hidden units, up) or ob (down)
+            // down: the row's assignment, its gate weight, and its token's
+            // slot rows, loaded while the tile's MMAs run
+            int tok = 0, rr0 = -1, rr1 = -1, nvalid = 0;
+            bool row_ok = false;
+            float wgt = 0.f;
+            if constexpr (MODE == kDown) {
+                if (valid) {
+                    const int q = __ldg(p.perm + row);
+                    if ((unsigned)q < nrows) {
+                        row_ok = true;
+                        wgt = __ldg(p.topk_w + q);
+                        tok = q / p.k;
+                        const int32_t* iv = p.inv + (size_t)tok * p.k;
+                        rr0 = __ldg(iv);
+                        rr1 = p.k > 1 ? __ldg(iv + 1) : -1;
+                        nvalid = ((unsigned)rr0 < nrows ? 1 : 0) + ((unsigned)rr1 < nrows ? 1 : 0);
+                        for (int j = 2; j < p.k; ++j) nvalid += (unsigned)__ldg(iv + j) < nrows ? 1 : 0;
+                    }
+                }
+            }
+            // every lane waits; the decision to stop is warp-uniform so the
+            // .sync.aligned TMEM loads below always run on a converged warp
+            // (the failure-detection test waits on a barrier that nothing completes)
+            const bool okw = p.stall_test
+                                 ? wait_bounded_pair(smem_u32(stall_bar), 0u, abort_flag, p.err, peer_abort, p.wait_limit_ns)
+                                 : wait_bounded_pair(smem_u32(&tfull[acc]), use & 1u, abort_flag, p.err, peer_abort,
+                                                     p.wait_limit_ns);
+            if (!__all_sync(0xffffffffu, okw)) break;
+            tc_fence_after();
+            // down: 128-column groups of this warp, [g_lo, g_hi) of the quadrant's
+            // G = NH * gpp groups (gpp per MMA part; part h of a tile covers
+            // output columns nb * NH * BN + h * BN ..)
+            const int ncol = shrt ? BN / 2 : BN;  // columns of each MMA part held by the quadrant
+            const int cbase = colhalf * (BN / 2);
+            const int gpp = ncol / kCombineCols;
+            const int G = NH * gpp;
+            const int g_lo = sub ? (G + 1) / 2 : 0, g_hi = sub ? G : (G + 1) / 2;
+            (void)g_lo;
+            (void)g_hi;
+            if constexpr (MODE == kUp) {
+                int unit = 0;  // output units of the tile so far (this warp takes unit % 2 == sub)
 #pragma unroll 1
-            for (int h = 0; h < NH; ++h) {
-                const uint32_t tacc = t_lane + acc * C::kTileN + h * BN;
-                const int hb = nb * (NH * BN / 2) + h * (BN / 2);
-                const int ob = nb * (NH * BN) + h * BN;
-                (void)hb;
-                (void)ob;
-                if constexpr (MODE == kUp) {
+                for (int h = 0; h < NH; ++h) {
+                    const uint32_t tacc = t_lane + acc * C::kTileN + h * BN;
+                    const int hb = nb * (NH * BN / 2) + h * (BN / 2);  // first hidden unit of MMA h
                     __nv_bfloat16* hrow = p.h + (size_t)row * p.n_out;
                     // 64-unit segments: hidden units c64 .. c64+63 of the tile have
                     // a at TMEM columns acol .. acol+63 and b at acol+bdelta ...
@@ -727,7 +919,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
                     //   pair, short: one half per lane group, at columns 0-127.
                     const int nseg = (CG == 1) ? BN / 128 : (shrt ? 1 : 2);
                     const int bdelta = (CG == 1) ? BN / 2 : 64;
-    #pragma unroll 1
+#pragma unroll 1
                     for (int seg = 0; seg < nseg; ++seg) {
                         if ((unit++ & 1) != sub) continue;
                         const int c64 = (shrt ? colhalf : seg) * 64;        // hidden offset in the tile
@@ -736,7 +928,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
                             if (lane == 0) bulk_wait_read_all();  // the buffer's previous store has read it
                             __syncwarp();
                         }
-    #pragma unroll 1
+#pragma unroll 1
                         for (int half = 0; half < 2; ++half) {
                             const int c = c64 + half * 32;
                             uint32_t a[32], b[32];
@@ -744,7 +936,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
                             tmem_ld32(tacc + acol + half * 32 + bdelta, b);
                             tmem_wait_ld();
                             uint4 pk[4];
-    #pragma unroll
+#pragma unroll
                             for (int g = 0; g < 4; ++g) {
                                 pk[g].x = pack_bf16x2(silu_mul(__uint_as_float(a[g * 8 + 0]), __uint_as_float(b[g * 8 + 0])),
                                                       silu_mul(__uint_as_float(a[g * 8 + 1]), __uint_as_float(b[g * 8 + 1])));
@@ -756,12 +948,12 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
                                                       silu_mul(__uint_as_float(a[g * 8 + 7]), __uint_as_float(b[g * 8 + 7])));
                             }
                             if (box_ok) {
-    #pragma unroll
+#pragma unroll
                                 for (int g = 0; g < 4; ++g)
                                     st_shared_v4(buf + lane * 128 + ((((half * 4 + g) ^ (lane & 7))) << 4), pk[g]);
                             } else if (valid) {
                                 const int col0 = hb + c;
-    #pragma unroll
+#pragma unroll
                                 for (int g = 0; g < 4; ++g)
                                     if (col0 + g * 8 < p.n_out) *reinterpret_cast<uint4*>(hrow + col0 + g * 8) = pk[g];
                             }
@@ -777,21 +969,19 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
                             }
                         }
                     }
-                } else {
-                    float wgt = 0.f;
-                    if (valid) {
-                        const int q = p.perm[row];
-                        wgt = ((unsigned)q < (unsigned)p.rows) ? p.topk_w[q] : 0.f;
-                    }
-                    float* orow = p.obuf + (size_t)row * p.n_out;
-                    // short pair tiles: this warp's lanes hold BN/2 columns,
-                    // starting at output column colhalf * BN/2
-                    const int ncol = shrt ? BN / 2 : BN;
-                    const int cbase = colhalf * (BN / 2);
-    #pragma unroll 1
-                    for (int cc = 0; cc < ncol; cc += 32) {
-                        if ((unit++ & 1) != sub) continue;
-                        const int c = cbase + cc;  // tile column
+                }
+            } else {
+                // park: the gate-scaled fp32 rows of this warp's groups in obuf
+                float* orow = p.obuf + (size_t)row * p.n_out;
+#pragma unroll 1
+                for (int g = g_lo; g < g_hi; ++g) {
+                    const int h = g / gpp;
+                    const uint32_t tacc = t_lane + acc * C::kTileN + h * BN;
+                    const int ob = nb * (NH * BN) + h * BN + cbase;  // output column of TMEM column 0 of part h
+#pragma unroll 1
+                    for (int u = 0; u < kCombineCols / 32; ++u) {
+                        const int cc = (g - h * gpp) * kCombineCols + u * 32;  // TMEM column within part h
+                        const int col = ob + cc;
                         if (box_ok) {
                             if (lane == 0) bulk_wait_read_all();  // the buffer's previous store has read it
                             __syncwarp();
@@ -800,27 +990,26 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
                         tmem_ld32(tacc + cc, o);
                         tmem_wait_ld();
                         uint4 v[8];
-    #pragma unroll
-                        for (int g = 0; g < 8; ++g) {
-                            v[g].x = __float_as_uint(wgt * __uint_as_float(o[g * 4 + 0]));
-                            v[g].y = __float_as_uint(wgt * __uint_as_float(o[g * 4 + 1]));
-                            v[g].z = __float_as_uint(wgt * __uint_as_float(o[g * 4 + 2]));
-                            v[g].w = __float_as_uint(wgt * __uint_as_float(o[g * 4 + 3]));
+#pragma unroll
+                        for (int i = 0; i < 8; ++i) {
+                            v[i].x = __float_as_uint(wgt * __uint_as_float(o[i * 4 + 0]));
+                            v[i].y = __float_as_uint(wgt * __uint_as_float(o[i * 4 + 1]));
+                            v[i].z = __float_as_uint(wgt * __uint_as_float(o[i * 4 + 2]));
+                            v[i].w = __float_as_uint(wgt * __uint_as_float(o[i * 4 + 3]));
                         }
                         if (box_ok) {
-    #pragma unroll
-                            for (int g = 0; g < 8; ++g) st_shared_v4(buf + lane * 128 + ((g ^ (lane & 7)) << 4), v[g]);
+#pragma unroll
+                            for (int i = 0; i < 8; ++i) st_shared_v4(buf + lane * 128 + ((i ^ (lane & 7)) << 4), v[i]);
                             fence_proxy_async_smem();
                             __syncwarp();
                             if (lane == 0) {
-                                if (ob + c < p.n_out) tma_store_2d(&tmOut, buf, ob + c, wrow0);
+                                if (col < p.n_out) tma_store_2d(&tmOut, buf, col, wrow0);
                                 bulk_commit();
                             }
                         } else if (valid) {
-                            const int col0 = ob + c;
-    #pragma unroll
-                            for (int g = 0; g < 8; ++g)
-                                if (col0 + g * 4 < p.n_out) *reinterpret_cast<uint4*>(orow + col0 + g * 4) = v[g];
+#pragma unroll
+                            for (int i = 0; i < 8; ++i)
+                                if (col + i * 4 < p.n_out) *reinterpret_cast<uint4*>(orow + col + i * 4) = v[i];
                         }
                     }
                 }
@@ -830,6 +1019,37 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
             if (lane == 0) {
                 if constexpr (CG == 1) mbar_arrive(smem_u32(&tempty[acc]));
                 else mbar_arrive_cluster(tempty_leader0 + acc * (uint32_t)sizeof(uint64_t));
+            }
+            if constexpr (MODE == kDown) {
+                // Count the parked groups (release: the park stores are complete
+                // and ordered before the counts), then let the last arrivals sum.
+                if (lane == 0) {
+                    bulk_wait_all();
+                    fence_proxy_async_global();
+                }
+                __syncwarp();
+                __threadfence();
+                unsigned last = 0;
+                if (row_ok) {
+                    for (int g = g_lo; g < g_hi; ++g) {
+                        const int h = g / gpp;
+                        const int col = nb * (NH * BN) + h * BN + cbase + (g - h * gpp) * kCombineCols;
+                        if (col >= p.n_out) continue;
+                        const bool is_last =
+                            p.k == 1 || atomicAdd(p.arrivals + (size_t)tok * ngrp + col / kCombineCols, 1u) == (unsigned)(nvalid - 1);
+                        if (is_last) last |= 1u << (g - g_lo);
+                    }
+                }
+                if (__any_sync(0xffffffffu, last != 0)) {
+                    __threadfence();  // acquire: the other slots' parked rows
+                    for (int g = g_lo; g < g_hi; ++g) {
+                        const unsigned m = __ballot_sync(0xffffffffu, (last >> (g - g_lo)) & 1u);
+                        if (!m) continue;
+                        const int h = g / gpp;
+                        const int col = nb * (NH * BN) + h * BN + cbase + (g - h * gpp) * kCombineCols;
+                        combine_group(m, tok, rr0, rr1, col, p, lane);
+                    }
+                }
             }
         }
         if (lane == 0) bulk_wait_all();  // stores complete before the CTA's shared memory goes away
@@ -849,6 +1069,15 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
 
 // ---------------------------------------------------------------------------
 // Host side: tensor maps through the driver entry point (no libcuda link).
+
+// Process-wide settings of the test and measurement hooks (moe.h:
+// moe_set_gemm_variant, moe_set_wait_test); 0 = automatic / default.
+std::atomic<int> g_force_cg{0};         // 1 single-CTA tiles, 2 CTA pairs, 3 hybrid
+std::atomic<int> g_force_up_bn{0};      // 128 or 256: single-CTA up-projection tile width
+std::atomic<int> g_force_rows{0};       // 32 or 128: token rows of a single-CTA tile
+std::atomic<int> g_force_pair_cols{0};  // 256 or 512: columns of a pair tile
+std::atomic<unsigned long long> g_wait_limit_ns{kWaitLimitNs};
+std::atomic<int> g_stall_test{0};
 
 PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
 const char* g_init_err = nullptr;
@@ -895,9 +1124,12 @@ struct GemmMaps {
 
 template <int MODE, int CG, int BN, int RB, int NH = 1>
 cudaError_t launch_gemm(const GroupedGemmArgs& a, const CUtensorMap& mA, const CUtensorMap& mAs,
-                        const CUtensorMap& mB0, const CUtensorMap& mB1, const CUtensorMap& mOut, const KParams& p,
+                        const CUtensorMap& mB0, const CUtensorMap& mB1, const CUtensorMap& mOut, const KParams& p0,
                         cudaStream_t s) {
     using C = Cfg<CG, BN, RB, NH>;
+    KParams p = p0;
+    p.wait_limit_ns = g_wait_limit_ns.load(std::memory_order_relaxed);
+    p.stall_test = g_stall_test.load(std::memory_order_relaxed);
     static int units_cache[64] = {0};
     int dev = 0;
     cudaGetDevice(&dev);
@@ -951,14 +1183,11 @@ cudaError_t launch_gemm(const GroupedGemmArgs& a, const CUtensorMap& mA, const C
 //    the remaining rows) was slower: the second launch has only 1-2 row
 //    tiles per weight tile and streams every expert's weights again;
 //  * decode (a few rows per expert): single-CTA tiles of 32 token rows.
-// Pairs are used once experts average 512 rows; MOE_GEMM_CTA_GROUP = 1, 2 or
-// h forces a variant (all exact; the tests run each).
+// Pairs are used once experts average 512 rows; moe_set_gemm_variant forces
+// a variant (all exact; the tests run each).
 int choose_cta_group(const GroupedGemmArgs& a, int mode) {
-    if (const char* env = getenv("MOE_GEMM_CTA_GROUP")) {
-        if (env[0] == '1') return 1;
-        if (env[0] == '2') return 2;
-        if (env[0] == 'h') return 3;
-    }
+    const int forced = g_force_cg.load(std::memory_order_relaxed);
+    if (forced) return forced;
     (void)mode;
     return a.rows >= 512 * a.E ? 2 : 1;
 }
@@ -970,37 +1199,49 @@ const char* gemm_init_error() {
     return g_init_err;
 }
 
+int set_gemm_variant(int cta_group, int up_bn, int token_rows, int pair_cols) {
+    if (cta_group < 0 || cta_group > 3 || (up_bn && up_bn != 128 && up_bn != 256) ||
+        (token_rows && token_rows != 32 && token_rows != 128) ||
+        (pair_cols && pair_cols != 256 && pair_cols != 512))
+        return -1;
+    g_force_cg.store(cta_group);
+    g_force_up_bn.store(up_bn);
+    g_force_rows.store(token_rows);
+    g_force_pair_cols.store(pair_cols);
+    return 0;
+}
+
+void set_wait_test(unsigned long long wait_limit_ns, int stall) {
+    g_wait_limit_ns.store(wait_limit_ns ? wait_limit_ns : kWaitLimitNs);
+    g_stall_test.store(stall ? 1 : 0);
+}
+
 namespace {
 
 // N width of the up-projection tiles: 256 (128 hidden units of W1 and of
 // W3).  128-wide tiles (64 + 64) exist for finer load balance, but measured
 // on B200 at decode (T = 32) they were slower (0.336 vs 0.323 ms): twice the
 // tiles cost more per-tile work than the shorter last wave saves.
-// MOE_GEMM_BN = 128 selects them (exact; the tests run both widths).
+// moe_set_gemm_variant can select them (exact; the tests run both widths).
 int choose_up_bn(const GroupedGemmArgs&) {
-    if (const char* env = getenv("MOE_GEMM_BN")) {
-        if (env[0] == '1') return 128;
-    }
-    return 256;
+    const int forced = g_force_up_bn.load(std::memory_order_relaxed);
+    return forced ? forced : 256;
 }
 
 // Token rows per single-CTA tile: 32 when experts average at most 16 rows
 // (decode), so tiles do not stream 128 mostly unused A rows from L2 for every
-// weight tile; 128 otherwise.  MOE_GEMM_RB = 32 or 128 forces it.
+// weight tile; 128 otherwise (or as moe_set_gemm_variant forces).
 int choose_rb(const GroupedGemmArgs& a) {
-    if (const char* env = getenv("MOE_GEMM_RB")) {
-        if (env[0] == '3') return 32;
-        if (env[0] == '1') return 128;
-    }
+    const int forced = g_force_rows.load(std::memory_order_relaxed);
+    if (forced) return forced;
     return a.rows <= 16 * a.E ? 32 : 128;
 }
 
 // Pair tiles of 256 x 512 (two N = 256 MMAs sharing each A tile; default)
 // or 256 x 256 (two TMEM accumulator buffers, epilogue overlapped).
-// MOE_GEMM_WIDE = 1 or 0 forces one.
 bool choose_wide(const GroupedGemmArgs&) {
-    if (const char* env = getenv("MOE_GEMM_WIDE")) return env[0] == '1';
-    return true;
+    const int forced = g_force_pair_cols.load(std::memory_order_relaxed);
+    return forced ? forced == 512 : true;
 }
 
 template <int MODE, int BN>
@@ -1035,7 +1276,7 @@ cudaError_t launch_variant(const GroupedGemmArgs& a, const GemmMaps& m, const KP
 cudaError_t launch_up_swiglu(const GroupedGemmArgs& a, const __nv_bfloat16* x_perm,
                              const __nv_bfloat16* W1, const __nv_bfloat16* W3, __nv_bfloat16* h,
                              cudaStream_t s) {
-    // pairs and the hybrid use 256-column tiles whatever MOE_GEMM_BN says
+    // pairs and the hybrid use 256-column tiles whatever the forced width
     const int bn = choose_cta_group(a, kUp) == 1 ? choose_up_bn(a) : 256;
     GemmMaps m;
     if (!make_map(&m.A, x_perm, (uint64_t)a.rows, (uint64_t)a.d, BM) ||
@@ -1055,15 +1296,13 @@ cudaError_t launch_up_swiglu(const GroupedGemmArgs& a, const __nv_bfloat16* x_pe
     return bn == 128 ? launch_variant<kUp, 128>(a, m, p, s) : launch_variant<kUp, 256>(a, m, p, s);
 }
 
-cudaError_t launch_down_scaled(const GroupedGemmArgs& a, const __nv_bfloat16* h,
-                               const __nv_bfloat16* W2, const int32_t* perm, const float* topk_w,
-                               float* obuf, cudaStream_t s) {
+cudaError_t launch_down_combine(const GroupedGemmArgs& a, const DownCombineArgs& c, cudaStream_t s) {
     GemmMaps m;
-    if (!make_map(&m.A, h, (uint64_t)a.rows, (uint64_t)a.f, BM) ||
-        !make_map(&m.A32, h, (uint64_t)a.rows, (uint64_t)a.f, 32) ||
-        !make_map(&m.A64, h, (uint64_t)a.rows, (uint64_t)a.f, 64) ||
-        !make_map(&m.B0, W2, (uint64_t)a.E * a.d, (uint64_t)a.f, 128) ||
-        !make_map(&m.Out, obuf, (uint64_t)a.rows, (uint64_t)a.d, 32, true))
+    if (!make_map(&m.A, c.h, (uint64_t)a.rows, (uint64_t)a.f, BM) ||
+        !make_map(&m.A32, c.h, (uint64_t)a.rows, (uint64_t)a.f, 32) ||
+        !make_map(&m.A64, c.h, (uint64_t)a.rows, (uint64_t)a.f, 64) ||
+        !make_map(&m.B0, c.W2, (uint64_t)a.E * a.d, (uint64_t)a.f, 128) ||
+        !make_map(&m.Out, c.obuf, (uint64_t)a.rows, (uint64_t)a.d, 32, true))
         return cudaErrorInvalidValue;
     m.B1 = m.B0;
     m.B0p = m.B0;
@@ -1071,7 +1310,9 @@ cudaError_t launch_down_scaled(const GroupedGemmArgs& a, const __nv_bfloat16* h,
     KParams p{};
     p.offsets = a.offsets; p.E = a.E; p.n_out = a.d; p.Kdim = a.f;
     p.n_tiles = (a.d + 255) / 256; p.b_rows_per_expert = a.d;
-    p.perm = perm; p.topk_w = topk_w; p.obuf = obuf; p.rows = a.rows;
+    p.perm = c.perm; p.inv = c.inv; p.topk_w = c.topk_w; p.obuf = c.obuf;
+    p.arrivals = c.arrivals; p.y = c.y; p.residual = c.residual; p.k = c.k;
+    p.rows = a.rows;
     p.err = a.err;
     p.tile_counter = a.tile_counters + 2;
     return launch_variant<kDown, 256>(a, m, p, s);

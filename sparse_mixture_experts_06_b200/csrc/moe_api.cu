@@ -1,6 +1,7 @@
 // C ABI of the sparse MoE layer (declared in include/moe.h): argument
 // validation, workspace layout, and the launch sequence
-//   router_topk -> permute -> [gather] -> up GEMM -> down GEMM -> combine
+//   bf16: router_topk -> permute -> [gather] -> up GEMM -> down GEMM (+ combine)
+//   fp32: router_topk -> permute -> fp32 expert kernels -> combine
 // on the caller's stream.  Nothing here waits on the device.
 
 #include <cstdarg>
@@ -99,6 +100,8 @@ Workspace carve_workspace(void* base, int T, int d, int f, int E, int k, bool bf
     w.h = take(n * f * (bf16 ? 2 : 4));
     w.obuf = reinterpret_cast<float*>(take(n * d * 4));
     w.tile_counters = reinterpret_cast<int32_t*>(take(kTileCounters * 4));
+    w.arrivals_bytes = align256((size_t)T * ((d + kCombineCols - 1) / kCombineCols) * 4);
+    w.arrivals = reinterpret_cast<unsigned int*>(take(w.arrivals_bytes));
     w.chunk_base = reinterpret_cast<int32_t*>(take((size_t)E * ((n + kChunkA - 1) / kChunkA) * 4));
     w.bytes = off;
     return w;
@@ -111,7 +114,7 @@ namespace {
 // ---- optional per-stage event timing (moe_profile_*) --------------------
 enum Stage { kRouter = 0, kPermute, kGather, kUp, kDown, kCombine, kFfnF32, kNumStages };
 const char* const kStageNames[kNumStages] = {"router_topk", "permute", "gather_rows", "up_swiglu_gemm",
-                                             "down_scaled_gemm", "combine", "ffn_f32"};
+                                             "down_combine_gemm", "combine", "ffn_f32"};
 constexpr int kMaxProfiled = 8192;
 struct Prof {
     std::mutex mu;
@@ -142,9 +145,15 @@ struct StageTimer {
     }
 };
 
+// What the permutation kernels clear for the GEMMs of carved workspace `w`.
+moe::ZeroArgs zero_args(const moe::Workspace& w) {
+    return moe::ZeroArgs{w.tile_counters, reinterpret_cast<uint4*>(w.arrivals), (long long)(w.arrivals_bytes / 16)};
+}
+
 // Experts + combine on carved workspace `w` (routing fields supplied by the
 // caller).  x_gathered: w.x_perm already holds the permuted rows of x and the
-// tile counters are zero (the chunked permutation did both).
+// counters are clear (the chunked permutation did both).  bf16: the combine
+// runs in the down-projection GEMM's epilogue; fp32: a separate kernel.
 int run_ffn(const void* x, const void* W1, const void* W3, const void* W2, const int32_t* offsets,
             const int32_t* perm, const int32_t* inv, const float* topk_w, const void* residual,
             int T, int d, int f, int E, int k, bool bf16, const moe::Workspace& w, void* y,
@@ -155,8 +164,9 @@ int run_ffn(const void* x, const void* W1, const void* W3, const void* W2, const
         if (const char* msg = moe::gemm_init_error()) return fail(MOE_ERR_CUDA, "%s", msg);
         if (!x_gathered) {
             StageTimer tm(kGather, s);
+            const moe::UnroutedArgs u{inv, T, k, d, y, residual};
             e = moe::launch_gather_rows_bf16(static_cast<const __nv_bfloat16*>(x), perm, rows, d, k,
-                                             static_cast<__nv_bfloat16*>(w.x_perm), w.tile_counters, s);
+                                             static_cast<__nv_bfloat16*>(w.x_perm), zero_args(w), u, s);
             tm.done(s);
             if (e != cudaSuccess) return cuda_fail(e, "gather_rows");
         }
@@ -173,12 +183,16 @@ int run_ffn(const void* x, const void* W1, const void* W3, const void* W2, const
         if (e != cudaSuccess) return cuda_fail(e, "grouped up-projection GEMM");
         {
             StageTimer tm(kDown, s);
-            e = moe::launch_down_scaled(a, static_cast<const __nv_bfloat16*>(w.h),
-                                        static_cast<const __nv_bfloat16*>(W2), perm, topk_w, w.obuf, s);
+            moe::DownCombineArgs c{static_cast<const __nv_bfloat16*>(w.h), static_cast<const __nv_bfloat16*>(W2),
+                                   perm, inv, topk_w, w.obuf, w.arrivals,
+                                   static_cast<const __nv_bfloat16*>(residual), static_cast<__nv_bfloat16*>(y), k};
+            e = moe::launch_down_combine(a, c, s);
             tm.done(s);
         }
         if (e != cudaSuccess) return cuda_fail(e, "grouped down-projection GEMM");
-    } else {
+        return MOE_OK;
+    }
+    {
         StageTimer tm(kFfnF32, s);
         e = moe::launch_ffn_f32(static_cast<const float*>(x), static_cast<const float*>(W1),
                                 static_cast<const float*>(W3), static_cast<const float*>(W2), offsets, perm,
@@ -188,7 +202,7 @@ int run_ffn(const void* x, const void* W1, const void* W3, const void* W2, const
     }
     {
         StageTimer tm(kCombine, s);
-        e = moe::launch_combine(w.obuf, inv, residual, T, d, k, bf16, y, s);
+        e = moe::launch_combine_f32(w.obuf, inv, static_cast<const float*>(residual), T, d, k, static_cast<float*>(y), s);
         tm.done(s);
     }
     if (e != cudaSuccess) return cuda_fail(e, "combine");
@@ -198,18 +212,29 @@ int run_ffn(const void* x, const void* W1, const void* W3, const void* W2, const
 struct Pool {
     void* ptr = nullptr;
     size_t bytes = 0;
+    cudaEvent_t last_use = nullptr;  // recorded after the work of every call that used ptr
 };
 std::mutex g_pool_mu;
 Pool g_pool[64];
 
 // The library-owned workspace of device `dev`, at least `need` bytes:
-// grown (stream-ordered free + malloc on s) when a larger shape arrives.
+// grown (stream-ordered free + malloc on s) when a larger shape arrives.  The
+// free waits for the last work that used the old workspace, on whatever
+// stream that was (pool_used records it).
 int pool_workspace(int dev, size_t need, cudaStream_t s, void** out) {
     std::lock_guard<std::mutex> lock(g_pool_mu);
     Pool& p = g_pool[dev];
+    if (!p.last_use) {
+        cudaError_t e = cudaEventCreateWithFlags(&p.last_use, cudaEventDisableTiming);
+        if (e != cudaSuccess) {
+            p.last_use = nullptr;
+            return cuda_fail(e, "cudaEventCreate(workspace)");
+        }
+    }
     if (p.bytes < need) {
         if (p.ptr) {
-            cudaError_t e = cudaFreeAsync(p.ptr, s);
+            cudaError_t e = cudaStreamWaitEvent(s, p.last_use, 0);
+            if (e == cudaSuccess) e = cudaFreeAsync(p.ptr, s);
             p.ptr = nullptr;
             p.bytes = 0;
             if (e != cudaSuccess) return cuda_fail(e, "cudaFreeAsync(workspace)");
@@ -223,6 +248,20 @@ int pool_workspace(int dev, size_t need, cudaStream_t s, void** out) {
     }
     *out = p.ptr;
     return MOE_OK;
+}
+
+// Marks the end of the work just enqueued on s with the pool's workspace.
+// Not during a stream capture: an event recorded there belongs to the graph
+// and cannot order work outside it (a captured call runs on a workspace that
+// exists before the capture and is kept while the graph lives).
+int pool_used(int dev, cudaStream_t s) {
+    cudaStreamCaptureStatus st = cudaStreamCaptureStatusNone;
+    cudaError_t e = cudaStreamIsCapturing(s, &st);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaStreamIsCapturing");
+    if (st != cudaStreamCaptureStatusNone) return MOE_OK;
+    std::lock_guard<std::mutex> lock(g_pool_mu);
+    e = cudaEventRecord(g_pool[dev].last_use, s);
+    return e == cudaSuccess ? MOE_OK : cuda_fail(e, "cudaEventRecord(workspace)");
 }
 
 // Copy streams, events and staging memory of moe_layer_forward_host, per
@@ -408,7 +447,7 @@ int moe_layer_forward_ex(const void* x, const void* Wg, const void* W1, const vo
         StageTimer tm(kGather, s);
         e = moe::launch_chunk_scatter(w.topk_idx, T * k, E, k, w.chunk_base, w.perm, w.inv,
                                       bf16 ? static_cast<const __nv_bfloat16*>(x) : nullptr, d,
-                                      bf16 ? static_cast<__nv_bfloat16*>(w.x_perm) : nullptr, w.tile_counters, s);
+                                      bf16 ? static_cast<__nv_bfloat16*>(w.x_perm) : nullptr, zero_args(w), s);
         tm.done(s);
         if (e != cudaSuccess) return cuda_fail(e, "permutation scatter");
     }
@@ -460,7 +499,8 @@ int moe_layer_forward(const void* x, const void* Wg, const void* W1, const void*
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     void* ws = nullptr;
     CHECK(pool_workspace(dev, need, s, &ws));
-    return moe_layer_forward_ex(x, Wg, W1, W3, W2, nullptr, T, d, f, E, k, MOE_BF16, ws, need, y, stream);
+    CHECK(moe_layer_forward_ex(x, Wg, W1, W3, W2, nullptr, T, d, f, E, k, MOE_BF16, ws, need, y, stream));
+    return pool_used(dev, s);
 }
 
 int moe_layer_forward_host(const void* x_host, const void* Wg, const void* W1, const void* W3,
@@ -532,6 +572,7 @@ int moe_layer_forward_host(const void* x_host, const void* Wg, const void* W1, c
             return cuda_fail(e, "cudaStreamWaitEvent");
         CHECK(moe_layer_forward_ex(xbuf[b], Wg, W1, W3, W2, nullptr, tc, d, f, E, k, MOE_BF16, ws, ws_need,
                                    ybuf[b], stream));
+        CHECK(pool_used(dev, s));
         if ((e = cudaEventRecord(P.comp_done[b], s)) != cudaSuccess)
             return cuda_fail(e, "cudaEventRecord");
         // y rows out
@@ -578,7 +619,8 @@ int moe_release_workspace(moe_stream_t stream) {
         std::lock_guard<std::mutex> lock(g_pool_mu);
         Pool& p = g_pool[dev];
         if (p.ptr) {
-            e = cudaFreeAsync(p.ptr, s);
+            e = cudaStreamWaitEvent(s, p.last_use, 0);
+            if (e == cudaSuccess) e = cudaFreeAsync(p.ptr, s);
             p.ptr = nullptr;
             p.bytes = 0;
             if (e != cudaSuccess) return cuda_fail(e, "cudaFreeAsync(workspace)");
@@ -674,6 +716,20 @@ int moe_profile_select(unsigned int stage_mask) {
 
 const char* moe_profile_stage_name(int stage) {
     return (stage >= 0 && stage < kNumStages) ? kStageNames[stage] : "";
+}
+
+int moe_set_gemm_variant(int cta_group, int up_bn, int token_rows, int pair_cols) {
+    g_last_error.clear();
+    if (moe::set_gemm_variant(cta_group, up_bn, token_rows, pair_cols) != 0)
+        return fail(MOE_ERR_INVALID_ARG, "moe_set_gemm_variant(%d, %d, %d, %d): a value outside its choices",
+                    cta_group, up_bn, token_rows, pair_cols);
+    return MOE_OK;
+}
+
+int moe_set_wait_test(unsigned long long wait_limit_ns, int stall_epilogue) {
+    g_last_error.clear();
+    moe::set_wait_test(wait_limit_ns, stall_epilogue);
+    return MOE_OK;
 }
 
 const char* moe_last_error_string(void) { return g_last_error.c_str(); }

@@ -34,6 +34,25 @@ constexpr int kMaxTopK = kMaxExperts;  // any k <= E
 constexpr int kTileCounters = 4;        // up, up (second hybrid launch), down, down (second)
 constexpr int kChunkA = 64;             // assignments per chunk of the layer's permutation
 constexpr int kChunkScanMaxCells = 48 * 1024;  // E x chunks counted in shared memory (192 KiB)
+constexpr int kCombineCols = 128;       // output columns per arrival counter of the fused combine
+
+// Memory the permutation kernels clear for the GEMMs that follow on the
+// stream: the tile counters and the combine's arrival counters.
+struct ZeroArgs {
+    int32_t* tile_counters;  // [kTileCounters] (may be null)
+    uint4* arrivals;         // [n16] 16-byte words (may be null)
+    long long n16;
+};
+
+// Tokens none of whose k slots is routed (inv out of range; only from a
+// caller's own routing) get no row in the down-projection, whose epilogue
+// writes y: the row gather writes their y rows (the residual, or zero).
+struct UnroutedArgs {
+    const int32_t* inv;   // [T*k]
+    int T, k, d;
+    void* y;              // [T, d] bf16; null: nothing to do
+    const void* residual;  // [T, d] bf16 or null
+};
 
 // 256-byte aligned carve-up of one workspace blob.
 struct Workspace {
@@ -46,6 +65,9 @@ struct Workspace {
     void* h;            // [T*k, f]  bf16 or f32
     float* obuf;        // [T*k, d]  gate-scaled expert outputs, fp32
     int32_t* tile_counters;  // [kTileCounters] GEMM tile schedulers, zeroed by the row gather
+    unsigned int* arrivals;  // [T, ceil(d / kCombineCols)] slot arrivals of the fused combine, zeroed
+                             // with the tile counters
+    size_t arrivals_bytes;   // bytes of the arrivals region (a multiple of 256)
     int32_t* chunk_base;     // [E * ceil(T*k / kChunkA)] first row of each (expert, chunk)
     size_t bytes;
 };
@@ -61,20 +83,22 @@ cudaError_t launch_permute(const int32_t* idx, int n, int E, int32_t* offsets, i
 // expert counts, their scan into chunk_base and offsets), then scatter (one
 // block per chunk: ranks, writes perm / inv and, if x_perm is not null,
 // copies the x rows).  Same results as launch_permute followed by
-// launch_gather_rows_bf16, whose work it replaces, including the zeroing of
-// tile_counters (may be null).  Only when chunked_permute_fits(n, E).
+// launch_gather_rows_bf16, whose work it replaces, including the clearing
+// of `z`.  Only when chunked_permute_fits(n, E).
 bool chunked_permute_fits(int n, int E);
 cudaError_t launch_chunk_count_scan(const int32_t* idx, int n, int E, int32_t* chunk_base, int32_t* offsets,
                                     cudaStream_t s);
 cudaError_t launch_chunk_scatter(const int32_t* idx, int n, int E, int k, const int32_t* chunk_base,
                                  int32_t* perm, int32_t* inv, const __nv_bfloat16* x, int d,
-                                 __nv_bfloat16* x_perm, int32_t* tile_counters, cudaStream_t s);
-// Also zeroes tile_counters[0 .. kTileCounters) for the GEMMs that follow on
-// the same stream.
+                                 __nv_bfloat16* x_perm, const ZeroArgs& z, cudaStream_t s);
+// Also clears the memory of `z` for the GEMMs that follow on the same stream
+// and writes the y rows of unrouted tokens (`u`).
 cudaError_t launch_gather_rows_bf16(const __nv_bfloat16* x, const int32_t* perm, int rows, int d,
-                                    int k, __nv_bfloat16* x_perm, int32_t* tile_counters, cudaStream_t s);
-cudaError_t launch_combine(const float* obuf, const int32_t* inv, const void* residual, int T,
-                           int d, int k, bool bf16, void* y, cudaStream_t s);
+                                    int k, __nv_bfloat16* x_perm, const ZeroArgs& z, const UnroutedArgs& u,
+                                    cudaStream_t s);
+// fp32 path: y[t] = (residual[t] +) sum_j obuf[inv[t*k + j]] in slot order
+cudaError_t launch_combine_f32(const float* obuf, const int32_t* inv, const float* residual, int T, int d, int k,
+                               float* y, cudaStream_t s);
 
 cudaError_t launch_routing_stats(const int32_t* idx, int T, int E, int k, int seq_len, unsigned int* out,
                                  cudaStream_t s);
@@ -91,10 +115,28 @@ struct GroupedGemmArgs {
 cudaError_t launch_up_swiglu(const GroupedGemmArgs& a, const __nv_bfloat16* x_perm,
                              const __nv_bfloat16* W1, const __nv_bfloat16* W3, __nv_bfloat16* h,
                              cudaStream_t s);
-cudaError_t launch_down_scaled(const GroupedGemmArgs& a, const __nv_bfloat16* h,
-                               const __nv_bfloat16* W2, const int32_t* perm, const float* topk_w,
-                               float* obuf, cudaStream_t s);
+// Down-projection with the gate weighting and the combine in its epilogue:
+// y[t] = (residual[t] +) sum_j topk_w[t*k+j] * (W2_e h_{inv[t*k+j]}), slots
+// in order, one rounding to bf16.  obuf parks the gate-scaled rows; the
+// arrival counters must be zero at launch.
+struct DownCombineArgs {
+    const __nv_bfloat16* h;
+    const __nv_bfloat16* W2;
+    const int32_t* perm;
+    const int32_t* inv;
+    const float* topk_w;
+    float* obuf;
+    unsigned int* arrivals;
+    const __nv_bfloat16* residual;  // may be null
+    __nv_bfloat16* y;
+    int k;
+};
+cudaError_t launch_down_combine(const GroupedGemmArgs& a, const DownCombineArgs& c, cudaStream_t s);
 const char* gemm_init_error();  // non-null if the driver entry point is missing
+// Test and measurement hooks (moe_set_gemm_variant, moe_set_wait_test):
+// process-wide, read at every GEMM launch.
+int set_gemm_variant(int cta_group, int up_bn, int token_rows, int pair_cols);  // -1: invalid value
+void set_wait_test(unsigned long long wait_limit_ns, int stall);
 
 // fp32 SIMT expert path (ffn_f32.cu)
 cudaError_t launch_ffn_f32(const float* x, const float* W1, const float* W3, const float* W2,

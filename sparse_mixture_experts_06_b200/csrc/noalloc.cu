@@ -11,9 +11,9 @@
 // uses a fixed scratch area compiled into the library instead.
 //
 // The scratch is a file-scope device array of kStaticScratchBytes (32 MiB),
-// enough for T*k*(2d + 2f + 4d) bytes plus small routing buffers: at the
-// Mixtral-8x7B dimensions (d = 4096, f = 14336, k = 2) that is up to 314
-// tokens per call.  Every GPU that loads this part of the library keeps the
+// enough for T*k*(2d + 2f + 4d) bytes plus small routing buffers and
+// counters: at the Mixtral-8x7B dimensions (d = 4096, f = 14336, k = 2) that
+// is up to 314 tokens per call.  Every GPU that loads this part of the library keeps the
 // 32 MiB until the process exits.  In host code the array's name is only a
 // stand-in, so its device address is looked up with cudaGetSymbolAddress on
 // the first call on each device (with that device current) and cached; make
@@ -21,7 +21,11 @@
 // the one array and the next call overwrites it: calls whose work overlaps
 // on the GPU (different streams, or different host threads) race and must be
 // serialised by the caller.  Nothing in the array has to start at zero:
-// every byte a kernel reads is written earlier in the same call.
+// every byte a kernel reads is written earlier in the same call (the
+// counters the expert GEMMs need at zero are cleared by the call's
+// permutation kernels).  The cached address dies with the device's context:
+// after cudaDeviceReset the library must not be used on that device again
+// in this process.
 
 #include <cstdio>
 #include <mutex>

@@ -9,7 +9,8 @@
 //                   per 64-assignment chunk ranks it stably, writes perm / inv
 //                   and copies the x rows to their permuted places
 //  gather_rows      x_perm[r] = x[perm[r] / k]            (bf16 path)
-//  combine_kernel   y[t] = (residual[t] +) sum_j obuf[inv[t*k + j]]
+//  combine_f32      y[t] = (residual[t] +) sum_j obuf[inv[t*k + j]]   (fp32
+//                   path; the bf16 down-projection GEMM does it in its epilogue)
 //
 // The gather and the combine give each row a block of threads that keep
 // 4 sixteen-byte loads each in flight (HBM-bound, not latency-bound).
@@ -102,6 +103,15 @@ permute_kernel(const int32_t* __restrict__ idx, int n, int E, int32_t* __restric
 constexpr int kFlatThreads = 256;
 constexpr int kUnroll = 4;  // 16-byte pieces in flight per thread in the row copies
 
+// Clears the GEMMs' tile counters (block 0) and the combine's arrival
+// counters (grid-strided) for the GEMMs that follow on the stream.
+__device__ __forceinline__ void clear_for_gemms(const ZeroArgs& z) {
+    if (blockIdx.x == 0 && z.tile_counters && threadIdx.x < kTileCounters) z.tile_counters[threadIdx.x] = 0;
+    const long long stride = (long long)gridDim.x * blockDim.x;
+    for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < z.n16; i += stride)
+        z.arrivals[i] = make_uint4(0u, 0u, 0u, 0u);
+}
+
 // ---- chunked permutation ---------------------------------------------------
 // Assignments q = 0 .. n-1 are cut into chunks of kChunkA.  base[e * nch + c]
 // = the first permuted row of chunk c's assignments to expert e = the
@@ -193,12 +203,12 @@ chunk_count_scan_kernel(const int32_t* __restrict__ idx, int n, int E, int nch, 
 
 // Block (chunk c, part): ranks the chunk's assignments; part 0 writes perm
 // and inv; every part copies the x rows of its share of the chunk (bf16
-// path; xp may be null).  Block 0 also zeroes the GEMM tile counters.
+// path; xp may be null).  The blocks also clear the memory of z.
 __global__ void __launch_bounds__(kScatThreads)
 chunk_scatter_kernel(const int32_t* __restrict__ idx, int n, int E, int nch, int k, int parts,
                      const int32_t* __restrict__ base, int32_t* __restrict__ perm, int32_t* __restrict__ inv,
                      const __nv_bfloat16* __restrict__ x, int d, __nv_bfloat16* __restrict__ xp,
-                     int32_t* __restrict__ tile_counters) {
+                     const ZeroArgs z) {
     constexpr int kRankWarps = kChunkA / 32;
     __shared__ int s_wcnt[kRankWarps][kMaxExperts];
     __shared__ int s_pos[kChunkA];
@@ -207,7 +217,7 @@ chunk_scatter_kernel(const int32_t* __restrict__ idx, int n, int E, int nch, int
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     pdl_wait();
     pdl_trigger();
-    if (blockIdx.x == 0 && tile_counters && tid < kTileCounters) tile_counters[tid] = 0;
+    clear_for_gemms(z);
     for (int i = tid; i < kRankWarps * kMaxExperts; i += kScatThreads) (&s_wcnt[0][0])[i] = 0;
     __syncthreads();
     const int q = c * kChunkA + tid;
@@ -270,10 +280,25 @@ chunk_scatter_kernel(const int32_t* __restrict__ idx, int n, int E, int nch, int
 // x_perm[r, :] = x[perm[r] / k, :]  (a row with an invalid assignment id is zero)
 __global__ void __launch_bounds__(kFlatThreads)
 gather_rows_kernel(const __nv_bfloat16* __restrict__ x, const int32_t* __restrict__ perm, int rows,
-                   int d, int k, __nv_bfloat16* __restrict__ xp, int32_t* __restrict__ tile_counters) {
+                   int d, int k, __nv_bfloat16* __restrict__ xp, const ZeroArgs z, const UnroutedArgs u) {
     pdl_wait();
     pdl_trigger();
-    if (blockIdx.x == 0 && threadIdx.x < kTileCounters) tile_counters[threadIdx.x] = 0;
+    clear_for_gemms(z);
+    if (u.y) {
+        // y rows of tokens with no routed slot: residual or zero (rare; a
+        // thread per token)
+        const int stride = gridDim.x * blockDim.x;
+        for (int t = blockIdx.x * blockDim.x + threadIdx.x; t < u.T; t += stride) {
+            bool any = false;
+            for (int j = 0; j < u.k; ++j) any |= (unsigned)__ldg(u.inv + (size_t)t * u.k + j) < (unsigned)rows;
+            if (any) continue;
+            uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(u.y) + (size_t)t * u.d);
+            const uint4* res = u.residual ? reinterpret_cast<const uint4*>(
+                                                static_cast<const __nv_bfloat16*>(u.residual) + (size_t)t * u.d)
+                                          : nullptr;
+            for (int v = 0; v < u.d / 8; ++v) dst[v] = res ? __ldg(res + v) : make_uint4(0u, 0u, 0u, 0u);
+        }
+    }
     const int nvec = d / 8;
     for (int r = blockIdx.x; r < rows; r += gridDim.x) {
         const int q = __ldg(perm + r);
@@ -296,42 +321,11 @@ gather_rows_kernel(const __nv_bfloat16* __restrict__ x, const int32_t* __restric
     }
 }
 
-// y[t, :] = (residual[t, :] +) sum_j obuf[inv[t*k + j], :]  (slot order; fp32
-// sum, one rounding to y's dtype).  A slot whose row id is out of range adds
-// nothing.
-template <bool BF16>
-__device__ __forceinline__ void combine_store(const float4& acc0, const void* residual, void* y, int t, int v,
-                                              int d) {
-    float4 acc = acc0;
-    if constexpr (BF16) {
-        if (residual) {
-            const uint2 rq = __ldg(reinterpret_cast<const uint2*>(
-                reinterpret_cast<const __nv_bfloat16*>(residual) + (size_t)t * d) + v);
-            acc.x = __uint_as_float(rq.x << 16) + acc.x;
-            acc.y = __uint_as_float(rq.x & 0xFFFF0000u) + acc.y;
-            acc.z = __uint_as_float(rq.y << 16) + acc.z;
-            acc.w = __uint_as_float(rq.y & 0xFFFF0000u) + acc.w;
-        }
-        __nv_bfloat162 lo = __floats2bfloat162_rn(acc.x, acc.y);
-        __nv_bfloat162 hi = __floats2bfloat162_rn(acc.z, acc.w);
-        uint2 out;
-        out.x = *reinterpret_cast<uint32_t*>(&lo);
-        out.y = *reinterpret_cast<uint32_t*>(&hi);
-        reinterpret_cast<uint2*>(reinterpret_cast<__nv_bfloat16*>(y) + (size_t)t * d)[v] = out;
-    } else {
-        if (residual) {
-            const float4 r = __ldg(reinterpret_cast<const float4*>(
-                reinterpret_cast<const float*>(residual) + (size_t)t * d) + v);
-            acc.x = r.x + acc.x; acc.y = r.y + acc.y; acc.z = r.z + acc.z; acc.w = r.w + acc.w;
-        }
-        reinterpret_cast<float4*>(reinterpret_cast<float*>(y) + (size_t)t * d)[v] = acc;
-    }
-}
-
-template <bool BF16>
+// fp32 path: y[t, :] = (residual[t, :] +) sum_j obuf[inv[t*k + j], :] (slot
+// order; one fp32 sum).  A slot whose row id is out of range adds nothing.
 __global__ void __launch_bounds__(kFlatThreads)
-combine_kernel(const float* __restrict__ obuf, const int32_t* __restrict__ inv,
-               const void* __restrict__ residual, int T, int d, int k, void* __restrict__ y) {
+combine_f32_kernel(const float* __restrict__ obuf, const int32_t* __restrict__ inv,
+                   const float* __restrict__ residual, int T, int d, int k, float* __restrict__ y) {
     pdl_wait();
     pdl_trigger();
     const int nvec = d / 4;
@@ -363,7 +357,13 @@ combine_kernel(const float* __restrict__ obuf, const int32_t* __restrict__ inv,
 #pragma unroll
             for (int u = 0; u < kUnroll; ++u) {
                 const int v = v0 + u * kFlatThreads;
-                if (v < nvec) combine_store<BF16>(acc[u], residual, y, t, v, d);
+                if (v >= nvec) continue;
+                float4 a = acc[u];
+                if (residual) {
+                    const float4 r = __ldg(reinterpret_cast<const float4*>(residual + (size_t)t * d) + v);
+                    a.x = r.x + a.x; a.y = r.y + a.y; a.z = r.z + a.z; a.w = r.w + a.w;
+                }
+                reinterpret_cast<float4*>(y + (size_t)t * d)[v] = a;
             }
         }
     }
@@ -453,7 +453,7 @@ cudaError_t launch_chunk_count_scan(const int32_t* idx, int n, int E, int32_t* c
 
 cudaError_t launch_chunk_scatter(const int32_t* idx, int n, int E, int k, const int32_t* chunk_base,
                                  int32_t* perm, int32_t* inv, const __nv_bfloat16* x, int d,
-                                 __nv_bfloat16* x_perm, int32_t* tile_counters, cudaStream_t s) {
+                                 __nv_bfloat16* x_perm, const ZeroArgs& z, cudaStream_t s) {
     const int nch = (n + kChunkA - 1) / kChunkA;
     // about two blocks per SM: split each chunk's row copies over `parts` blocks
     const int want = 2 * 148;
@@ -461,19 +461,18 @@ cudaError_t launch_chunk_scatter(const int32_t* idx, int n, int E, int k, const 
     parts = parts < 1 ? 1 : (parts > 8 ? 8 : parts);
     if (!x_perm) parts = 1;
     return launch_pdl(chunk_scatter_kernel, nch * parts, kScatThreads, 0, s, idx, n, E, nch, k, parts, chunk_base,
-                      perm, inv, x, d, x_perm, tile_counters);
+                      perm, inv, x, d, x_perm, z);
 }
 
 cudaError_t launch_gather_rows_bf16(const __nv_bfloat16* x, const int32_t* perm, int rows, int d,
-                                    int k, __nv_bfloat16* x_perm, int32_t* tile_counters, cudaStream_t s) {
-    return launch_pdl(gather_rows_kernel, flat_grid(rows), kFlatThreads, 0, s, x, perm, rows, d, k, x_perm,
-                      tile_counters);
+                                    int k, __nv_bfloat16* x_perm, const ZeroArgs& z, const UnroutedArgs& u,
+                                    cudaStream_t s) {
+    return launch_pdl(gather_rows_kernel, flat_grid(rows), kFlatThreads, 0, s, x, perm, rows, d, k, x_perm, z, u);
 }
 
-cudaError_t launch_combine(const float* obuf, const int32_t* inv, const void* residual, int T,
-                           int d, int k, bool bf16, void* y, cudaStream_t s) {
-    if (bf16) return launch_pdl(combine_kernel<true>, flat_grid(T), kFlatThreads, 0, s, obuf, inv, residual, T, d, k, y);
-    return launch_pdl(combine_kernel<false>, flat_grid(T), kFlatThreads, 0, s, obuf, inv, residual, T, d, k, y);
+cudaError_t launch_combine_f32(const float* obuf, const int32_t* inv, const float* residual, int T, int d, int k,
+                               float* y, cudaStream_t s) {
+    return launch_pdl(combine_f32_kernel, flat_grid(T), kFlatThreads, 0, s, obuf, inv, residual, T, d, k, y);
 }
 
 }  // namespace moe

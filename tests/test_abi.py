@@ -47,10 +47,12 @@ def _sz(T, d, f, E, k, dt):
     n = T * k
     a = lambda b: (b + 255) // 256 * 256  # noqa: E731
     esz = 2 if dt == moe.MOE_BF16 else 4
-    # idx, w, perm, inv; offsets; x_perm (bf16); h; obuf; 4 GEMM tile counters; chunk bases of the
-    # permutation (E per 64 assignments)
+    # idx, w, perm, inv; offsets; x_perm (bf16); h; obuf; 4 GEMM tile counters; the combine's arrival
+    # counters (one per token and 128 output columns); chunk bases of the permutation (E per 64
+    # assignments)
     return (a(4 * n) * 4 + a(4 * (E + 1)) + (a(n * d * 2) if dt == moe.MOE_BF16 else 0)
-            + a(n * f * esz) + a(n * d * 4) + a(4 * 4) + a(4 * E * ((n + 63) // 64)))
+            + a(n * f * esz) + a(n * d * 4) + a(4 * 4) + a(4 * T * ((d + 127) // 128))
+            + a(4 * E * ((n + 63) // 64)))
 
 
 @pytest.mark.parametrize("shape", [(4096, 4096, 14336, 8, 2), (32, 4096, 14336, 8, 2), (16, 64, 128, 8, 2),
@@ -174,3 +176,17 @@ def test_noalloc_token_limit_matches_its_documentation():
     cap = 32 << 20
     assert moe.moe_workspace_size(314, 4096, 14336, 8, 2, 0) <= cap
     assert moe.moe_workspace_size(315, 4096, 14336, 8, 2, 0) > cap
+
+
+def test_test_hooks_validate_their_values():
+    """moe_set_gemm_variant takes 0 (automatic) or one of each knob's
+    choices; anything else is refused and changes nothing."""
+    f = moe.lib.moe_set_gemm_variant
+    assert f(4, 0, 0, 0) == 1 and "outside its choices" in moe.moe_last_error_string()
+    assert f(-1, 0, 0, 0) == 1
+    assert f(0, 64, 0, 0) == 1
+    assert f(0, 0, 16, 0) == 1
+    assert f(0, 0, 0, 384) == 1
+    for args in [(1, 128, 32, 0), (2, 0, 0, 256), (3, 256, 128, 512), (0, 0, 0, 0)]:
+        assert f(*args) == 0
+    assert moe.lib.moe_set_wait_test(0, 0) == 0

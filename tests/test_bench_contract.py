@@ -19,7 +19,7 @@ def test_traffic_is_reported_only_for_the_captured_source(tmp_path, monkeypatch)
     rec = {"up_swiglu_gemm": {"source_sha256_16": h, "bytes_per_launch": 123}}
     (prof / "traffic.json").write_text(json.dumps(rec))
     assert bench.traffic_record("up_swiglu_gemm")["bytes_per_launch"] == 123
-    assert bench.traffic_record("down_scaled_gemm") is None
+    assert bench.traffic_record("down_combine_gemm") is None
     (src / "gemm_sm100.cu").write_text("// kernel v2\n")  # the kernel changed since the capture
     assert bench.traffic_record("up_swiglu_gemm") is None
 

@@ -27,7 +27,16 @@ import sparse_mixture_experts_06_b200 as moe  # noqa: E402
 @pytest.fixture(autouse=True)
 def no_device_errors():
     yield
+    moe.moe_set_gemm_variant()  # back to the automatic choice
     assert moe.moe_device_errors() == 0
+
+
+def force_variant(cta_group, bn="0", rb="0", wide=None):
+    """Tile variant by the test's labels: cta_group 1 / 2 / h (hybrid), up
+    tile width, token rows, and pair tiles 512 (wide = "1") or 256 columns."""
+    cg = {"1": 1, "2": 2, "h": 3}[cta_group]
+    cols = 0 if wide is None else (512 if wide == "1" else 256)
+    moe.moe_set_gemm_variant(cg, int(bn), int(rb), cols)
 
 
 def run_layer(t, k, residual=None):
@@ -224,17 +233,13 @@ GEMM_VARIANTS = [("1", "256", "128", "0"), ("1", "128", "128", "0"), ("1", "256"
 
 @pytest.mark.parametrize("variant", GEMM_VARIANTS, ids=lambda v: "cg%s-bn%s-rb%s-wide%s" % v)
 @pytest.mark.parametrize("shape", BF16_SHAPES, ids=lambda s: s.name)
-def test_layer_parity_every_token_bf16(shape, variant, monkeypatch):
+def test_layer_parity_every_token_bf16(shape, variant):
     """Every GEMM variant: single-CTA tiles of 128 or 32 token rows, CTA-pair
     tiles (256 rows, or 128 for an expert's short last block) 256 or 512
     columns wide, the hybrid (pairs on whole 256-row blocks, single CTAs on
     the rest), and 256- or 128-column up-projection tiles (pairs always use
     256-column MMAs)."""
-    cta_group, bn, rb, wide = variant
-    monkeypatch.setenv("MOE_GEMM_CTA_GROUP", cta_group)
-    monkeypatch.setenv("MOE_GEMM_BN", bn)
-    monkeypatch.setenv("MOE_GEMM_RB", rb)
-    monkeypatch.setenv("MOE_GEMM_WIDE", wide)
+    force_variant(*variant)
     rel, _ = full_check(shape)
     assert rel <= 1e-2
 
@@ -246,12 +251,11 @@ BLOCK_SIZES = [1, 64, 65, 128, 129, 200, 384, 385]
 
 
 @pytest.mark.parametrize("cta_group,wide", [("1", "0"), ("2", "0"), ("2", "1"), ("h", "0")])
-def test_expert_blocks_at_tile_edges(cta_group, wide, monkeypatch):
+def test_expert_blocks_at_tile_edges(cta_group, wide):
     """moe_expert_ffn on a routing built to give the experts the block sizes
     above (k = 1, tokens shuffled, arbitrary gate weights), ragged in both
     output widths (f = 320, d = 384), against the oracle on every token."""
-    monkeypatch.setenv("MOE_GEMM_CTA_GROUP", cta_group)
-    monkeypatch.setenv("MOE_GEMM_WIDE", wide)
+    force_variant(cta_group, wide=wide)
     E, d, f = len(BLOCK_SIZES), 384, 320
     T = sum(BLOCK_SIZES)
     s = synth.MoEShape("blocks", T, d, f, E, 1, "bf16")
@@ -364,6 +368,58 @@ def test_entry_points_agree_and_are_deterministic():
     moe.moe_release_workspace()
 
 
+@pytest.mark.parametrize("T", [100, 2304], ids=["one-block-permutation", "chunked-permutation"])
+def test_bf16_layer_runs_five_kernels(T):
+    """The bf16 layer is router, permutation (count/scan or one block), row
+    scatter or gather, up-projection GEMM and down-projection GEMM: the
+    combine runs in the down GEMM's epilogue, with no kernel of its own."""
+    s = synth.MoEShape("launches", T, 256, 512, 8, 2, "bf16")
+    t = device_inputs(s, 3)
+    ws = torch.empty(moe.moe_workspace_size(T, s.d, s.f, s.E, s.k, 0), dtype=torch.uint8, device="cuda")
+    run_layer(t, 2)  # set-up outside the record
+    torch.cuda.synchronize()
+    moe.moe_profile_select(None)
+    moe.moe_profile_enable(True)
+    y = moe.moe_layer_forward_ex(t["x"], t["Wg"], t["W1"], t["W3"], t["W2"], 2, workspace=ws)
+    torch.cuda.synchronize()
+    prof = moe.moe_profile_read()
+    moe.moe_profile_enable(False)
+    n = {name: cnt for name, (_, cnt) in prof.items()}
+    assert n["combine"] == 0 and n["down_combine_gemm"] == 1 and n["up_swiglu_gemm"] == 1
+    assert sum(n.values()) == 5, n
+    h = host_copy(t)
+    y_ref, _, _ = oracle_rows(h, 2, np.arange(T))
+    assert_close(to64(y), y_ref, "bf16")
+
+
+def test_unrouted_and_repeated_slots():
+    """moe_expert_ffn on a caller's routing with slots the permutation skips
+    (expert id -1: inv = -1, flagged) and tokens that name one expert twice.
+    Skipped slots add nothing, a token with no routed slot gets y = 0, and a
+    repeated expert adds both weighted copies; the oracle reads the same
+    routing (a slot with an id outside [0, E) contributes nothing there)."""
+    s = synth.MoEShape("unrouted", 300, 256, 384, 8, 2, "bf16")
+    t = device_inputs(s, 12)
+    rng = np.random.default_rng(3)
+    idx = np.stack([rng.choice(8, size=2, replace=False) for _ in range(s.T)]).astype(np.int32)
+    tok = np.arange(s.T)
+    idx[tok % 3 == 0, 1] = -1
+    idx[tok % 5 == 0, 0] = -1          # tokens 0, 15, 30, ...: no routed slot at all
+    idx[tok % 7 == 1, 1] = idx[tok % 7 == 1, 0]
+    w = rng.uniform(0.1, 0.9, size=(s.T, 2)).astype(np.float32)
+    idx_d, w_d = torch.from_numpy(idx).cuda(), torch.from_numpy(w).cuda()
+    off, perm, inv = moe.moe_permute(idx_d, s.E)
+    y = torch.full_like(t["x"], float("nan"))
+    moe.moe_expert_ffn(t["x"], t["W1"], t["W3"], t["W2"], off, perm, inv, w_d, y=y)
+    torch.cuda.synchronize()
+    assert moe.moe_device_errors() == 2  # MOE_DEVERR_BAD_EXPERT, from the permutation
+    h = host_copy(t)
+    y_ref, _, _ = oracle_rows(h, 2, tok, routing=(idx, w.astype(np.float64)))
+    got = to64(y)
+    assert_close(got, y_ref, "bf16")
+    assert (got[tok % 15 == 0] == 0).all()
+
+
 def test_zero_tokens_is_a_no_op():
     s = synth.MoEShape("z", 4, 64, 128, 8, 2, "bf16")
     t = device_inputs(s, 8)
@@ -419,12 +475,9 @@ def test_prefill_full_shape(mixtral_weights):
     ("decode", "h", "256", "128", "0"),
     ("prefill", "1", "128", "128", "0"), ("prefill", "2", "256", "128", "0"), ("prefill", "2", "256", "128", "1"),
     ("prefill", "1", "256", "128", "0"), ("prefill", "1", "256", "32", "0")])
-def test_full_shapes_other_gemm_variant(name, cta_group, bn, rb, wide, mixtral_weights, monkeypatch):
+def test_full_shapes_other_gemm_variant(name, cta_group, bn, rb, wide, mixtral_weights):
     """Variants the size heuristics do not pick, at the full shapes."""
-    monkeypatch.setenv("MOE_GEMM_CTA_GROUP", cta_group)
-    monkeypatch.setenv("MOE_GEMM_BN", bn)
-    monkeypatch.setenv("MOE_GEMM_RB", rb)
-    monkeypatch.setenv("MOE_GEMM_WIDE", wide)
+    force_variant(cta_group, bn, rb, wide)
     big_check(name, mixtral_weights, None if name == "decode" else 256)
 
 

@@ -81,6 +81,31 @@ def test_router_logits_exact_sum_within_bound():
     assert float(bound.max()) < 1e-12
 
 
+def test_logit_sum_bound_is_gamma_d_minus_1_times_the_absolute_sum():
+    """The near-tie bound against Higham's gamma_{d-1} * sum_i |x_i Wg[e, i]|
+    (Accuracy and Stability of Numerical Algorithms, §4.2), worked by hand in
+    exact rationals for d = 3: n = d - 1 = 2 and gamma_2 = 2u / (1 - 2u),
+    u = 2^-53.  Products (x, Wg rows below):
+      token 0, expert 0: |1.5*0.5| + |-2*3| + |0.25*-4|   = 0.75 + 6 + 1     = 31/4
+      token 0, expert 1: |1.5*-1| + |-2*0.125| + |0.25*2| = 1.5 + 0.25 + 0.5 = 9/4
+      token 1, expert 0: |0.5*0.5| + |0*3| + |-8*-4|      = 0.25 + 0 + 32    = 129/4
+      token 1, expert 1: |0.5*-1| + |0*0.125| + |-8*2|    = 0.5 + 0 + 16     = 33/2
+    A wrong n (d instead of d - 1), a missing absolute value, a transposed
+    operand or a slip of the unit roundoff all miss by far more than the
+    few ulps of the fp64 evaluation allowed here."""
+    x = np.array([[1.5, -2.0, 0.25], [0.5, 0.0, -8.0]])
+    Wg = np.array([[0.5, 3.0, -4.0], [-1.0, 0.125, 2.0]])
+    u = Fraction(1, 2 ** 53)
+    gamma2 = 2 * u / (1 - 2 * u)
+    sums = [[Fraction(31, 4), Fraction(9, 4)], [Fraction(129, 4), Fraction(33, 2)]]
+    got = oracle.logit_sum_bound(x, Wg)
+    assert got.shape == (2, 2)
+    for t in range(2):
+        for e in range(2):
+            exact = gamma2 * sums[t][e]
+            assert abs(Fraction(float(got[t, e])) - exact) <= exact * Fraction(1, 2 ** 50), (t, e)
+
+
 def test_router_logits_orientation():
     """Wg is stored (n_experts, dim): logit e uses row e.  A transposed or
     mis-indexed router fails on a one-hot x."""

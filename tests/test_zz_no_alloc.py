@@ -23,8 +23,12 @@ import sparse_mixture_experts_06_b200 as moe  # noqa: E402
     synth.CONFIGS["decode"],
 ], ids=["small", "mixtral-decode"])
 def test_noalloc_matches_the_regular_entry_point_twice(shape):
+    """Two calls in a row (different tokens and weights): each equals the
+    regular entry point within the bf16 bound, and the first is also checked
+    on its own against the fp64 oracle (every token, expert indices exact)."""
     if not torch.cuda.is_available():
         pytest.skip("no CUDA device")
+    from tests.gpu_util import assert_close, check_routing, f64, host_copy, oracle_rows
     from synth.device import device_inputs
     for call, seed in enumerate((11, 12)):   # two calls in a row, different tokens and weights
         t = device_inputs(shape, seed)
@@ -36,6 +40,12 @@ def test_noalloc_matches_the_regular_entry_point_twice(shape):
         b = y_ref.float().double().cpu().numpy()
         assert np.isfinite(a).all(), "call %d left unwritten outputs" % call
         assert np.abs(a - b).max() <= 1e-2 * np.abs(b).max(), "call %d differs" % call
+        if call == 0:
+            idx, w = moe.moe_router_topk(t["x"], t["Wg"], shape.k)
+            h = host_copy(t)
+            check_routing(idx.cpu().numpy(), w.cpu().numpy(), f64(h["x"]), f64(h["Wg"]), shape.k)
+            y_o, _, _ = oracle_rows(h, shape.k, np.arange(shape.T))
+            assert_close(a, y_o, "bf16", "noalloc y")
     assert moe.moe_device_errors() == 0
 
 
