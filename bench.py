@@ -260,7 +260,7 @@ def timed_loop(step, steps, flush, stream):
     return evs
 
 
-def bench_workload(args, s, rank, world, device, dist, extras_for_decode=False):
+def bench_workload(args, s, rank, world, device, dist, extras_for_decode=False, record_up=True):
     import torch
     import sparse_mixture_experts_06_b200 as moe
     t = make_inputs(s, rank, device)
@@ -279,10 +279,13 @@ def bench_workload(args, s, rank, world, device, dist, extras_for_decode=False):
         dist.barrier()
     torch.cuda.synchronize(device)
     # inside the timed steps only the up-projection GEMM (the roofline's kernel)
-    # is bracketed by events: events between kernels serialise them and cost
-    # ~50 us per prefill step
-    moe.moe_profile_select(["up_swiglu_gemm"])
-    moe.moe_profile_enable(True)
+    # is bracketed by events: events between kernels serialise them (they undo
+    # the programmatic-launch overlap with its neighbours) and cost ~50 us per
+    # prefill step if every kernel had them; record_up=False times the steps
+    # with no event inside at all
+    if record_up:
+        moe.moe_profile_select(["up_swiglu_gemm"])
+        moe.moe_profile_enable(True)
     props = torch.cuda.get_device_properties(device)
     bus = "%04x:%02x:%02x" % (getattr(props, "pci_domain_id", 0), getattr(props, "pci_bus_id", 0),
                               getattr(props, "pci_device_id", 0)) if hasattr(props, "pci_bus_id") else ""
@@ -297,7 +300,7 @@ def bench_workload(args, s, rank, world, device, dist, extras_for_decode=False):
     torch.cuda.synchronize(device)
     clocks = sampler.stop() if sampler else None
     moe.moe_profile_enable(False)
-    prof_up = moe.moe_profile_read()
+    prof_up = moe.moe_profile_read() if record_up else None
     step_ms = [a.elapsed_time(b) for a, b in evs]
     total_ms = max_over_ranks(sum(step_ms), dist, device)
     # per-stage breakdown: a separate, untimed pass with every stage recorded
@@ -593,16 +596,19 @@ def main():
     if not args.no_extras and args.workload == "prefill":
         d = synth.CONFIGS["decode"]
         dargs = argparse.Namespace(**vars(args))
-        dargs.steps = max(20, min(200, K))
-        rd = bench_workload(dargs, d, rank, world, device, dist, extras_for_decode=True)
+        dargs.steps = 200  # ~0.1 s of decode steps whatever K is: a stable mean
+        # the timed decode steps carry no events inside (the layer as a caller
+        # runs it); the GEMMs' rates come from the breakdown pass
+        rd = bench_workload(dargs, d, rank, world, device, dist, extras_for_decode=True, record_up=False)
         p, dnb = rd["prof"], rd["breakdown_steps"]
         dms = rd["total_ms"] / dargs.steps
         counts = None
         wbytes = 3.0 * d.E * d.d * d.f * 2  # all 8 experts are touched at T=32 with near-uniform routing
-        ups, upn = rd["prof_up"]["up_swiglu_gemm"]
+        ups, upn = p["up_swiglu_gemm"]
         dns, dnn = p["down_combine_gemm"]
         gms = graph_step_ms(rd, d, device, dargs.steps)
         line["decode"] = {"workload": workload_desc(d, world)["workload"], "ms_per_step": dms,
+                          "ms_per_step_median": statistics.median(rd["step_ms"]), "steps": dargs.steps,
                           "ms_per_step_cuda_graph": gms,
                           "cuda_graph_note": "one captured layer replayed back to back; no L2 flush (the 2.82 GB "
                                              "of weights exceed L2)",
@@ -613,6 +619,7 @@ def main():
                           "frac_of_hbm": wbytes / (dms * 1e-3) / 1e9 / pk["hbm_gbs"],
                           "up_gemm_GBps": (2.0 * d.E * d.f * d.d * 2) / (ups / upn * 1e-3) / 1e9,
                           "down_gemm_GBps": (1.0 * d.E * d.f * d.d * 2) / (dns / dnn * 1e-3) / 1e9,
+                          "gemm_rates_note": "from the breakdown pass (events around every kernel)",
                           "stages_ms_per_step": {k: round(v[0] / dnb, 4) for k, v in p.items() if v[1]},
                           "device_error_flags": rd["deverr"]}
         del rd, counts
@@ -620,7 +627,7 @@ def main():
         sk = synth.CONFIGS["skewed"]
         sargs = argparse.Namespace(**vars(args))
         sargs.steps = max(10, min(60, K))
-        rs = bench_workload(sargs, sk, rank, world, device, dist, extras_for_decode=True)
+        rs = bench_workload(sargs, sk, rank, world, device, dist, extras_for_decode=True, record_up=False)
         sms = rs["total_ms"] / sargs.steps
         line["skewed"] = {"workload": workload_desc(sk, world)["workload"] + ", Zipf-shaped load (hottest expert 35%)",
                           "ms_per_step": sms, "tokens_per_s": world * sk.T / (sms * 1e-3),

@@ -75,6 +75,7 @@ constexpr int TMEM_COLS = 512;                 // 2 accumulators x 256 fp32 colu
 constexpr unsigned long long kWaitLimitNs = 4000000000ull;  // default bound of a pipeline wait
 constexpr unsigned long long kDrainLimitNs = 1000000000ull;  // bound of the exit drain of issued MMAs
 constexpr unsigned long long kQuiesceNs = 100000ull;         // after an abort: copies in flight land
+constexpr long long kPrefetchBytes = 64ll << 20;              // weights warmed in L2 ahead of a decode GEMM
 
 
 enum Mode { kUp = 0, kDown = 1 };
@@ -101,6 +102,7 @@ struct KParams {
     int* tile_counter;       // next tile to hand out; zero at launch (the row gather zeroes it)
     unsigned long long wait_limit_ns;  // bound of every pipeline wait
     int stall_test;          // failure-detection test: the epilogue waits on a barrier nothing completes
+    int prefetch_kblocks;    // weight-streaming tiles: k-blocks of the first weight tile warmed in L2
 };
 
 // Row ranges: all rows of each expert; only its whole 256-row blocks; or
@@ -149,6 +151,14 @@ __device__ __forceinline__ bool mbar_try_wait_cluster(uint32_t bar, uint32_t par
         : "r"(bar), "r"(parity)
         : "memory");
     return ok != 0;
+}
+
+// Bulk tensor prefetch of one box into L2 (no shared memory, no barrier).
+__device__ __forceinline__ void tma_prefetch_2d(const CUtensorMap* map, int c0, int c1) {
+    asm volatile("cp.async.bulk.prefetch.tensor.2d.L2.global.tile [%0, {%1, %2}];" ::"l"(
+                     reinterpret_cast<uint64_t>(map)),
+                 "r"(c0), "r"(c1)
+                 : "memory");
 }
 
 __device__ __forceinline__ void mbar_arrive_expect_tx(uint32_t bar, uint32_t bytes) {
@@ -635,8 +645,28 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
             asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
         }
     }
-    // the set-up above overlaps the previous kernel's tail; offsets, the A
-    // rows and the tile counter are earlier kernels' outputs
+    // Weight-streaming tiles (32 token rows, the decode case): warm L2 with
+    // the first k-blocks of the weight tile this CTA most likely takes first,
+    // while the routing kernels still run.  The tile is a guess (number
+    // blockIdx.x with one row block per expert; the first wave takes tiles
+    // 0 .. grid-1 in some order); no kernel this one waits for writes the
+    // weights, and a wrong guess costs only bandwidth.
+    if constexpr (CG == 1 && RB == 32) {
+        if (warp == 0 && lane == 0 && p.prefetch_kblocks > 0) {
+            const int e = (int)blockIdx.x / p.n_tiles, nb = (int)blockIdx.x % p.n_tiles;
+            if (e < p.E) {
+                const int r0 = e * p.b_rows_per_expert + nb * (MODE == kUp ? BN / 2 : BN);
+                const int r1 = (MODE == kUp) ? r0 : r0 + BN / 2;
+                const int nk = min(p.prefetch_kblocks, (p.Kdim + BK - 1) / BK);
+                for (int kb = 0; kb < nk; ++kb) {
+                    tma_prefetch_2d(&tmB0, kb * BK, r0);
+                    tma_prefetch_2d(&tmB1, kb * BK, r1);
+                }
+            }
+        }
+    }
+    // the set-up above overlaps the previous kernels; offsets, the A rows and
+    // the tile counter are earlier kernels' outputs
     pdl_wait();
     pdl_trigger();
     if (threadIdx.x < p.E) {
@@ -1122,6 +1152,46 @@ struct GemmMaps {
     CUtensorMap A, A32, A64, B0, B1, B0p, B1p, Out;
 };
 
+// Tensor maps of recent calls.  A map is a pure function of its pointer,
+// shape and box, so a call whose pointers and sizes equal an earlier one's
+// reuses that call's maps (a serving loop or a layer stack repeats them)
+// instead of encoding 5-8 maps per GEMM on the host.
+struct MapKey {
+    int mode, bn;
+    const void* p[4];
+    int rows, d, f, E;
+    bool operator==(const MapKey& o) const {
+        return mode == o.mode && bn == o.bn && p[0] == o.p[0] && p[1] == o.p[1] && p[2] == o.p[2] &&
+               p[3] == o.p[3] && rows == o.rows && d == o.d && f == o.f && E == o.E;
+    }
+};
+constexpr int kMapCacheSlots = 16;
+struct MapCache {
+    std::mutex mu;
+    MapKey key[kMapCacheSlots];
+    GemmMaps maps[kMapCacheSlots];
+    int used = 0, next = 0;
+} g_map_cache;
+
+bool map_cache_get(const MapKey& k, GemmMaps* out) {
+    std::lock_guard<std::mutex> lock(g_map_cache.mu);
+    for (int i = 0; i < g_map_cache.used; ++i)
+        if (g_map_cache.key[i] == k) {
+            *out = g_map_cache.maps[i];
+            return true;
+        }
+    return false;
+}
+
+void map_cache_put(const MapKey& k, const GemmMaps& m) {
+    std::lock_guard<std::mutex> lock(g_map_cache.mu);
+    const int i = g_map_cache.next;
+    g_map_cache.key[i] = k;
+    g_map_cache.maps[i] = m;
+    g_map_cache.next = (i + 1) % kMapCacheSlots;
+    if (g_map_cache.used < kMapCacheSlots) ++g_map_cache.used;
+}
+
 template <int MODE, int CG, int BN, int RB, int NH = 1>
 cudaError_t launch_gemm(const GroupedGemmArgs& a, const CUtensorMap& mA, const CUtensorMap& mAs,
                         const CUtensorMap& mB0, const CUtensorMap& mB1, const CUtensorMap& mOut, const KParams& p0,
@@ -1166,6 +1236,8 @@ cudaError_t launch_gemm(const GroupedGemmArgs& a, const CUtensorMap& mA, const C
     const long long ub = (long long)p.n_tiles * ((a.rows + C::kTileRows - 1) / C::kTileRows + a.E);
     const int grid_units = (int)(ub < units ? ub : units);
     if (grid_units <= 0) return cudaSuccess;
+    // L2 warm-up of weight-streaming tiles: about kPrefetchBytes over the grid
+    p.prefetch_kblocks = (CG == 1 && RB == 32) ? (int)(kPrefetchBytes / ((long long)grid_units * BN * BK * 2)) : 0;
     cfg.gridDim = dim3(grid_units * CG);
     set_pdl(attr[cfg.numAttrs++]);  // after the occupancy query, which takes the cluster attribute only
     return cudaLaunchKernelEx(&cfg, grouped_gemm_kernel<MODE, CG, BN, RB, NH>, mA, mAs, mB0, mB1, mOut, p);
@@ -1279,15 +1351,19 @@ cudaError_t launch_up_swiglu(const GroupedGemmArgs& a, const __nv_bfloat16* x_pe
     // pairs and the hybrid use 256-column tiles whatever the forced width
     const int bn = choose_cta_group(a, kUp) == 1 ? choose_up_bn(a) : 256;
     GemmMaps m;
-    if (!make_map(&m.A, x_perm, (uint64_t)a.rows, (uint64_t)a.d, BM) ||
-        !make_map(&m.A32, x_perm, (uint64_t)a.rows, (uint64_t)a.d, 32) ||
-        !make_map(&m.A64, x_perm, (uint64_t)a.rows, (uint64_t)a.d, 64) ||
-        !make_map(&m.B0, W1, (uint64_t)a.E * a.f, (uint64_t)a.d, bn / 2) ||
-        !make_map(&m.B1, W3, (uint64_t)a.E * a.f, (uint64_t)a.d, bn / 2) ||
-        !make_map(&m.B0p, W1, (uint64_t)a.E * a.f, (uint64_t)a.d, 64) ||
-        !make_map(&m.B1p, W3, (uint64_t)a.E * a.f, (uint64_t)a.d, 64) ||
-        !make_map(&m.Out, h, (uint64_t)a.rows, (uint64_t)a.f, 32))
-        return cudaErrorInvalidValue;
+    const MapKey key{kUp, bn, {x_perm, W1, W3, h}, a.rows, a.d, a.f, a.E};
+    if (!map_cache_get(key, &m)) {
+        if (!make_map(&m.A, x_perm, (uint64_t)a.rows, (uint64_t)a.d, BM) ||
+            !make_map(&m.A32, x_perm, (uint64_t)a.rows, (uint64_t)a.d, 32) ||
+            !make_map(&m.A64, x_perm, (uint64_t)a.rows, (uint64_t)a.d, 64) ||
+            !make_map(&m.B0, W1, (uint64_t)a.E * a.f, (uint64_t)a.d, bn / 2) ||
+            !make_map(&m.B1, W3, (uint64_t)a.E * a.f, (uint64_t)a.d, bn / 2) ||
+            !make_map(&m.B0p, W1, (uint64_t)a.E * a.f, (uint64_t)a.d, 64) ||
+            !make_map(&m.B1p, W3, (uint64_t)a.E * a.f, (uint64_t)a.d, 64) ||
+            !make_map(&m.Out, h, (uint64_t)a.rows, (uint64_t)a.f, 32))
+            return cudaErrorInvalidValue;
+        map_cache_put(key, m);
+    }
     KParams p{};
     p.offsets = a.offsets; p.E = a.E; p.n_out = a.f; p.Kdim = a.d;
     p.n_tiles = (a.f + bn / 2 - 1) / (bn / 2); p.b_rows_per_expert = a.f; p.h = h; p.rows = a.rows;
@@ -1298,15 +1374,19 @@ cudaError_t launch_up_swiglu(const GroupedGemmArgs& a, const __nv_bfloat16* x_pe
 
 cudaError_t launch_down_combine(const GroupedGemmArgs& a, const DownCombineArgs& c, cudaStream_t s) {
     GemmMaps m;
-    if (!make_map(&m.A, c.h, (uint64_t)a.rows, (uint64_t)a.f, BM) ||
-        !make_map(&m.A32, c.h, (uint64_t)a.rows, (uint64_t)a.f, 32) ||
-        !make_map(&m.A64, c.h, (uint64_t)a.rows, (uint64_t)a.f, 64) ||
-        !make_map(&m.B0, c.W2, (uint64_t)a.E * a.d, (uint64_t)a.f, 128) ||
-        !make_map(&m.Out, c.obuf, (uint64_t)a.rows, (uint64_t)a.d, 32, true))
-        return cudaErrorInvalidValue;
-    m.B1 = m.B0;
-    m.B0p = m.B0;
-    m.B1p = m.B0;
+    const MapKey key{kDown, 256, {c.h, c.W2, c.obuf, nullptr}, a.rows, a.d, a.f, a.E};
+    if (!map_cache_get(key, &m)) {
+        if (!make_map(&m.A, c.h, (uint64_t)a.rows, (uint64_t)a.f, BM) ||
+            !make_map(&m.A32, c.h, (uint64_t)a.rows, (uint64_t)a.f, 32) ||
+            !make_map(&m.A64, c.h, (uint64_t)a.rows, (uint64_t)a.f, 64) ||
+            !make_map(&m.B0, c.W2, (uint64_t)a.E * a.d, (uint64_t)a.f, 128) ||
+            !make_map(&m.Out, c.obuf, (uint64_t)a.rows, (uint64_t)a.d, 32, true))
+            return cudaErrorInvalidValue;
+        m.B1 = m.B0;
+        m.B0p = m.B0;
+        m.B1p = m.B0;
+        map_cache_put(key, m);
+    }
     KParams p{};
     p.offsets = a.offsets; p.E = a.E; p.n_out = a.d; p.Kdim = a.f;
     p.n_tiles = (a.d + 255) / 256; p.b_rows_per_expert = a.d;

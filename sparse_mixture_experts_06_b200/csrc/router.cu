@@ -26,11 +26,11 @@
 // Reduction (fixed order, so the result is deterministic): each warp's MMAs
 // alternate between two accumulators (even and odd m) that are added at the
 // end; CTA 0 of the cluster adds the CTAs' partial logits in rank order
-// through distributed shared memory, then one thread per token does the
-// top-k (k rounds of a strict-greater arg-max in increasing expert order, so
-// an exact tie keeps the lower index; slot 0 = largest) and the fp32 softmax
-// of the kept logits.  The split changes the summation order but not the
-// rule: logits are fp64 sums of exact products.
+// through distributed shared memory, then selects the top-k with warp
+// shuffles (a segment of lanes per token; k rounds of arg-max, an exact tie
+// keeps the lower index; slot 0 = largest) and computes the fp32 softmax of
+// the kept logits.  The split changes the summation order but not the rule:
+// logits are fp64 sums of exact products.
 
 #include <cooperative_groups.h>
 
@@ -108,8 +108,8 @@ __global__ void __launch_bounds__(kWarps * 32, BF16 ? 4 : 2)  // bf16: 64 regist
 router_topk_kernel(const void* __restrict__ x, const void* __restrict__ Wg, int T, int d, int E, int k,
                    int32_t* __restrict__ idx_out, float* __restrict__ w_out) {
     extern __shared__ __align__(16) unsigned char smem_raw[];
+    pdl_trigger();  // successors may launch and set up now; they wait for this grid before reading
     pdl_wait();     // x may be the previous kernel's output (a layer stack)
-    pdl_trigger();
     double* wfrag = reinterpret_cast<double*>(smem_raw);  // [kChunks][8][32]
     double* part = wfrag + kFragDoubles;                  // [kTokBlock][E]
     cg::cluster_group cluster = cg::this_cluster();
@@ -199,34 +199,61 @@ router_topk_kernel(const void* __restrict__ x, const void* __restrict__ Wg, int 
     cluster.sync();  // peers keep their shared memory until CTA 0 has read it
     if (rank != 0) return;
     __syncthreads();
-    for (int tl = threadIdx.x; tl < kTokBlock; tl += kWarps * 32) {
+    // Top-k, warp-level: a segment of S lanes per token (S = E rounded up to
+    // a power of two, at most 32; lane sl of the segment holds experts sl,
+    // sl + S), so a warp selects for 32 / S tokens at once.  Each of the k
+    // rounds takes the segment's arg-max over the experts not yet taken with
+    // butterfly shuffles; a larger logit wins, an equal one goes to the lower
+    // expert index, so slot 0 holds the largest logit and ties keep the lower
+    // index.  The segment's first lane writes the index and the fp32 softmax
+    // numerator exp(l_j - l_0) of each slot, then divides them by their
+    // slot-ordered sum.
+    const int S = E >= 32 ? 32 : (E <= 1 ? 1 : 1 << (32 - __clz(E - 1)));
+    const int per = (E + S - 1) / S;  // experts per lane: 1, or 2 when E > 32
+    const int tpw = 32 / S;           // tokens per warp per pass
+    const int sl = lane & (S - 1);
+    for (int base = warp * tpw; base < kTokBlock; base += kWarps * tpw) {
+        const int tl = base + lane / S;
         const int t = tok0 + tl;
-        if (t >= T) continue;
-        const double* lg = wfrag + (size_t)tl * E;
-        // k rounds of arg-max; indices are written as they are found and the
-        // fp32 softmax numerators exp(l_j - l_0) are parked in w_out, then
-        // divided by their slot-ordered sum (any k <= E, no per-k arrays)
-        uint64_t taken = 0;
-        double l0 = 0.0;
-        float sum = 0.f;
+        const bool live = t < T;  // uniform in a segment
+        double v[2];
+        bool open[2];
+#pragma unroll
+        for (int i = 0; i < 2; ++i) {
+            const int e = sl + i * S;
+            open[i] = live && i < per && e < E;
+            v[i] = open[i] ? wfrag[(size_t)tl * E + e] : 0.0;
+        }
         int32_t* io = idx_out + (size_t)t * k;
         float* wo = w_out + (size_t)t * k;
+        double l0 = 0.0;
+        float sum = 0.f;
         for (int j = 0; j < k; ++j) {
-            int bi = -1;
-            double best = 0.0;
-            for (int e = 0; e < E; ++e) {
-                if ((taken >> e) & 1ull) continue;
-                const double v = lg[e];
-                if (bi < 0 || v > best) { best = v; bi = e; }
+            // this lane's best open expert (its lower index first)
+            int be = -1;
+            double bv = 0.0;
+#pragma unroll
+            for (int i = 0; i < 2; ++i)
+                if (open[i] && (be < 0 || v[i] > bv)) { bv = v[i]; be = sl + i * S; }
+            // the segment's arg-max
+            for (int off = S >> 1; off > 0; off >>= 1) {
+                const double ov = __shfl_xor_sync(0xffffffffu, bv, off, S);
+                const int oe = __shfl_xor_sync(0xffffffffu, be, off, S);
+                if (oe >= 0 && (be < 0 || ov > bv || (ov == bv && oe < be))) { bv = ov; be = oe; }
             }
-            taken |= 1ull << bi;
-            if (j == 0) l0 = best;
-            const float ex = expf((float)(best - l0));
-            io[j] = bi;
-            wo[j] = ex;
-            sum += ex;
+            if (be >= 0 && (be & (S - 1)) == sl) {
+                if (be < S) open[0] = false; else open[1] = false;
+            }
+            if (live && sl == 0) {
+                if (j == 0) l0 = bv;
+                const float ex = expf((float)(bv - l0));
+                io[j] = be;
+                wo[j] = ex;
+                sum += ex;
+            }
         }
-        for (int j = 0; j < k; ++j) wo[j] = wo[j] / sum;
+        if (live && sl == 0)
+            for (int j = 0; j < k; ++j) wo[j] = wo[j] / sum;
     }
 }
 
