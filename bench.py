@@ -52,8 +52,9 @@ def parse():
     ap.add_argument("--no-extras", action="store_true", help="skip the decode line and the CPU baseline")
     ap.add_argument("--cpu-sample", type=int, default=4096,
                     help="tokens in the oracle's timed CPU-baseline sample (default: the whole prefill batch)")
-    ap.add_argument("--ref-sample", type=int, default=128,
-                    help="tokens per step of --impl reference (keeps --steps K --warmup W within minutes)")
+    ap.add_argument("--ref-sample", type=int, default=4096,
+                    help="tokens per step of --impl reference: by default the whole prefill batch, the same "
+                         "sample as the cpu_baseline leg (~4 s per step on 16 cores)")
     ap.add_argument("--e2e-chunks", type=int, default=1,
                     help="pieces the end-to-end leg pipelines host copies and compute in")
     ap.add_argument("--gemm-vs-cublas", action="store_true",
@@ -228,7 +229,9 @@ def run_reference(args):
             "data": "synthetic", "config": workload_desc(s, 1),
             "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": threads, "kind": "oracle",
                              "sample": "%d random tokens of the %s workload per step (router, top-k, both "
-                                       "experts, combine in fp64)" % (min(n, s.T), s.name)},
+                                       "experts, combine in fp64; the same sample size as the cpu_baseline "
+                                       "leg of the default run, so the two throughputs agree)"
+                                       % (min(n, s.T), s.name)},
             "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
     return 0
@@ -250,17 +253,21 @@ def make_inputs(s, rank, device):
 
 
 def timed_loop(step, steps, flush, stream):
+    """K steps, each between two events on the launching stream; with `flush`
+    (a buffer larger than L2) written before each step, outside its events;
+    with flush=None the steps run back to back (inputs larger than L2)."""
     import torch
     evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
     for a, b in evs:
-        flush.zero_()
+        if flush is not None:
+            flush.zero_()
         a.record(stream)
         step()
         b.record(stream)
     return evs
 
 
-def bench_workload(args, s, rank, world, device, dist, extras_for_decode=False, record_up=True):
+def bench_workload(args, s, rank, world, device, dist, extras_for_decode=False, record_up=True, l2_flush=True):
     import torch
     import sparse_mixture_experts_06_b200 as moe
     t = make_inputs(s, rank, device)
@@ -293,12 +300,18 @@ def bench_workload(args, s, rank, world, device, dist, extras_for_decode=False, 
     if sampler:
         sampler.start()
         time.sleep(0.5)
-    evs = timed_loop(step, args.steps, flush, stream)
+    evs = timed_loop(step, args.steps, flush if l2_flush else None, stream)
     torch.cuda.synchronize(device)
     if dist is not None:
         dist.barrier()
     torch.cuda.synchronize(device)
     clocks = sampler.stop() if sampler else None
+    flushed_ms = None
+    if not l2_flush:
+        # the same steps with the L2 flush between them, for comparison
+        fe = timed_loop(step, args.steps, flush, stream)
+        torch.cuda.synchronize(device)
+        flushed_ms = [a.elapsed_time(b) for a, b in fe]
     moe.moe_profile_enable(False)
     prof_up = moe.moe_profile_read() if record_up else None
     step_ms = [a.elapsed_time(b) for a, b in evs]
@@ -313,6 +326,7 @@ def bench_workload(args, s, rank, world, device, dist, extras_for_decode=False, 
     prof = moe.moe_profile_read()
     deverr = moe.moe_device_errors()
     res = {"t": t, "y": y, "ws": ws, "total_ms": total_ms, "step_ms": step_ms, "prof_up": prof_up, "prof": prof,
+           "flushed_step_ms": flushed_ms,
            "breakdown_steps": nb, "clocks": clocks, "deverr": deverr, "stream": stream}
     return res
 
@@ -599,7 +613,8 @@ def main():
         dargs.steps = 200  # ~0.1 s of decode steps whatever K is: a stable mean
         # the timed decode steps carry no events inside (the layer as a caller
         # runs it); the GEMMs' rates come from the breakdown pass
-        rd = bench_workload(dargs, d, rank, world, device, dist, extras_for_decode=True, record_up=False)
+        rd = bench_workload(dargs, d, rank, world, device, dist, extras_for_decode=True, record_up=False,
+                            l2_flush=False)
         p, dnb = rd["prof"], rd["breakdown_steps"]
         dms = rd["total_ms"] / dargs.steps
         counts = None
@@ -607,8 +622,13 @@ def main():
         ups, upn = p["up_swiglu_gemm"]
         dns, dnn = p["down_combine_gemm"]
         gms = graph_step_ms(rd, d, device, dargs.steps)
+        fl = rd["flushed_step_ms"]
         line["decode"] = {"workload": workload_desc(d, world)["workload"], "ms_per_step": dms,
                           "ms_per_step_median": statistics.median(rd["step_ms"]), "steps": dargs.steps,
+                          "l2": "steps back to back: the 2.82 GB of expert weights exceed the 126 MB L2, and each "
+                                "step streams all of them, so no step finds another's weights in L2",
+                          "ms_per_step_l2_flushed": sum(fl) / len(fl),
+                          "frac_of_hbm_l2_flushed": wbytes / (sum(fl) / len(fl) * 1e-3) / 1e9 / pk["hbm_gbs"],
                           "ms_per_step_cuda_graph": gms,
                           "cuda_graph_note": "one captured layer replayed back to back; no L2 flush (the 2.82 GB "
                                              "of weights exceed L2)",

@@ -75,7 +75,6 @@ constexpr int TMEM_COLS = 512;                 // 2 accumulators x 256 fp32 colu
 constexpr unsigned long long kWaitLimitNs = 4000000000ull;  // default bound of a pipeline wait
 constexpr unsigned long long kDrainLimitNs = 1000000000ull;  // bound of the exit drain of issued MMAs
 constexpr unsigned long long kQuiesceNs = 100000ull;         // after an abort: copies in flight land
-constexpr long long kPrefetchBytes = 64ll << 20;              // weights warmed in L2 ahead of a decode GEMM
 
 
 enum Mode { kUp = 0, kDown = 1 };
@@ -102,7 +101,6 @@ struct KParams {
     int* tile_counter;       // next tile to hand out; zero at launch (the row gather zeroes it)
     unsigned long long wait_limit_ns;  // bound of every pipeline wait
     int stall_test;          // failure-detection test: the epilogue waits on a barrier nothing completes
-    int prefetch_kblocks;    // weight-streaming tiles: k-blocks of the first weight tile warmed in L2
 };
 
 // Row ranges: all rows of each expert; only its whole 256-row blocks; or
@@ -151,14 +149,6 @@ __device__ __forceinline__ bool mbar_try_wait_cluster(uint32_t bar, uint32_t par
         : "r"(bar), "r"(parity)
         : "memory");
     return ok != 0;
-}
-
-// Bulk tensor prefetch of one box into L2 (no shared memory, no barrier).
-__device__ __forceinline__ void tma_prefetch_2d(const CUtensorMap* map, int c0, int c1) {
-    asm volatile("cp.async.bulk.prefetch.tensor.2d.L2.global.tile [%0, {%1, %2}];" ::"l"(
-                     reinterpret_cast<uint64_t>(map)),
-                 "r"(c0), "r"(c1)
-                 : "memory");
 }
 
 __device__ __forceinline__ void mbar_arrive_expect_tx(uint32_t bar, uint32_t bytes) {
@@ -509,6 +499,13 @@ struct Sched {
 
 __device__ __forceinline__ float4 ldcg_f4(const float* a) { return __ldcg(reinterpret_cast<const float4*>(a)); }
 
+// Drops a 128-byte L2 line without writing it back (its contents become
+// undefined): a parked row is dead once the last arrival has read it, so a
+// line still in L2 then never reaches DRAM.
+__device__ __forceinline__ void discard_l2_line(const void* a) {
+    asm volatile("discard.global.L2 [%0], 128;" ::"l"(a) : "memory");
+}
+
 // a = v for the first routed slot, a += v after it (slot order)
 __device__ __forceinline__ void add_slot(float4& a, const float4& v, bool& first) {
     if (first) {
@@ -579,6 +576,19 @@ __device__ __forceinline__ void combine_group(unsigned m, int t, int rr0, int rr
             out.y = pack_bf16x2(a.z, a.w);
             *reinterpret_cast<uint2*>(p.y + (size_t)tb[b] * d + c) = out;
         }
+        // the parked rows of slots 0 and 1 are dead: lanes 0-3 and 4-7 drop
+        // their 128-byte lines (whole lines of the row only: d % 32 == 0),
+        // after every lane's loads of them have returned
+        __syncwarp();
+        if ((d & 31) == 0 && lane < 8) {
+            const int line = lane & 3;
+            const int col = c0 + 32 * line;
+#pragma unroll
+            for (int b = 0; b < B; ++b) {
+                const int r = lane < 4 ? r0[b] : r1[b];
+                if (src[b] >= 0 && col < d && (unsigned)r < nrows) discard_l2_line(p.obuf + (size_t)r * d + col);
+            }
+        }
     }
 }
 
@@ -645,28 +655,8 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
             asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
         }
     }
-    // Weight-streaming tiles (32 token rows, the decode case): warm L2 with
-    // the first k-blocks of the weight tile this CTA most likely takes first,
-    // while the routing kernels still run.  The tile is a guess (number
-    // blockIdx.x with one row block per expert; the first wave takes tiles
-    // 0 .. grid-1 in some order); no kernel this one waits for writes the
-    // weights, and a wrong guess costs only bandwidth.
-    if constexpr (CG == 1 && RB == 32) {
-        if (warp == 0 && lane == 0 && p.prefetch_kblocks > 0) {
-            const int e = (int)blockIdx.x / p.n_tiles, nb = (int)blockIdx.x % p.n_tiles;
-            if (e < p.E) {
-                const int r0 = e * p.b_rows_per_expert + nb * (MODE == kUp ? BN / 2 : BN);
-                const int r1 = (MODE == kUp) ? r0 : r0 + BN / 2;
-                const int nk = min(p.prefetch_kblocks, (p.Kdim + BK - 1) / BK);
-                for (int kb = 0; kb < nk; ++kb) {
-                    tma_prefetch_2d(&tmB0, kb * BK, r0);
-                    tma_prefetch_2d(&tmB1, kb * BK, r1);
-                }
-            }
-        }
-    }
-    // the set-up above overlaps the previous kernels; offsets, the A rows and
-    // the tile counter are earlier kernels' outputs
+    // the set-up above overlaps the previous kernel's tail; offsets, the A
+    // rows and the tile counter are earlier kernels' outputs
     pdl_wait();
     pdl_trigger();
     if (threadIdx.x < p.E) {
@@ -1236,8 +1226,6 @@ cudaError_t launch_gemm(const GroupedGemmArgs& a, const CUtensorMap& mA, const C
     const long long ub = (long long)p.n_tiles * ((a.rows + C::kTileRows - 1) / C::kTileRows + a.E);
     const int grid_units = (int)(ub < units ? ub : units);
     if (grid_units <= 0) return cudaSuccess;
-    // L2 warm-up of weight-streaming tiles: about kPrefetchBytes over the grid
-    p.prefetch_kblocks = (CG == 1 && RB == 32) ? (int)(kPrefetchBytes / ((long long)grid_units * BN * BK * 2)) : 0;
     cfg.gridDim = dim3(grid_units * CG);
     set_pdl(attr[cfg.numAttrs++]);  // after the occupancy query, which takes the cluster attribute only
     return cudaLaunchKernelEx(&cfg, grouped_gemm_kernel<MODE, CG, BN, RB, NH>, mA, mAs, mB0, mB1, mOut, p);

@@ -14,16 +14,13 @@ cudaError_t read_clear_device_errors(unsigned int* out);
 
 // Programmatic dependent launch.  The layer's kernels are launched with
 // programmatic stream serialisation, so a kernel may start (launch, set up)
-// while its predecessor on the stream still runs; each one calls pdl_wait()
-// before it reads or writes anything an earlier kernel touches (the wait
-// returns once the predecessor grid has completed and its writes are
-// visible; it returns at once for a kernel launched without the attribute)
-// and pdl_trigger() to let its own successor launch early.  The small
-// kernels trigger before they wait, so a whole chain of launches and
-// set-ups (up to the expert GEMMs' barrier and tensor-memory set-up and
-// their first weight prefetches) runs ahead of the data; a successor only
-// launches once every CTA of its predecessor has started, so a waiting grid
-// never holds resources an earlier grid of the chain still needs.
+// while its predecessor on the stream finishes; each one calls pdl_wait()
+// before it reads anything an earlier kernel wrote (the wait returns once
+// the predecessor grid has completed and its writes are visible; it returns
+// at once for a kernel launched without the attribute) and pdl_trigger()
+// to let its own successor launch early.  (Triggering before the wait, so a
+// whole chain of launches runs ahead of the data, measured no faster on
+// B200: prefill +22 us, decode +1 us per layer in a paired A/B.)
 __device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 __device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
 inline void set_pdl(cudaLaunchAttribute& a) {

@@ -34,8 +34,8 @@ constexpr int kPermThreads = 1024;
 __global__ void __launch_bounds__(kPermThreads)
 permute_kernel(const int32_t* __restrict__ idx, int n, int E, int32_t* __restrict__ offsets,
                int32_t* __restrict__ perm, int32_t* __restrict__ inv) {
-    pdl_trigger();  // successors may launch and set up now; they wait for this grid before reading
     pdl_wait();
+    pdl_trigger();
     __shared__ int s_cnt[kMaxExperts];
     __shared__ int s_base[kMaxExperts];
     __shared__ int s_tile[kMaxExperts];
@@ -130,8 +130,8 @@ chunk_count_scan_kernel(const int32_t* __restrict__ idx, int n, int E, int nch, 
     extern __shared__ int s_cnt[];  // [E * nch], expert-major
     __shared__ int s_wsum[32];
     __shared__ int s_carry;
-    pdl_trigger();  // successors may launch and set up now; they wait for this grid before reading
     pdl_wait();
+    pdl_trigger();
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int m = E * nch;
     for (int i = tid; i < m; i += kScanThreads) s_cnt[i] = 0;
@@ -215,8 +215,8 @@ chunk_scatter_kernel(const int32_t* __restrict__ idx, int n, int E, int nch, int
     __shared__ int s_tok[kChunkA];
     const int c = blockIdx.x / parts, part = blockIdx.x - c * parts;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    pdl_trigger();  // successors may launch and set up now; they wait for this grid before reading
     pdl_wait();
+    pdl_trigger();
     clear_for_gemms(z);
     for (int i = tid; i < kRankWarps * kMaxExperts; i += kScatThreads) (&s_wcnt[0][0])[i] = 0;
     __syncthreads();
@@ -281,8 +281,8 @@ chunk_scatter_kernel(const int32_t* __restrict__ idx, int n, int E, int nch, int
 __global__ void __launch_bounds__(kFlatThreads)
 gather_rows_kernel(const __nv_bfloat16* __restrict__ x, const int32_t* __restrict__ perm, int rows,
                    int d, int k, __nv_bfloat16* __restrict__ xp, const ZeroArgs z, const UnroutedArgs u) {
-    pdl_trigger();  // successors may launch and set up now; they wait for this grid before reading
     pdl_wait();
+    pdl_trigger();
     clear_for_gemms(z);
     if (u.y) {
         // y rows of tokens with no routed slot: residual or zero (rare; a
@@ -326,8 +326,8 @@ gather_rows_kernel(const __nv_bfloat16* __restrict__ x, const int32_t* __restric
 __global__ void __launch_bounds__(kFlatThreads)
 combine_f32_kernel(const float* __restrict__ obuf, const int32_t* __restrict__ inv,
                    const float* __restrict__ residual, int T, int d, int k, float* __restrict__ y) {
-    pdl_trigger();  // successors may launch and set up now; they wait for this grid before reading
     pdl_wait();
+    pdl_trigger();
     const int nvec = d / 4;
     const unsigned n = (unsigned)(T * k);
     for (int t = blockIdx.x; t < T; t += gridDim.x) {

@@ -25,11 +25,12 @@
 //
 // Reduction (fixed order, so the result is deterministic): each warp's MMAs
 // alternate between two accumulators (even and odd m) that are added at the
-// end; CTA 0 of the cluster adds the CTAs' partial logits in rank order
-// through distributed shared memory, then selects the top-k with warp
-// shuffles (a segment of lanes per token; k rounds of arg-max, an exact tie
-// keeps the lower index; slot 0 = largest) and computes the fp32 softmax of
-// the kept logits.  The split changes the summation order but not the rule:
+// end; each CTA of the cluster then takes an eighth of the block's tokens,
+// adds the CTAs' partial logits of those tokens in rank order through
+// distributed shared memory, selects their top-k with warp shuffles (a
+// segment of lanes per token; k rounds of arg-max, an exact tie keeps the
+// lower index; slot 0 = largest) and computes the fp32 softmax of the kept
+// logits.  The split changes the summation order but not the rule:
 // logits are fp64 sums of exact products.
 
 #include <cooperative_groups.h>
@@ -50,8 +51,8 @@ constexpr int kFragDoubles = kChunks * 8 * 32;  // 4096 doubles = 32 KiB
 
 // Dynamic shared memory: the fp64 weight fragments wfrag[kChunks][8][32] and
 // this CTA's partial logits part[kTokBlock][E].  After the cluster reduction
-// CTA 0 keeps the final logits [kTokBlock][E] in the wfrag area
-// (kTokBlock * E <= 64 * 64 = kFragDoubles).
+// each CTA keeps the final logits of its share of the tokens [kTokBlock / 8][E]
+// in the wfrag area.
 __host__ __device__ constexpr size_t router_smem_bytes(int E) {
     return sizeof(double) * ((size_t)kFragDoubles + (size_t)kTokBlock * E);
 }
@@ -108,8 +109,8 @@ __global__ void __launch_bounds__(kWarps * 32, BF16 ? 4 : 2)  // bf16: 64 regist
 router_topk_kernel(const void* __restrict__ x, const void* __restrict__ Wg, int T, int d, int E, int k,
                    int32_t* __restrict__ idx_out, float* __restrict__ w_out) {
     extern __shared__ __align__(16) unsigned char smem_raw[];
-    pdl_trigger();  // successors may launch and set up now; they wait for this grid before reading
     pdl_wait();     // x may be the previous kernel's output (a layer stack)
+    pdl_trigger();
     double* wfrag = reinterpret_cast<double*>(smem_raw);  // [kChunks][8][32]
     double* part = wfrag + kFragDoubles;                  // [kTokBlock][E]
     cg::cluster_group cluster = cg::this_cluster();
@@ -187,18 +188,16 @@ router_topk_kernel(const void* __restrict__ x, const void* __restrict__ Wg, int 
     }
 
     cluster.sync();  // every CTA's partial logits are complete and visible
-    if (rank == 0) {
-        // logits = sum over the CTAs in rank order, written over wfrag
-        double* lg_all = wfrag;
-        for (int i = threadIdx.x; i < kTokBlock * E; i += kWarps * 32) {
-            double s = 0.0;
-            for (int r = 0; r < nranks; ++r) s += cluster.map_shared_rank(part, r)[i];
-            lg_all[i] = s;
-        }
+    // CTA r finishes tokens r*tpr .. r*tpr + tpr-1 of the block: their logits
+    // are the CTAs' partial sums added in rank order (written over wfrag)
+    const int tpr = kTokBlock / nranks;
+    for (int i = threadIdx.x; i < tpr * E; i += kWarps * 32) {
+        const size_t cell = (size_t)(rank * tpr) * E + i;
+        double sum = 0.0;
+        for (int r = 0; r < nranks; ++r) sum += cluster.map_shared_rank(part, r)[cell];
+        wfrag[i] = sum;
     }
-    cluster.sync();  // peers keep their shared memory until CTA 0 has read it
-    if (rank != 0) return;
-    __syncthreads();
+    cluster.sync();  // no CTA leaves while another still reads its partials
     // Top-k, warp-level: a segment of S lanes per token (S = E rounded up to
     // a power of two, at most 32; lane sl of the segment holds experts sl,
     // sl + S), so a warp selects for 32 / S tokens at once.  Each of the k
@@ -212,17 +211,17 @@ router_topk_kernel(const void* __restrict__ x, const void* __restrict__ Wg, int 
     const int per = (E + S - 1) / S;  // experts per lane: 1, or 2 when E > 32
     const int tpw = 32 / S;           // tokens per warp per pass
     const int sl = lane & (S - 1);
-    for (int base = warp * tpw; base < kTokBlock; base += kWarps * tpw) {
-        const int tl = base + lane / S;
-        const int t = tok0 + tl;
-        const bool live = t < T;  // uniform in a segment
+    for (int base = warp * tpw; base < tpr; base += kWarps * tpw) {
+        const int tm = base + lane / S;  // token of this CTA's share
+        const int t = tok0 + rank * tpr + tm;
+        const bool live = tm < tpr && t < T;  // uniform in a segment
         double v[2];
         bool open[2];
 #pragma unroll
         for (int i = 0; i < 2; ++i) {
             const int e = sl + i * S;
             open[i] = live && i < per && e < E;
-            v[i] = open[i] ? wfrag[(size_t)tl * E + e] : 0.0;
+            v[i] = open[i] ? wfrag[(size_t)tm * E + e] : 0.0;
         }
         int32_t* io = idx_out + (size_t)t * k;
         float* wo = w_out + (size_t)t * k;
