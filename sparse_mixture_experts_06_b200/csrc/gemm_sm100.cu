@@ -329,6 +329,10 @@ __device__ __forceinline__ void st_shared_v4(uint32_t addr, uint4 v) {
 // r * 128 + ((j ^ (r & 7)) << 4), which also makes the 32 lanes'
 // shared-memory writes conflict-free.
 constexpr int kOutBoxBytes = 32 * 128;
+// Whole 32-row boxes go out through shared memory and bulk tensor stores.
+// (false: every lane stores its row's 128-byte line directly; measured on
+// B200 slower: prefill +81 us, skewed +348 us per layer.)
+constexpr bool kStagedStores = true;
 constexpr int kOutBytes = kEpiWarps * kOutBoxBytes;
 
 // ---------------------------------------------------------------------------
@@ -885,7 +889,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
             // uses per-row stores (a full-box store would overwrite the next
             // expert's rows)
             const int wrow0 = row - lane;
-            const bool box_ok = wrow0 + 32 <= tile_end;
+            const bool box_ok = kStagedStores && wrow0 + 32 <= tile_end;
             // down: the row's assignment, its gate weight, and its token's
             // slot rows, loaded while the tile's MMAs run
             int tok = 0, rr0 = -1, rr1 = -1, nvalid = 0;
@@ -944,10 +948,6 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
                         if ((unit++ & 1) != sub) continue;
                         const int c64 = (shrt ? colhalf : seg) * 64;        // hidden offset in the tile
                         const int acol = (CG == 1) ? seg * 64 : (shrt ? 0 : seg * 128);
-                        if (box_ok) {
-                            if (lane == 0) bulk_wait_read_all();  // the buffer's previous store has read it
-                            __syncwarp();
-                        }
 #pragma unroll 1
                         for (int half = 0; half < 2; ++half) {
                             const int c = c64 + half * 32;
@@ -968,6 +968,12 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
                                                       silu_mul(__uint_as_float(a[g * 8 + 7]), __uint_as_float(b[g * 8 + 7])));
                             }
                             if (box_ok) {
+                                if (half == 0) {
+                                    // the buffer's previous store has read it (waited for
+                                    // only now, so the wait overlaps the loads and the math)
+                                    if (lane == 0) bulk_wait_read_all();
+                                    __syncwarp();
+                                }
 #pragma unroll
                                 for (int g = 0; g < 4; ++g)
                                     st_shared_v4(buf + lane * 128 + ((((half * 4 + g) ^ (lane & 7))) << 4), pk[g]);
@@ -1002,10 +1008,6 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
                     for (int u = 0; u < kCombineCols / 32; ++u) {
                         const int cc = (g - h * gpp) * kCombineCols + u * 32;  // TMEM column within part h
                         const int col = ob + cc;
-                        if (box_ok) {
-                            if (lane == 0) bulk_wait_read_all();  // the buffer's previous store has read it
-                            __syncwarp();
-                        }
                         uint32_t o[32];
                         tmem_ld32(tacc + cc, o);
                         tmem_wait_ld();
@@ -1018,6 +1020,10 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
                             v[i].w = __float_as_uint(wgt * __uint_as_float(o[i * 4 + 3]));
                         }
                         if (box_ok) {
+                            // the buffer's previous store has read it (waited for only
+                            // now, so the wait overlaps the load and the scaling)
+                            if (lane == 0) bulk_wait_read_all();
+                            __syncwarp();
 #pragma unroll
                             for (int i = 0; i < 8; ++i) st_shared_v4(buf + lane * 128 + ((i ^ (lane & 7)) << 4), v[i]);
                             fence_proxy_async_smem();
