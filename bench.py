@@ -432,89 +432,94 @@ def e2e_leg(args, s, t, device, steps):
 
 def gemm_vs_cublas(args, device):
     """The expert GEMMs of the prefill layer (T = 4096, d = 4096, f = 14336,
-    E = 8, k = 2) against cuBLAS through torch.matmul, for context:
-      * one dense GEMM of all 8192 rows (up: [8192, d] x [d, 2f]; down:
-        [8192, f] x [f, d]), cuBLAS's best case;
-      * cuBLAS per expert on the rows the router actually gave each expert
-        (the grouped work, one call per expert, no SwiGLU or gate fusion);
-      * ours on a one-expert layer of 8192 rows (E = 1, k = 1: no ragged
-        tiles) for each CTA grouping, and ours on the grouped prefill layer,
-        both from the library's stage profiler.
-    cuBLAS here is a measuring stick only; the layer never calls it."""
+    E = 8, k = 2) against cuBLAS through torch.matmul, for context.  Four
+    arms, run in turn within every step (so that all see the same clocks
+    under the power cap), each after an L2 flush; medians over the steps:
+      * cuBLAS on one dense GEMM of all 8192 rows (up: [8192, d] x [d, 2f];
+        down: [8192, f] x [f, d]), no SwiGLU or gate: cuBLAS's best case;
+      * ours on one expert of 8192 rows (E = k = 1): no expert tails;
+      * ours on the router's routing of the prefill batch (its expert row
+        counts leave short last row blocks, the tails);
+      * ours on a balanced routing (token t -> experts 2t mod 8, 2t+1 mod 8:
+        1024 rows per expert, a multiple of the 256-row pair tiles).
+    Ours through moe_expert_ffn, the GEMM times from the library's stage
+    profiler.  cuBLAS is a measuring stick only; the layer never calls it."""
+    import numpy as np
     import torch
     import synth
     import sparse_mixture_experts_06_b200 as moe
     from synth.device import device_inputs
 
-    def t_ms(fn, reps=20):
-        for _ in range(3):
-            fn()
-        torch.cuda.synchronize(device)
-        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        a.record()
-        for _ in range(reps):
-            fn()
-        b.record()
-        torch.cuda.synchronize(device)
-        return a.elapsed_time(b) / reps
-
     s = synth.CONFIGS["prefill"]
     M, d, f = s.T * s.k, s.d, s.f
-    tf = lambda flop, ms: round(flop / ms / 1e9, 1)  # noqa: E731
+    flush = torch.empty(512 << 20, dtype=torch.uint8, device=device)
     g = torch.Generator(device=device).manual_seed(0)
     x = torch.randn(M, d, device=device, generator=g).to(torch.bfloat16)
     W13 = (torch.randn(2 * f, d, device=device, generator=g) / 64).to(torch.bfloat16)
     h = torch.randn(M, f, device=device, generator=g).to(torch.bfloat16)
     W2 = (torch.randn(d, f, device=device, generator=g) / 120).to(torch.bfloat16)
-    out = {"mode": "gemm_vs_cublas", "unit": "TFLOP/s", "rows": M, "d": d, "f": f}
-    up = t_ms(lambda: x @ W13.t())
-    dn = t_ms(lambda: h @ W2.t())
-    out["cublas_dense"] = {"up_ms": round(up, 4), "up": tf(4.0 * M * d * f, up),
-                           "down_ms": round(dn, 4), "down": tf(2.0 * M * d * f, dn)}
-    del x, W13, h, W2
 
-    # grouped: the router's per-expert row counts of the prefill batch
-    t = make_inputs(s, 0, device)
-    idx, _ = moe.moe_router_topk(t["x"], t["Wg"], s.k)
-    counts = torch.bincount(idx.flatten().long(), minlength=s.E).tolist()
-    xs = [torch.randn(c, d, device=device, generator=g).to(torch.bfloat16) for c in counts]
-    hs = [torch.randn(c, f, device=device, generator=g).to(torch.bfloat16) for c in counts]
-    W13e = torch.cat([t["W1"], t["W3"]], dim=1)  # [E, 2f, d]
-    upg = t_ms(lambda: [xe @ W13e[e].t() for e, xe in enumerate(xs)])
-    dng = t_ms(lambda: [he @ t["W2"][e].t() for e, he in enumerate(hs)])
-    out["cublas_per_expert"] = {"counts": counts, "up_ms": round(upg, 4), "up": tf(4.0 * M * d * f, upg),
-                                "down_ms": round(dng, 4), "down": tf(2.0 * M * d * f, dng)}
-    del xs, hs, W13e
+    def timed(fn):
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        fn()
+        b.record()
+        b.synchronize()
+        return a.elapsed_time(b)
 
-    def ours(shape, tt, key, cta_group=0):
-        moe.moe_set_gemm_variant(cta_group)
-        try:
-            y = torch.empty_like(tt["x"])
-            ws = torch.empty(moe.moe_workspace_size(shape.T, d, f, shape.E, shape.k, 0), dtype=torch.uint8,
-                             device=device)
-            run = lambda: moe.moe_layer_forward_ex(tt["x"], tt["Wg"], tt["W1"], tt["W3"], tt["W2"], shape.k,  # noqa: E731
-                                                   y=y, workspace=ws)
-            for _ in range(3):
-                run()
-            torch.cuda.synchronize(device)
+    def cublas():
+        up = timed(lambda: x @ W13.t())
+        flush.zero_()
+        return up, timed(lambda: h @ W2.t())
+
+    def ours(tt, routing, ws, y):
+        off, perm, inv, w = routing
+
+        def run():
+            moe.moe_profile_select(None)
             moe.moe_profile_enable(True)
-            for _ in range(20):
-                run()
-            torch.cuda.synchronize(device)
-            p = moe.moe_profile_read()
+            moe.moe_expert_ffn(tt["x"], tt["W1"], tt["W3"], tt["W2"], off, perm, inv, w, y=y, workspace=ws)
+            torch.cuda.synchronize()
+            pr = moe.moe_profile_read()
             moe.moe_profile_enable(False)
-        finally:
-            moe.moe_set_gemm_variant()
-        u, w = p["up_swiglu_gemm"][0] / 20, p["down_combine_gemm"][0] / 20
-        out[key] = {"up_ms": round(u, 4), "up": tf(4.0 * M * d * f, u), "down_ms": round(w, 4),
-                    "down": tf(2.0 * M * d * f, w)}
+            return pr["up_swiglu_gemm"][0], pr["down_combine_gemm"][0]
+        return run
 
     one = synth.MoEShape("one-expert", M, d, f, 1, 1, "bf16")
     t1 = device_inputs(one, 0, device=device)
-    for cg in (1, 2):
-        ours(one, t1, "ours_one_expert_cta_group_%d" % cg, cta_group=cg)
-    del t1
-    ours(s, t, "ours_grouped_prefill")
+    r1 = (*moe.moe_permute(torch.zeros(M, 1, dtype=torch.int32, device=device), 1),
+          torch.ones(M, 1, dtype=torch.float32, device=device))
+    ws1 = torch.empty(moe.moe_workspace_size(M, d, f, 1, 1, 0), dtype=torch.uint8, device=device)
+    tp = make_inputs(s, 0, device)
+    idx, w = moe.moe_router_topk(tp["x"], tp["Wg"], s.k)
+    rr = (*moe.moe_permute(idx, s.E), w)
+    bal = np.stack([(2 * np.arange(s.T)) % s.E, (2 * np.arange(s.T) + 1) % s.E], 1).astype(np.int32)
+    rb = (*moe.moe_permute(torch.from_numpy(bal).to(device), s.E), w)
+    wsp = torch.empty(moe.moe_workspace_size(s.T, d, f, s.E, s.k, 0), dtype=torch.uint8, device=device)
+    y1 = torch.empty(M, d, dtype=torch.bfloat16, device=device)
+    yp = torch.empty(s.T, d, dtype=torch.bfloat16, device=device)
+    arms = {"cublas_dense": cublas, "ours_one_expert": ours(t1, r1, ws1, y1),
+            "ours_router_routing": ours(tp, rr, wsp, yp), "ours_balanced_routing": ours(tp, rb, wsp, yp)}
+    for fn in arms.values():
+        for _ in range(3):
+            flush.zero_()
+            torch.cuda.synchronize()
+            fn()
+    res = {k: [] for k in arms}
+    steps = max(10, min(args.steps, 40))
+    for i in range(steps):
+        for k in (list(arms) if i % 2 == 0 else list(arms)[::-1]):
+            flush.zero_()
+            torch.cuda.synchronize()
+            res[k].append(arms[k]())
+    tf = lambda flop, ms: round(flop / ms / 1e9, 1)  # noqa: E731
+    out = {"mode": "gemm_vs_cublas", "unit": "TFLOP/s", "rows": M, "d": d, "f": f, "steps": steps,
+           "router_counts": np.diff(rr[0].cpu().numpy()).tolist()}
+    for k, v in res.items():
+        up = statistics.median(a for a, _ in v)
+        dn = statistics.median(b for _, b in v)
+        out[k] = {"up_ms": round(up, 4), "up": tf(4.0 * M * d * f, up), "down_ms": round(dn, 4),
+                  "down": tf(2.0 * M * d * f, dn)}
     print(json.dumps(out))
     return 0
 
