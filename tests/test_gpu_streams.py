@@ -37,3 +37,34 @@ def test_concurrent_layers_on_two_streams_match_sequential(shapes):
     for r, y in zip(ref, outs):
         assert torch.equal(r.view(torch.int16), y.view(torch.int16))
     assert moe.moe_device_errors() == 0
+
+
+def test_library_workspace_grows_safely_across_streams():
+    """moe_layer_forward shares one library workspace per device.  A larger
+    shape that arrives on another stream while a call is still queued grows
+    it: the old workspace must be freed only after the queued call's work
+    (the library orders the free after an event recorded at the end of its
+    last user's work).  The first call's result must equal the same layer
+    run alone; the second call must be correct too."""
+    small = synth.MoEShape("grow-a", 2304, 256, 512, 8, 2, "bf16")
+    big = synth.MoEShape("grow-b", 6000, 256, 512, 8, 2, "bf16")
+    ta, tb = device_inputs(small, 61), device_inputs(big, 62)
+    ref_a = moe.moe_layer_forward_ex(ta["x"], ta["Wg"], ta["W1"], ta["W3"], ta["W2"], 2)
+    ref_b = moe.moe_layer_forward_ex(tb["x"], tb["Wg"], tb["W1"], tb["W3"], tb["W2"], 2)
+    torch.cuda.synchronize()
+    for _ in range(3):
+        moe.moe_release_workspace()  # start from a pool sized for nothing
+        torch.cuda.synchronize()
+        sa, sb = torch.cuda.Stream(), torch.cuda.Stream()
+        ya, yb = torch.empty_like(ta["x"]), torch.empty_like(tb["x"])
+        # a long kernel first on stream a, so its layer is still queued when b grows the pool
+        busy = torch.empty(1 << 30, dtype=torch.uint8, device="cuda")
+        with torch.cuda.stream(sa):
+            busy.fill_(1)
+        moe.moe_layer_forward(ta["x"], ta["Wg"], ta["W1"], ta["W3"], ta["W2"], 2, y=ya, stream=sa)
+        moe.moe_layer_forward(tb["x"], tb["Wg"], tb["W1"], tb["W3"], tb["W2"], 2, y=yb, stream=sb)
+        torch.cuda.synchronize()
+        assert torch.equal(ref_a.view(torch.int16), ya.view(torch.int16))
+        assert torch.equal(ref_b.view(torch.int16), yb.view(torch.int16))
+    moe.moe_release_workspace()
+    assert moe.moe_device_errors() == 0
