@@ -675,6 +675,17 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
     const uint32_t tmem_base = *tmem_slot;
 
     const int total = count_tiles_rows(s_beg, s_end, p.E, p.n_tiles, C::kTileRows);
+    // Weight-streaming tiles (32 token rows: HBM-bound) in even waves: with
+    // w = ceil(total / grid) waves, only ceil(total / w) CTAs take tiles, so
+    // no last wave of a few tiles streams alone while the others idle (at
+    // decode 896 tiles run as 7 waves of 128, not 6 of 148 and one of 8).
+    // The other CTAs take no tile and leave.
+    int active = (int)gridDim.x / CG;
+    if constexpr (CG == 1 && RB == 32) {
+        const int waves = (total + active - 1) / active;
+        if (waves > 0) active = (total + waves - 1) / waves;
+    }
+    const bool takes_tiles = (int)blockIdx.x / CG < active;
     const int kblocks = (p.Kdim + BK - 1) / BK;
     // a reader of tile-ring slot i: wait for the number, read it, release the slot
     const uint32_t sempty_leader0 = (CG == 2) ? map_to_rank(smem_u32(&sempty[0]), 0) : smem_u32(&sempty[0]);
@@ -699,7 +710,9 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
             bool ok = true;
             // The next tile's number is taken while the last STG stages of the
             // current tile are issued, so the atomic's latency is hidden.
-            int next = leader ? atomicAdd(p.tile_counter, 1) : -1;  // the odd CTA of a pair reads the even one's
+            // (the odd CTA of a pair reads the even one's; a CTA beyond the
+            // active ones publishes the end at once)
+            int next = leader ? (takes_tiles ? atomicAdd(p.tile_counter, 1) : total) : -1;
             for (uint32_t ti = 0; ok; ++ti) {
                 int tile;
                 if (leader) {
