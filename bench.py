@@ -81,28 +81,88 @@ def workload_desc(s, n):
 
 
 class ClockSampler:
-    """nvidia-smi samples every 200 ms while the timed region runs."""
+    """SM clock, power and clock-event reasons of the benchmarked GPU while
+    the timed region runs: NVML read every 2 ms from a side thread (read-only
+    queries), else `nvidia-smi -lms 200` if NVML cannot be loaded.  The GPU
+    is found by its PCI bus id (NVML numbers all GPUs of the host, whatever
+    CUDA_VISIBLE_DEVICES says)."""
 
     FIELDS = ("index,pci.bus_id,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    REASONS = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+    PERIOD_S = 0.002
 
     def __init__(self, bus_id):
         self.bus_id = (bus_id or "").lower()
         self.proc = None
         self.path = None
+        self.nvml = None
+        self.handle = None
+        self.thread = None
+        self.halt = threading.Event()
+        self.rows = []
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            key = self.bus_id[-5:] + "."  # "bb:dd." of domain:bus:device
+            for i in range(pynvml.nvmlDeviceGetCount()):
+                h = pynvml.nvmlDeviceGetHandleByIndex(i)
+                bid = pynvml.nvmlDeviceGetPciInfo(h).busId
+                bid = (bid.decode() if isinstance(bid, bytes) else bid).lower()
+                if self.bus_id and key in bid:
+                    self.handle = h
+                    break
+            if self.handle is not None:
+                self.nvml = pynvml
+        except Exception:
+            self.nvml = None
+
+    def _poll(self):
+        n = self.nvml
+        bits = (n.nvmlClocksEventReasonHwSlowdown, n.nvmlClocksEventReasonHwThermalSlowdown,
+                n.nvmlClocksEventReasonSwThermalSlowdown, n.nvmlClocksEventReasonSwPowerCap)
+        while not self.halt.is_set():
+            try:
+                sm = n.nvmlDeviceGetClockInfo(self.handle, n.NVML_CLOCK_SM)
+                r = n.nvmlDeviceGetCurrentClocksEventReasons(self.handle)
+                w = n.nvmlDeviceGetPowerUsage(self.handle) / 1000.0
+                self.rows.append((sm, w, tuple(bool(r & b) for b in bits)))
+            except Exception:
+                return
+            time.sleep(self.PERIOD_S)
 
     def start(self):
+        if self.nvml is not None:
+            self.thread = threading.Thread(target=self._poll, daemon=True)
+            self.thread.start()
+            return
         try:
             fd, self.path = tempfile.mkstemp(suffix=".csv")
             os.close(fd)
             self.proc = subprocess.Popen(["nvidia-smi", "--query-gpu=" + self.FIELDS, "--format=csv,noheader,nounits",
                                           "-lms", "200", "-f", self.path], stdout=subprocess.DEVNULL,
                                          stderr=subprocess.DEVNULL)
+            time.sleep(0.5)
         except Exception:
             self.proc = None
 
     def stop(self):
+        if self.thread is not None:
+            self.halt.set()
+            self.thread.join()
+            if not self.rows:
+                return None
+            n = self.nvml
+            try:
+                mx = float(n.nvmlDeviceGetMaxClockInfo(self.handle, n.NVML_CLOCK_SM))
+            except Exception:
+                mx = None
+            reasons = sorted({self.REASONS[i] for _, _, f in self.rows for i in range(4) if f[i]})
+            sm = [float(r[0]) for r in self.rows]
+            return {"sm_mhz": statistics.median(sm), "sm_min_mhz": min(sm), "sm_max_mhz": mx, "reasons": reasons,
+                    "samples": len(self.rows), "source": "NVML every %g ms during the timed steps" % (1e3 * self.PERIOD_S),
+                    "power_w_max": max(r[1] for r in self.rows)}
         if self.proc is None:
             return None
         self.proc.terminate()
@@ -123,10 +183,10 @@ class ClockSampler:
             return None
         sm = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
         mx = max(float(r[3]) for r in rows if r[3].replace(".", "").isdigit())
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        reasons = sorted({names[i] for r in rows for i in range(4) if r[6 + i].lower().startswith("active")})
+        reasons = sorted({self.REASONS[i] for r in rows for i in range(4) if r[6 + i].lower().startswith("active")})
         return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": mx, "reasons": reasons,
-                "samples": len(rows), "power_w_max": max(float(r[4]) for r in rows if r[4].replace(".", "").isdigit())}
+                "samples": len(rows), "source": "nvidia-smi every 200 ms",
+                "power_w_max": max(float(r[4]) for r in rows if r[4].replace(".", "").isdigit())}
 
 
 def gemm_source_hash():
@@ -299,7 +359,6 @@ def bench_workload(args, s, rank, world, device, dist, extras_for_decode=False, 
     sampler = ClockSampler(bus) if rank == 0 and not extras_for_decode else None
     if sampler:
         sampler.start()
-        time.sleep(0.5)
     evs = timed_loop(step, args.steps, flush if l2_flush else None, stream)
     torch.cuda.synchronize(device)
     if dist is not None:

@@ -40,8 +40,14 @@
 //
 // Tiles are enumerated per expert from the device-side offsets (no host
 // round trip): expert e owns ceil(M_e / tile rows) row blocks x n_tiles column
-// blocks, numbered with the row block fastest so that the CTAs running at
-// the same time share weight tiles through L2.  Tiles are handed out
+// blocks.  The row blocks are taken in groups of G; inside a group the row
+// block is the fastest index, so the P tiles that run at the same time cover
+// ~G row blocks x P / G column blocks and share both operands through L2.
+// G = sqrt(P x tile columns / tile rows) makes the bytes of those distinct
+// A rows and B columns least (G x A-tile + P / G x B-tile, with the A and B
+// tiles' bytes in proportion to their rows); an expert of at most G row
+// blocks is one group (every expert at T = 4096 on Mixtral shapes; at
+// T = 16384 with skewed routing the hottest expert has 45).  Tiles are handed out
 // dynamically: the producer (the even CTA's, for pairs) takes the next tile
 // number from a global counter and passes it to the other roles (and to the
 // odd CTA) through a small shared-memory ring, so short and full tiles
@@ -56,7 +62,9 @@
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
+#include <algorithm>
 #include <atomic>
+#include <cmath>
 #include <cstdlib>
 #include <mutex>
 
@@ -101,6 +109,7 @@ struct KParams {
     int* tile_counter;       // next tile to hand out; zero at launch (the row gather zeroes it)
     unsigned long long wait_limit_ns;  // bound of every pipeline wait
     int stall_test;          // failure-detection test: the epilogue waits on a barrier nothing completes
+    int m_group;             // row blocks per group of the tile order (>= 1)
 };
 
 // Row ranges: all rows of each expert; only its whole 256-row blocks; or
@@ -278,12 +287,33 @@ __device__ __forceinline__ void tma_load_2d_pair(uint32_t dst, const CUtensorMap
         : "memory");
 }
 
+// A_USE: how the MMA treats the tensor core's collector buffer for A.
+// 0: A read from shared memory (no reuse); 1 (fill): read from shared
+// memory and kept in the collector; 2 (lastuse): taken from the collector,
+// which the previous MMA filled with the same A, and released.  The two
+// MMAs of a 256 x 512 pair tile share each A block, so the second one
+// reads no A from shared memory.
+template <int A_USE = 0>
 __device__ __forceinline__ void umma_bf16_pair(uint32_t d_tmem, uint64_t a, uint64_t b, uint32_t idesc, uint32_t acc) {
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "setp.ne.b32 p, %4, 0;\n\t"
-        "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}\n" ::"r"(d_tmem),
-        "l"(a), "l"(b), "r"(idesc), "r"(acc));
+    if constexpr (A_USE == 1) {
+        asm volatile(
+            "{\n\t.reg .pred p;\n\t"
+            "setp.ne.b32 p, %4, 0;\n\t"
+            "tcgen05.mma.cta_group::2.kind::f16.collector::a::fill [%0], %1, %2, %3, p;\n\t}\n" ::"r"(d_tmem),
+            "l"(a), "l"(b), "r"(idesc), "r"(acc));
+    } else if constexpr (A_USE == 2) {
+        asm volatile(
+            "{\n\t.reg .pred p;\n\t"
+            "setp.ne.b32 p, %4, 0;\n\t"
+            "tcgen05.mma.cta_group::2.kind::f16.collector::a::lastuse [%0], %1, %2, %3, p;\n\t}\n" ::"r"(d_tmem),
+            "l"(a), "l"(b), "r"(idesc), "r"(acc));
+    } else {
+        asm volatile(
+            "{\n\t.reg .pred p;\n\t"
+            "setp.ne.b32 p, %4, 0;\n\t"
+            "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}\n" ::"r"(d_tmem),
+            "l"(a), "l"(b), "r"(idesc), "r"(acc));
+    }
 }
 
 // Arrive-one on the mbarrier at the same offset in both CTAs of the pair when
@@ -397,16 +427,23 @@ __device__ __forceinline__ int count_tiles_rows(const int* s_beg, const int* s_e
     return total;
 }
 
+// Tile number -> (expert, row block, column block): experts in order; inside
+// an expert, groups of G row blocks (the last one may be shorter); inside a
+// group, column block major and row block fastest.
 __device__ __forceinline__ void decode_tile_rows(int tile, const int* s_beg, const int* s_end, int E, int n_tiles,
-                                                 int rows_per_tile, int& e, int& m_blk, int& n_blk) {
+                                                 int rows_per_tile, int G, int& e, int& m_blk, int& n_blk) {
     int base = 0;
     for (e = 0; e < E; ++e) {
         const int mt = (s_end[e] - s_beg[e] + rows_per_tile - 1) / rows_per_tile;
         const int tiles = mt * n_tiles;
         if (tile < base + tiles) {
             const int local = tile - base;
-            n_blk = local / mt;
-            m_blk = local - n_blk * mt;
+            const int g = local / (G * n_tiles);
+            const int g0 = g * G;
+            const int gs = min(G, mt - g0);  // row blocks of this group
+            const int r = local - g0 * n_tiles;
+            n_blk = r / gs;
+            m_blk = g0 + (r - n_blk * gs);
             return;
         }
         base += tiles;
@@ -736,7 +773,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
                 }
                 if (tile < 0) break;
                 int e, mb, nb;
-                decode_tile_rows(tile, s_beg, s_end, p.E, p.n_tiles, C::kTileRows, e, mb, nb);
+                decode_tile_rows(tile, s_beg, s_end, p.E, p.n_tiles, C::kTileRows, p.m_group, e, mb, nb);
                 const int start = s_beg[e] + mb * C::kTileRows;
                 const bool shrt = (CG == 2) && short_pair_tile(start, min(s_end[e], start + C::kTileRows));
                 const int rowA = start + (int)rank * (shrt ? 64 : 128);
@@ -819,7 +856,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
                 uint32_t idesc = C::kIdesc;
                 if constexpr (CG == 2) {
                     int e, mb, nb;
-                    decode_tile_rows(tile, s_beg, s_end, p.E, p.n_tiles, C::kTileRows, e, mb, nb);
+                    decode_tile_rows(tile, s_beg, s_end, p.E, p.n_tiles, C::kTileRows, p.m_group, e, mb, nb);
                     const int start = s_beg[e] + mb * C::kTileRows;
                     if (short_pair_tile(start, min(s_end[e], start + C::kTileRows))) idesc = C::kIdescShort;
                 }
@@ -837,11 +874,16 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
                             umma_bf16(d_tmem, adesc + (uint64_t)(kk * 2), bdesc + (uint64_t)(kk * 2), C::kIdesc,
                                       (kb | kk) != 0 ? 1u : 0u);
                         } else {
-#pragma unroll
-                            for (int h = 0; h < NH; ++h)  // part h of B (kBHalf bytes = kBHalf >> 4 descriptor units)
-                                umma_bf16_pair(d_tmem + h * BN, adesc + (uint64_t)(kk * 2),
-                                               bdesc + (uint64_t)(h * (C::kBHalf >> 4) + kk * 2), idesc,
-                                               (kb | kk) != 0 ? 1u : 0u);
+                            // part h of B (kBHalf bytes = kBHalf >> 4 descriptor units)
+                            const uint64_t ak = adesc + (uint64_t)(kk * 2);
+                            const uint32_t accum = (kb | kk) != 0 ? 1u : 0u;
+                            if constexpr (NH == 2) {
+                                umma_bf16_pair<1>(d_tmem, ak, bdesc + (uint64_t)(kk * 2), idesc, accum);
+                                umma_bf16_pair<2>(d_tmem + BN, ak, bdesc + (uint64_t)((C::kBHalf >> 4) + kk * 2),
+                                                  idesc, accum);
+                            } else {
+                                umma_bf16_pair(d_tmem, ak, bdesc + (uint64_t)(kk * 2), idesc, accum);
+                            }
                         }
                     }
                     if constexpr (CG == 1) umma_commit(smem_u32(&empty[s])); else umma_commit_pair(smem_u32(&empty[s]));
@@ -883,7 +925,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
             if (lane == 0) release_tile(tcount);
             if (tile < 0) break;
             int e, mb, nb;
-            decode_tile_rows(tile, s_beg, s_end, p.E, p.n_tiles, C::kTileRows, e, mb, nb);
+            decode_tile_rows(tile, s_beg, s_end, p.E, p.n_tiles, C::kTileRows, p.m_group, e, mb, nb);
             const uint32_t acc = tcount % C::kNAcc;
             const uint32_t use = tcount / C::kNAcc;
             const int start = s_beg[e] + mb * C::kTileRows;
@@ -1245,6 +1287,8 @@ cudaError_t launch_gemm(const GroupedGemmArgs& a, const CUtensorMap& mA, const C
     const long long ub = (long long)p.n_tiles * ((a.rows + C::kTileRows - 1) / C::kTileRows + a.E);
     const int grid_units = (int)(ub < units ? ub : units);
     if (grid_units <= 0) return cudaSuccess;
+    // row blocks per group of the tile order: sqrt(units x tile columns / tile rows)
+    p.m_group = std::max(1, (int)std::lround(std::sqrt((double)grid_units * C::kTileN / C::kTileRows)));
     cfg.gridDim = dim3(grid_units * CG);
     set_pdl(attr[cfg.numAttrs++]);  // after the occupancy query, which takes the cluster attribute only
     return cudaLaunchKernelEx(&cfg, grouped_gemm_kernel<MODE, CG, BN, RB, NH>, mA, mAs, mB0, mB1, mOut, p);

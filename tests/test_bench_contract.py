@@ -31,3 +31,55 @@ def test_peaks_fall_back_when_the_measured_file_is_absent(tmp_path, monkeypatch)
     (tmp_path / "MEASURED_PEAKS.json").write_text(json.dumps({"hbm_gbs": 1.0, "bf16_tflops": 2.0}))
     pk, kind = bench.peaks()
     assert kind == "measured" and pk["bf16_tflops"] == 2.0
+
+
+class _FakeNvml:
+    """Read-only NVML stand-in: two GPUs, the second one the benchmarked one,
+    its clock held at 1500 MHz by the power cap."""
+    NVML_CLOCK_SM = 1
+    nvmlClocksEventReasonHwSlowdown = 0x8
+    nvmlClocksEventReasonHwThermalSlowdown = 0x40
+    nvmlClocksEventReasonSwThermalSlowdown = 0x20
+    nvmlClocksEventReasonSwPowerCap = 0x4
+
+    class _Pci:
+        def __init__(self, bid):
+            self.busId = bid
+
+    def nvmlInit(self):
+        pass
+
+    def nvmlDeviceGetCount(self):
+        return 2
+
+    def nvmlDeviceGetHandleByIndex(self, i):
+        return i
+
+    def nvmlDeviceGetPciInfo(self, h):
+        return self._Pci([b"00000000:1A:00.0", b"00000000:1B:00.0"][h])
+
+    def nvmlDeviceGetClockInfo(self, h, kind):
+        assert h == 1 and kind == self.NVML_CLOCK_SM
+        return 1500
+
+    def nvmlDeviceGetMaxClockInfo(self, h, kind):
+        return 1965
+
+    def nvmlDeviceGetCurrentClocksEventReasons(self, h):
+        return self.nvmlClocksEventReasonSwPowerCap | 0x1  # 0x1 (idle) is not a reason the report keeps
+
+    def nvmlDeviceGetPowerUsage(self, h):
+        return 998000  # mW
+
+
+def test_clock_sampler_reads_the_benchmarked_gpu_through_nvml(monkeypatch):
+    import sys
+    import time
+    monkeypatch.setitem(sys.modules, "pynvml", _FakeNvml())
+    s = bench.ClockSampler("0000:1b:00")
+    s.start()
+    time.sleep(0.05)
+    c = s.stop()
+    assert c["samples"] >= 2 and c["sm_mhz"] == 1500.0 and c["sm_max_mhz"] == 1965.0
+    assert c["reasons"] == ["sw_power_cap"] and c["power_w_max"] == 998.0
+    assert "NVML" in c["source"]
