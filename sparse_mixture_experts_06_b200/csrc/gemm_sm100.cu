@@ -696,10 +696,23 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
             asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
         }
     }
-    // the set-up above overlaps the previous kernel's tail; offsets, the A
-    // rows and the tile counter are earlier kernels' outputs
-    pdl_wait();
-    pdl_trigger();
+    // The set-up above overlaps the previous kernel's tail.  The A rows, the
+    // tile counter and (for the down projection) the arrival counters are
+    // written by the kernel launched just before this one, so they are read
+    // only after pdl_wait().  Weight-streaming launches (kEarlyB) read the
+    // offsets before it: they come from a permutation kernel launched at
+    // least two launches earlier, and the previous kernel let this one start
+    // only after its own wait, i.e. after that kernel had completed and its
+    // writes were visible.  Their producer then issues the weight loads of
+    // its first tile's first stages (the weights are inputs no kernel of the
+    // layer writes) before it waits, so the HBM stream starts while the
+    // previous kernel finishes.
+    constexpr bool kEarlyB = (CG == 1 && RB == 32);
+    const bool early_producer = kEarlyB && warp == 0 && lane == 0;
+    if constexpr (!kEarlyB) {
+        pdl_wait();
+        pdl_trigger();
+    }
     if (threadIdx.x < p.E) {
         const int o0 = p.offsets[threadIdx.x], o1 = p.offsets[threadIdx.x + 1];
         const int split = o0 + ((o1 - o0) / 256) * 256;  // end of the whole 256-row blocks
@@ -709,6 +722,10 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
     tc_fence_before();
     if constexpr (CG == 2) cluster_sync_all(); else __syncthreads();
     tc_fence_after();
+    if (kEarlyB && !early_producer) {
+        pdl_wait();
+        pdl_trigger();
+    }
     const uint32_t tmem_base = *tmem_slot;
 
     const int total = count_tiles_rows(s_beg, s_end, p.E, p.n_tiles, C::kTileRows);
@@ -748,8 +765,30 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
             // The next tile's number is taken while the last STG stages of the
             // current tile are issued, so the atomic's latency is hidden.
             // (the odd CTA of a pair reads the even one's; a CTA beyond the
-            // active ones publishes the end at once)
-            int next = leader ? (takes_tiles ? atomicAdd(p.tile_counter, 1) : total) : -1;
+            // active ones publishes the end at once).  Weight-streaming
+            // launches take tile blockIdx.x first, without the counter (it is
+            // cleared by the previous kernel), and the counter's numbers
+            // after the first wave.
+            const int counter_base = kEarlyB ? active : 0;
+            int next = leader ? (takes_tiles ? (kEarlyB ? (int)blockIdx.x : atomicAdd(p.tile_counter, 1)) : total) : -1;
+            int pre = 0;  // stages of the first tile whose weight loads were issued before the wait
+            if constexpr (kEarlyB) {
+                if (next < total) {
+                    int e, mb, nb;
+                    decode_tile_rows(next, s_beg, s_end, p.E, p.n_tiles, C::kTileRows, p.m_group, e, mb, nb);
+                    const int rowB0 = e * p.b_rows_per_expert + nb * (MODE == kUp ? BN / 2 : BN);
+                    const int rowB1 = (MODE == kUp) ? rowB0 : rowB0 + BN / 2;
+                    pre = kblocks < STG ? kblocks : STG;
+                    for (int kb = 0; kb < pre; ++kb) {  // fresh stages: nothing to wait for
+                        const uint32_t fb = smem_u32(&full[kb]);
+                        mbar_arrive_expect_tx(fb, C::kABytes + C::kBBytes);
+                        tma_load_2d(smem_u32(sB + kb * C::kBBytes), &tmB0, fb, kb * BK, rowB0);
+                        tma_load_2d(smem_u32(sB + kb * C::kBBytes + C::kBHalf), &tmB1, fb, kb * BK, rowB1);
+                    }
+                }
+                pdl_wait();
+                pdl_trigger();
+            }
             for (uint32_t ti = 0; ok; ++ti) {
                 int tile;
                 if (leader) {
@@ -793,9 +832,15 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
                 }
                 const int kb_next = kblocks > STG ? kblocks - STG : 0;
                 for (int kb = 0; kb < kblocks; ++kb, ++it) {
-                    if (leader && kb == kb_next) next = atomicAdd(p.tile_counter, 1);
+                    if (leader && kb == kb_next) next = counter_base + atomicAdd(p.tile_counter, 1);
                     const uint32_t s = it % STG;
                     const uint32_t ph = (it / STG) & 1u;
+                    if constexpr (kEarlyB) {
+                        if (ti == 0 && kb < pre) {  // weights already on their way: the A rows only
+                            tma_load_2d(smem_u32(sA + s * A_TILE), &tmA, smem_u32(&full[s]), kb * BK, rowA);
+                            continue;
+                        }
+                    }
                     if (!wait_bounded_pair(smem_u32(&empty[s]), ph ^ 1u, abort_flag, p.err, peer_abort, p.wait_limit_ns)) { ok = false; break; }
                     const uint32_t fb = smem_u32(&full[s]);
                     if constexpr (CG == 1) {
