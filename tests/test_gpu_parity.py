@@ -273,6 +273,30 @@ def test_expert_blocks_at_tile_edges(cta_group, wide):
     assert_close(to64(y), y_ref, "bf16")
 
 
+@pytest.mark.parametrize("variant", [("2", "256", "128", "1"), ("1", "256", "128", "0"), ("1", "256", "32", "0")],
+                         ids=["pairs-512", "single-128", "single-32"])
+def test_large_expert_in_grouped_tile_order(variant):
+    """An expert whose rows span many more row blocks than one group of the
+    GEMMs' tile order (groups of about sqrt(2 x CTA pairs) 256-row blocks for
+    pairs, more for single-CTA tiles; 6000 rows = 23 pair blocks + a short
+    one, 47 + 1 single-CTA blocks of 128, 188 of 32), next to small and
+    ragged experts: moe_expert_ffn against the oracle on every token."""
+    force_variant(*variant)
+    sizes = [6000, 100, 333, 900]
+    E, d, f = len(sizes), 256, 512
+    T = sum(sizes)
+    s = synth.MoEShape("grouped", T, d, f, E, 1, "bf16")
+    t = device_inputs(s, 12)
+    rng = np.random.default_rng(6)
+    idx = rng.permutation(np.repeat(np.arange(E), sizes)).astype(np.int32).reshape(T, 1)
+    w = rng.uniform(0.25, 1.0, size=(T, 1)).astype(np.float32)
+    off, perm, inv = moe.moe_permute(torch.from_numpy(idx).cuda(), E)
+    y = moe.moe_expert_ffn(t["x"], t["W1"], t["W3"], t["W2"], off, perm, inv, torch.from_numpy(w).cuda())
+    h = host_copy(t)
+    y_ref, _, _ = oracle_rows(h, 1, np.arange(T), routing=(idx, w.astype(np.float64)))
+    assert_close(to64(y), y_ref, "bf16")
+
+
 @pytest.mark.parametrize("seed", range(1, 101))
 def test_tiny_fp32_many_seeds(seed):
     full_check(synth.CONFIGS["tiny"], seed)
