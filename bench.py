@@ -463,7 +463,11 @@ def e2e_leg(args, s, t, device, steps):
     the timed region; the library pipelines those copies with the compute of
     the neighbouring pieces (args.e2e_chunks per step, staging alternating
     across steps; x_ready, since the host tokens are ready at each call, and
-    y_async, with one moe_layer_forward_host_wait before the end event)."""
+    y_async, with one moe_layer_forward_host_wait before the end event).
+    All of every step's copies are inside the timed region, so the first
+    step's copy in and the last step's copy out, which have no neighbouring
+    compute to hide behind (~0.7 ms each at prefill over PCIe), add
+    ~1.4 ms / steps to the per-step time."""
     import torch
     import sparse_mixture_experts_06_b200 as moe
     x_h = t["x"].cpu().pin_memory()
@@ -664,7 +668,8 @@ def main():
     e_ms = max_over_ranks(e_ms, dist, device)
     if rank == 0:
         line["e2e"] = {"value": world * s.T / (e_ms * 1e-3), "unit": "tokens/s", "h2d_bytes_per_step": hb,
-                       "d2h_bytes_per_step": db, "ms_per_step": e_ms, "chunks": args.e2e_chunks,
+                       "d2h_bytes_per_step": db, "ms_per_step": e_ms, "steps": max(10, min(K, 100)),
+                       "chunks": args.e2e_chunks,
                        "path": "pinned host x -> moe_layer_forward_host (x_ready, y_async; each step's "
                                "copies pipelined with the compute of neighbouring pieces, %d per step) -> "
                                "pinned host y" % args.e2e_chunks}
