@@ -35,11 +35,12 @@ def restore_defaults():
     moe.moe_set_gemm_variant()
 
 
-@pytest.mark.parametrize("variant", [(1, 0, 128, 0), (2, 0, 0, 512), (2, 0, 0, 256)],
-                         ids=["single-cta", "pair-256x512", "pair-256x256"])
+@pytest.mark.parametrize("variant", [(1, 0, 128, 0), (1, 0, 32, 0), (2, 0, 0, 512), (2, 0, 0, 256)],
+                         ids=["single-cta", "single-cta-32-rows", "pair-256x512", "pair-256x256"])
 def test_pipeline_wait_bound_aborts_cleanly(variant):
-    # one expert (E = k = 1), 1024 rows: 4 pair row blocks or 8 single-CTA
-    # ones, several column tiles each
+    # one expert (E = k = 1), 1024 rows: 4 pair row blocks, or 8 (32) single-CTA
+    # ones of 128 (32) rows, several column tiles each; the 32-row tiles issue
+    # their first weight loads before the dependency wait
     s = synth.MoEShape("abort", 1024, 256, 1024, 1, 1, "bf16")
     t = device_inputs(s, 21)
     moe.moe_set_gemm_variant(*variant)
