@@ -237,9 +237,11 @@ unsigned int moe_device_errors(void);
 /* Per-stage device timing, for measurement: while enabled, every kernel the
  * library launches on the current device is bracketed by a pair of CUDA
  * events recorded on the launching stream (no synchronisation is added).
- * Stages: 0 router_topk, 1 permute, 2 gather, 3 up-projection GEMM (SwiGLU
- * epilogue), 4 down-projection GEMM (gate scaling and, on the bf16 path, the
- * combine), 5 combine (fp32 path), 6 fp32 expert kernels.  moe_profile_enable(1) clears and starts recording (up to 8192
+ * Stages: 0 router_topk (in a layer of up to 64 tokens and 256 assignments
+ * it also builds the permutation, and stage 1 has no launch), 1 permute,
+ * 2 gather, 3 up-projection GEMM (SwiGLU epilogue), 4 down-projection GEMM
+ * (gate scaling and, on the bf16 path, the combine), 5 combine (fp32 path),
+ * 6 fp32 expert kernels.  moe_profile_enable(1) clears and starts recording (up to 8192
  * launches), moe_profile_enable(0) stops.  moe_profile_read() waits for the
  * recorded events, writes per-stage total milliseconds and launch counts
  * for the first n stages, clears the record, and returns the number of

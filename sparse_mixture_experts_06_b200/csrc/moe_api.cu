@@ -427,16 +427,20 @@ int moe_layer_forward_ex(const void* x, const void* Wg, const void* W1, const vo
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     moe::Workspace w = moe::carve_workspace(workspace, T, d, f, E, k, bf16);
     cudaError_t e;
+    // chunked permutation: counts and scan ("permute" stage), then the
+    // stable scatter with the x row copies ("gather_rows" stage); a layer
+    // whose tokens fit one router cluster has the router permute as well
+    const bool chunked = moe::chunked_permute_fits(T * k, E);
+    const bool router_permutes = !chunked && moe::router_can_permute(T, k);
     {
         StageTimer tm(kRouter, s);
-        e = moe::launch_router_topk(x, Wg, T, d, E, k, bf16, w.topk_idx, w.topk_w, s);
+        moe::PermuteOut po;
+        if (router_permutes) po = moe::PermuteOut{w.offsets, w.perm, w.inv};
+        e = moe::launch_router_topk(x, Wg, T, d, E, k, bf16, w.topk_idx, w.topk_w, s, po);
         tm.done(s);
     }
     if (e != cudaSuccess) return cuda_fail(e, "router_topk");
-    // chunked permutation: counts and scan ("permute" stage), then the
-    // stable scatter with the x row copies ("gather_rows" stage)
-    const bool chunked = moe::chunked_permute_fits(T * k, E);
-    {
+    if (!router_permutes) {
         StageTimer tm(kPermute, s);
         e = chunked ? moe::launch_chunk_count_scan(w.topk_idx, T * k, E, w.chunk_base, w.offsets, s)
                     : moe::launch_permute(w.topk_idx, T * k, E, w.offsets, w.perm, w.inv, s);

@@ -77,8 +77,19 @@ struct Workspace {
 Workspace carve_workspace(void* base, int T, int d, int f, int E, int k, bool bf16);
 
 // ---- launchers (return cudaError_t of the launch) ------------------------
+// The router of a layer whose tokens fit one router cluster (up to 64
+// tokens and 256 assignments: router_can_permute) also writes the expert
+// permutation (offsets, perm, inv; the same bits as launch_permute) when
+// `po` names its buffers, which saves the permutation's launch.
+struct PermuteOut {
+    int32_t* offsets = nullptr;
+    int32_t* perm = nullptr;
+    int32_t* inv = nullptr;
+};
+bool router_can_permute(int T, int k);
 cudaError_t launch_router_topk(const void* x, const void* Wg, int T, int d, int E, int k,
-                               bool bf16, int32_t* idx, float* w, cudaStream_t s);
+                               bool bf16, int32_t* idx, float* w, cudaStream_t s,
+                               const PermuteOut& po = PermuteOut{});
 cudaError_t launch_permute(const int32_t* idx, int n, int E, int32_t* offsets, int32_t* perm,
                            int32_t* inv, cudaStream_t s);
 // The layer's permutation in two launches: count_scan (one block: per-chunk

@@ -104,10 +104,50 @@ __device__ __forceinline__ void dmma(double& d0, double& d1, double a, double b)
         : "d"(a), "d"(b));
 }
 
+// The layer's expert permutation for a layer whose tokens fit one cluster
+// (T <= kTokBlock, n = T*k <= kFusedPermute assignments), done by CTA 0
+// after every CTA's indices are visible: expert counts, their exclusive
+// scan (offsets), and each assignment's place in its expert's block in
+// increasing assignment id (the stable order of permute_kernel; the same
+// bits).  One thread per assignment; smem is the CTA's scratch.
+constexpr int kFusedPermute = kWarps * 32;
+
+__device__ __forceinline__ void permute_in_cta(const int32_t* idx, int n, int E, int32_t* offsets,
+                                               int32_t* perm, int32_t* inv, int* smem) {
+    int* s_idx = smem;                  // [kFusedPermute]
+    int* s_cnt = s_idx + kFusedPermute;  // [kMaxExperts]
+    int* s_off = s_cnt + kMaxExperts;    // [kMaxExperts]
+    const int q = threadIdx.x;
+    if (q < kMaxExperts) s_cnt[q] = 0;
+    if (q < n) s_idx[q] = __ldcg(idx + q);  // written by other CTAs of the cluster
+    __syncthreads();
+    if (q < n) atomicAdd(&s_cnt[s_idx[q]], 1);
+    __syncthreads();
+    if (q == 0) {
+        int run = 0;
+        for (int e = 0; e < E; ++e) {
+            s_off[e] = run;
+            offsets[e] = run;
+            run += s_cnt[e];
+        }
+        offsets[E] = run;
+    }
+    __syncthreads();
+    if (q < n) {
+        const int e = s_idx[q];
+        int r = 0;
+        for (int p = 0; p < q; ++p) r += s_idx[p] == e ? 1 : 0;
+        const int pos = s_off[e] + r;
+        perm[pos] = q;
+        inv[q] = pos;
+    }
+}
+
 template <bool BF16>
 __global__ void __launch_bounds__(kWarps * 32, BF16 ? 4 : 2)  // bf16: 64 registers, 4 CTAs per SM
 router_topk_kernel(const void* __restrict__ x, const void* __restrict__ Wg, int T, int d, int E, int k,
-                   int32_t* __restrict__ idx_out, float* __restrict__ w_out) {
+                   int32_t* __restrict__ idx_out, float* __restrict__ w_out, int32_t* __restrict__ offsets,
+                   int32_t* __restrict__ perm, int32_t* __restrict__ inv) {
     extern __shared__ __align__(16) unsigned char smem_raw[];
     pdl_wait();     // x may be the previous kernel's output (a layer stack)
     pdl_trigger();
@@ -254,11 +294,15 @@ router_topk_kernel(const void* __restrict__ x, const void* __restrict__ Wg, int 
         if (live && sl == 0)
             for (int j = 0; j < k; ++j) wo[j] = wo[j] / sum;
     }
+    if (perm != nullptr) {  // one cluster holds every token: the permutation here too
+        cluster.sync();     // every CTA's indices are written and visible in the cluster
+        if (rank == 0) permute_in_cta(idx_out, T * k, E, offsets, perm, inv, reinterpret_cast<int*>(wfrag));
+    }
 }
 
 template <bool BF16>
 cudaError_t launch_impl(const void* x, const void* Wg, int T, int d, int E, int k, int32_t* idx, float* w,
-                        cudaStream_t s) {
+                        const PermuteOut& po, cudaStream_t s) {
     static bool attr_done[64] = {false};
     int dev = 0;
     cudaGetDevice(&dev);
@@ -282,15 +326,19 @@ cudaError_t launch_impl(const void* x, const void* Wg, int T, int d, int E, int 
     cfg.stream = s;
     cfg.attrs = attr;
     cfg.numAttrs = 2;
-    return cudaLaunchKernelEx(&cfg, router_topk_kernel<BF16>, x, Wg, T, d, E, k, idx, w);
+    const bool fuse = po.perm != nullptr && router_can_permute(T, k);
+    return cudaLaunchKernelEx(&cfg, router_topk_kernel<BF16>, x, Wg, T, d, E, k, idx, w,
+                              fuse ? po.offsets : nullptr, fuse ? po.perm : nullptr, fuse ? po.inv : nullptr);
 }
 
 }  // namespace
 
+bool router_can_permute(int T, int k) { return T >= 1 && T <= kTokBlock && (long long)T * k <= kFusedPermute; }
+
 cudaError_t launch_router_topk(const void* x, const void* Wg, int T, int d, int E, int k,
-                               bool bf16, int32_t* idx, float* w, cudaStream_t s) {
-    return bf16 ? launch_impl<true>(x, Wg, T, d, E, k, idx, w, s)
-                : launch_impl<false>(x, Wg, T, d, E, k, idx, w, s);
+                               bool bf16, int32_t* idx, float* w, cudaStream_t s, const PermuteOut& po) {
+    return bf16 ? launch_impl<true>(x, Wg, T, d, E, k, idx, w, po, s)
+                : launch_impl<false>(x, Wg, T, d, E, k, idx, w, po, s);
 }
 
 }  // namespace moe

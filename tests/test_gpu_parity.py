@@ -174,7 +174,10 @@ def workspace_routing_views(ws, T, E, k):
 
 
 @pytest.mark.parametrize("shape", [
-    synth.MoEShape("perm-decode", 32, 256, 256, 8, 2, "bf16"),      # one-block permutation (few assignments)
+    synth.MoEShape("perm-decode", 32, 256, 256, 8, 2, "bf16"),      # the router permutes (one cluster)
+    synth.MoEShape("perm-router-256", 64, 128, 128, 16, 4, "bf16"),  # the router's largest: 256 assignments
+    synth.MoEShape("perm-router-T1", 1, 64, 128, 8, 2, "bf16"),
+    synth.MoEShape("perm-one-block", 65, 128, 128, 8, 2, "bf16"),    # one-block permutation kernel
     synth.MoEShape("perm-ragged", 1100, 128, 128, 8, 2, "bf16"),     # 2200 assignments: ragged last chunk
     synth.MoEShape("perm-4100", 4100, 128, 128, 8, 2, "bf16"),
     synth.MoEShape("perm-E64k8", 300, 128, 128, 64, 8, "bf16"),
@@ -182,8 +185,10 @@ def workspace_routing_views(ws, T, E, k):
     synth.MoEShape("perm-fallback", 50000, 64, 64, 64, 1, "bf16"),  # E x chunks above the scan's shared memory
 ], ids=lambda s: s.name)
 def test_layer_permutation_matches_the_stable_sort(shape):
-    """The permutation the layer builds for itself (chunked count/scan +
-    scatter, or the one-block kernel when E x chunks is too large) equals
+    """The permutation the layer builds for itself (in the router's cluster
+    up to 64 tokens and 256 assignments, else chunked count/scan + scatter,
+    or the one-block kernel for few assignments or when E x chunks is too
+    large) equals
     the oracle's stable counting sort of the router's choices, bit for bit,
     and the layer's output on sampled tokens matches the oracle."""
     t = device_inputs(shape, 31)
@@ -392,11 +397,14 @@ def test_entry_points_agree_and_are_deterministic():
     moe.moe_release_workspace()
 
 
-@pytest.mark.parametrize("T", [100, 2304], ids=["one-block-permutation", "chunked-permutation"])
-def test_bf16_layer_runs_five_kernels(T):
+@pytest.mark.parametrize("T,kernels", [(32, 4), (100, 5), (2304, 5)],
+                         ids=["router-permutes", "one-block-permutation", "chunked-permutation"])
+def test_bf16_layer_kernels(T, kernels):
     """The bf16 layer is router, permutation (count/scan or one block), row
     scatter or gather, up-projection GEMM and down-projection GEMM: the
-    combine runs in the down GEMM's epilogue, with no kernel of its own."""
+    combine runs in the down GEMM's epilogue, with no kernel of its own.  Up
+    to 64 tokens (one router cluster) the router writes the permutation too:
+    four kernels."""
     s = synth.MoEShape("launches", T, 256, 512, 8, 2, "bf16")
     t = device_inputs(s, 3)
     ws = torch.empty(moe.moe_workspace_size(T, s.d, s.f, s.E, s.k, 0), dtype=torch.uint8, device="cuda")
@@ -410,7 +418,8 @@ def test_bf16_layer_runs_five_kernels(T):
     moe.moe_profile_enable(False)
     n = {name: cnt for name, (_, cnt) in prof.items()}
     assert n["combine"] == 0 and n["down_combine_gemm"] == 1 and n["up_swiglu_gemm"] == 1
-    assert sum(n.values()) == 5, n
+    assert sum(n.values()) == kernels, n
+    assert n["permute"] == (0 if kernels == 4 else 1)
     h = host_copy(t)
     y_ref, _, _ = oracle_rows(h, 2, np.arange(T))
     assert_close(to64(y), y_ref, "bf16")
