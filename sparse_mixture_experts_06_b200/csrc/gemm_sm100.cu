@@ -1029,71 +1029,107 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
             const int g_lo = sub ? (G + 1) / 2 : 0, g_hi = sub ? G : (G + 1) / 2;
             (void)g_lo;
             (void)g_hi;
+            bool released = false;  // this warp's TMEM arrival for the tile done
             if constexpr (MODE == kUp) {
-                int unit = 0;  // output units of the tile so far (this warp takes unit % 2 == sub)
-#pragma unroll 1
-                for (int h = 0; h < NH; ++h) {
-                    const uint32_t tacc = t_lane + acc * C::kTileN + h * BN;
-                    const int hb = nb * (NH * BN / 2) + h * (BN / 2);  // first hidden unit of MMA h
-                    __nv_bfloat16* hrow = p.h + (size_t)row * p.n_out;
-                    // 64-unit segments: hidden units c64 .. c64+63 of the tile have
-                    // a at TMEM columns acol .. acol+63 and b at acol+bdelta ...
-                    //   single CTA: a = columns 0 .. BN/2-1, b = BN/2 .. BN-1;
-                    //   pair, full: [a 64 | b 64] per CTA half of B, two halves;
-                    //   pair, short: one half per lane group, at columns 0-127.
-                    const int nseg = (CG == 1) ? BN / 128 : (shrt ? 1 : 2);
-                    const int bdelta = (CG == 1) ? BN / 2 : 64;
-#pragma unroll 1
-                    for (int seg = 0; seg < nseg; ++seg) {
-                        if ((unit++ & 1) != sub) continue;
-                        const int c64 = (shrt ? colhalf : seg) * 64;        // hidden offset in the tile
-                        const int acol = (CG == 1) ? seg * 64 : (shrt ? 0 : seg * 128);
-#pragma unroll 1
-                        for (int half = 0; half < 2; ++half) {
-                            const int c = c64 + half * 32;
-                            uint32_t a[32], b[32];
-                            tmem_ld32(tacc + acol + half * 32, a);
-                            tmem_ld32(tacc + acol + half * 32 + bdelta, b);
-                            tmem_wait_ld();
-                            uint4 pk[4];
+                // The tile's output units (64-hidden-unit segments over all MMA
+                // parts, part-major); this warp takes units sub, sub + 2, ...,
+                // each as two 32-unit halves ("items", at most 4).  64-unit
+                // segments: hidden units c64 .. c64+63 of the tile have a at TMEM
+                // columns acol .. acol+63 and b at acol+bdelta ...
+                //   single CTA: a = columns 0 .. BN/2-1, b = BN/2 .. BN-1;
+                //   pair, full: [a 64 | b 64] per CTA half of B, two halves;
+                //   pair, short: one half per lane group, at columns 0-127.
+                // The TMEM loads of item i+1 are issued before item i's math, and
+                // the warp releases the accumulator after its last item's loads
+                // have landed, before that item's math and stores.
+                const int nseg = (CG == 1) ? BN / 128 : (shrt ? 1 : 2);
+                const int n_items = 2 * ((NH * nseg - sub + 1) / 2);
+                const int bdelta = (CG == 1) ? BN / 2 : 64;
+                __nv_bfloat16* hrow = p.h + (size_t)row * p.n_out;
+                auto item_cols = [&](int it, uint32_t& ta, int& hcol) {
+                    const int u = sub + 2 * (it >> 1);
+                    const int h = u / nseg, seg = u - h * nseg, half = it & 1;
+                    const int c64 = (shrt ? colhalf : seg) * 64;  // hidden offset in MMA part h
+                    const int acol = (CG == 1) ? seg * 64 : (shrt ? 0 : seg * 128);
+                    ta = t_lane + acc * C::kTileN + h * BN + acol + half * 32;
+                    hcol = nb * (NH * BN / 2) + h * (BN / 2) + c64 + half * 32;  // first hidden unit
+                };
+                constexpr int kMaxItems = (NH == 2) ? 4 : 2;
+                uint32_t ra[2][32], rb[32];
+                if (n_items > 0) {
+                    uint32_t ta;
+                    int hc;
+                    item_cols(0, ta, hc);
+                    tmem_ld32(ta, ra[0]);
+                    tmem_ld32(ta + bdelta, rb);
+                }
 #pragma unroll
-                            for (int g = 0; g < 4; ++g) {
-                                pk[g].x = pack_bf16x2(silu_mul(__uint_as_float(a[g * 8 + 0]), __uint_as_float(b[g * 8 + 0])),
-                                                      silu_mul(__uint_as_float(a[g * 8 + 1]), __uint_as_float(b[g * 8 + 1])));
-                                pk[g].y = pack_bf16x2(silu_mul(__uint_as_float(a[g * 8 + 2]), __uint_as_float(b[g * 8 + 2])),
-                                                      silu_mul(__uint_as_float(a[g * 8 + 3]), __uint_as_float(b[g * 8 + 3])));
-                                pk[g].z = pack_bf16x2(silu_mul(__uint_as_float(a[g * 8 + 4]), __uint_as_float(b[g * 8 + 4])),
-                                                      silu_mul(__uint_as_float(a[g * 8 + 5]), __uint_as_float(b[g * 8 + 5])));
-                                pk[g].w = pack_bf16x2(silu_mul(__uint_as_float(a[g * 8 + 6]), __uint_as_float(b[g * 8 + 6])),
-                                                      silu_mul(__uint_as_float(a[g * 8 + 7]), __uint_as_float(b[g * 8 + 7])));
-                            }
-                            if (box_ok) {
-                                if (half == 0) {
-                                    // the buffer's previous store has read it (waited for
-                                    // only now, so the wait overlaps the loads and the math)
-                                    if (lane == 0) bulk_wait_read_all();
-                                    __syncwarp();
-                                }
-#pragma unroll
-                                for (int g = 0; g < 4; ++g)
-                                    st_shared_v4(buf + lane * 128 + ((((half * 4 + g) ^ (lane & 7))) << 4), pk[g]);
-                            } else if (valid) {
-                                const int col0 = hb + c;
-#pragma unroll
-                                for (int g = 0; g < 4; ++g)
-                                    if (col0 + g * 8 < p.n_out) *reinterpret_cast<uint4*>(hrow + col0 + g * 8) = pk[g];
-                            }
+                for (int it = 0; it < kMaxItems; ++it) {
+                    if (it >= n_items) break;  // warp-uniform
+                    uint32_t ta;
+                    int hc;
+                    item_cols(it, ta, hc);
+                    tmem_wait_ld();
+                    if (it + 1 < n_items) {
+                        uint32_t tn;
+                        int hn;
+                        item_cols(it + 1, tn, hn);
+                        tmem_ld32(tn, ra[(it + 1) & 1]);
+                    } else {
+                        tc_fence_before();
+                        __syncwarp();
+                        if (lane == 0) {
+                            if constexpr (CG == 1) mbar_arrive(smem_u32(&tempty[acc]));
+                            else mbar_arrive_cluster(tempty_leader0 + acc * (uint32_t)sizeof(uint64_t));
                         }
-                        if (box_ok) {
+                        released = true;
+                    }
+                    const uint32_t* a = ra[it & 1];
+                    const uint32_t* b = rb;
+                    uint4 pk[4];
+#pragma unroll
+                    for (int g = 0; g < 4; ++g) {
+                        pk[g].x = pack_bf16x2(silu_mul(__uint_as_float(a[g * 8 + 0]), __uint_as_float(b[g * 8 + 0])),
+                                              silu_mul(__uint_as_float(a[g * 8 + 1]), __uint_as_float(b[g * 8 + 1])));
+                        pk[g].y = pack_bf16x2(silu_mul(__uint_as_float(a[g * 8 + 2]), __uint_as_float(b[g * 8 + 2])),
+                                              silu_mul(__uint_as_float(a[g * 8 + 3]), __uint_as_float(b[g * 8 + 3])));
+                        pk[g].z = pack_bf16x2(silu_mul(__uint_as_float(a[g * 8 + 4]), __uint_as_float(b[g * 8 + 4])),
+                                              silu_mul(__uint_as_float(a[g * 8 + 5]), __uint_as_float(b[g * 8 + 5])));
+                        pk[g].w = pack_bf16x2(silu_mul(__uint_as_float(a[g * 8 + 6]), __uint_as_float(b[g * 8 + 6])),
+                                              silu_mul(__uint_as_float(a[g * 8 + 7]), __uint_as_float(b[g * 8 + 7])));
+                    }
+                    if (it + 1 < n_items) {  // b of the next item, now that this one's b is consumed
+                        uint32_t tn;
+                        int hn;
+                        item_cols(it + 1, tn, hn);
+                        tmem_ld32(tn + bdelta, rb);
+                    }
+                    const int half = it & 1;
+                    if (box_ok) {
+                        if (half == 0) {
+                            // the buffer's previous store has read it (waited for
+                            // only now, so the wait overlaps the loads and the math)
+                            if (lane == 0) bulk_wait_read_all();
+                            __syncwarp();
+                        }
+#pragma unroll
+                        for (int g = 0; g < 4; ++g)
+                            st_shared_v4(buf + lane * 128 + ((((half * 4 + g) ^ (lane & 7))) << 4), pk[g]);
+                        if (half == 1) {
                             fence_proxy_async_smem();
                             __syncwarp();
                             if (lane == 0) {
                                 // a box wholly past the last column is not stored; the
                                 // (empty) group keeps one group per staged box
-                                if (hb + c64 < p.n_out) tma_store_2d(&tmOut, buf, hb + c64, wrow0);
+                                const int c64 = hc - 32;
+                                if (c64 < p.n_out) tma_store_2d(&tmOut, buf, c64, wrow0);
                                 bulk_commit();
                             }
                         }
+                    } else if (valid) {
+#pragma unroll
+                        for (int g = 0; g < 4; ++g)
+                            if (hc + g * 8 < p.n_out) *reinterpret_cast<uint4*>(hrow + hc + g * 8) = pk[g];
                     }
                 }
             } else {
@@ -1140,11 +1176,13 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
                     }
                 }
             }
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) {
-                if constexpr (CG == 1) mbar_arrive(smem_u32(&tempty[acc]));
-                else mbar_arrive_cluster(tempty_leader0 + acc * (uint32_t)sizeof(uint64_t));
+            if (!released) {
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) {
+                    if constexpr (CG == 1) mbar_arrive(smem_u32(&tempty[acc]));
+                    else mbar_arrive_cluster(tempty_leader0 + acc * (uint32_t)sizeof(uint64_t));
+                }
             }
             if constexpr (MODE == kDown) {
                 // Count the parked groups (release: the park stores are complete
