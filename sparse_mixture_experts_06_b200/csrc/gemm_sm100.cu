@@ -427,14 +427,26 @@ __device__ __forceinline__ int count_tiles_rows(const int* s_beg, const int* s_e
     return total;
 }
 
+// An expert's last row block is short when it holds at most 128 rows (pair
+// tiles: an M = 128 MMA).
+__device__ __forceinline__ bool short_last_block(int rows, int mt, int rows_per_tile) {
+    return mt > 0 && rows - (mt - 1) * rows_per_tile <= 128;
+}
+
 // Tile number -> (expert, row block, column block): experts in order; inside
 // an expert, groups of G row blocks (the last one may be shorter); inside a
-// group, column block major and row block fastest.
+// group, column block major and row block fastest.  With short_last (the
+// down projection's pair tiles) the short last row blocks are taken out of
+// that order and numbered after all other tiles, expert by expert, so the
+// shorter tiles come last and even out the CTA pairs' finishing times.
 __device__ __forceinline__ void decode_tile_rows(int tile, const int* s_beg, const int* s_end, int E, int n_tiles,
-                                                 int rows_per_tile, int G, int& e, int& m_blk, int& n_blk) {
+                                                 int rows_per_tile, int G, bool short_last, int& e, int& m_blk,
+                                                 int& n_blk) {
     int base = 0;
     for (e = 0; e < E; ++e) {
-        const int mt = (s_end[e] - s_beg[e] + rows_per_tile - 1) / rows_per_tile;
+        const int rows = s_end[e] - s_beg[e];
+        int mt = (rows + rows_per_tile - 1) / rows_per_tile;
+        if (short_last && short_last_block(rows, mt, rows_per_tile)) --mt;
         const int tiles = mt * n_tiles;
         if (tile < base + tiles) {
             const int local = tile - base;
@@ -447,6 +459,19 @@ __device__ __forceinline__ void decode_tile_rows(int tile, const int* s_beg, con
             return;
         }
         base += tiles;
+    }
+    if (short_last) {
+        for (e = 0; e < E; ++e) {
+            const int rows = s_end[e] - s_beg[e];
+            const int mt = (rows + rows_per_tile - 1) / rows_per_tile;
+            if (!short_last_block(rows, mt, rows_per_tile)) continue;
+            if (tile < base + n_tiles) {
+                m_blk = mt - 1;
+                n_blk = tile - base;
+                return;
+            }
+            base += n_tiles;
+        }
     }
     e = E - 1; m_blk = 0; n_blk = 0;  // not reached for tile < total
 }
@@ -729,6 +754,9 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
     const uint32_t tmem_base = *tmem_slot;
 
     const int total = count_tiles_rows(s_beg, s_end, p.E, p.n_tiles, C::kTileRows);
+    // the down projection's short pair tiles last (the up projection keeps
+    // them next to the full tiles that share their weight slices in L2)
+    constexpr bool kShortLast = (MODE == kDown && CG == 2);
     // Weight-streaming tiles (32 token rows: HBM-bound) in even waves: with
     // w = ceil(total / grid) waves, only ceil(total / w) CTAs take tiles, so
     // no last wave of a few tiles streams alone while the others idle (at
@@ -775,7 +803,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
             if constexpr (kEarlyB) {
                 if (next < total) {
                     int e, mb, nb;
-                    decode_tile_rows(next, s_beg, s_end, p.E, p.n_tiles, C::kTileRows, p.m_group, e, mb, nb);
+                    decode_tile_rows(next, s_beg, s_end, p.E, p.n_tiles, C::kTileRows, p.m_group, kShortLast, e, mb, nb);
                     const int rowB0 = e * p.b_rows_per_expert + nb * (MODE == kUp ? BN / 2 : BN);
                     const int rowB1 = (MODE == kUp) ? rowB0 : rowB0 + BN / 2;
                     pre = kblocks < STG ? kblocks : STG;
@@ -812,7 +840,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
                 }
                 if (tile < 0) break;
                 int e, mb, nb;
-                decode_tile_rows(tile, s_beg, s_end, p.E, p.n_tiles, C::kTileRows, p.m_group, e, mb, nb);
+                decode_tile_rows(tile, s_beg, s_end, p.E, p.n_tiles, C::kTileRows, p.m_group, kShortLast, e, mb, nb);
                 const int start = s_beg[e] + mb * C::kTileRows;
                 const bool shrt = (CG == 2) && short_pair_tile(start, min(s_end[e], start + C::kTileRows));
                 const int rowA = start + (int)rank * (shrt ? 64 : 128);
@@ -901,7 +929,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
                 uint32_t idesc = C::kIdesc;
                 if constexpr (CG == 2) {
                     int e, mb, nb;
-                    decode_tile_rows(tile, s_beg, s_end, p.E, p.n_tiles, C::kTileRows, p.m_group, e, mb, nb);
+                    decode_tile_rows(tile, s_beg, s_end, p.E, p.n_tiles, C::kTileRows, p.m_group, kShortLast, e, mb, nb);
                     const int start = s_beg[e] + mb * C::kTileRows;
                     if (short_pair_tile(start, min(s_end[e], start + C::kTileRows))) idesc = C::kIdescShort;
                 }
@@ -970,7 +998,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
             if (lane == 0) release_tile(tcount);
             if (tile < 0) break;
             int e, mb, nb;
-            decode_tile_rows(tile, s_beg, s_end, p.E, p.n_tiles, C::kTileRows, p.m_group, e, mb, nb);
+            decode_tile_rows(tile, s_beg, s_end, p.E, p.n_tiles, C::kTileRows, p.m_group, kShortLast, e, mb, nb);
             const uint32_t acc = tcount % C::kNAcc;
             const uint32_t use = tcount / C::kNAcc;
             const int start = s_beg[e] + mb * C::kTileRows;
