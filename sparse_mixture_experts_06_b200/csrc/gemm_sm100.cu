@@ -725,10 +725,11 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
     // tile counter and (for the down projection) the arrival counters are
     // written by the kernel launched just before this one, so they are read
     // only after pdl_wait().  Weight-streaming launches (kEarlyB) read the
-    // offsets before it: they come from a permutation kernel launched at
-    // least two launches earlier, and the previous kernel let this one start
-    // only after its own wait, i.e. after that kernel had completed and its
-    // writes were visible.  Their producer then issues the weight loads of
+    // offsets before it: they come from the kernel that built the
+    // permutation (the permutation kernels, or the router of a small
+    // layer), launched at least two launches earlier, and the previous
+    // kernel let this one start only after its own wait, i.e. after that
+    // kernel had completed and its writes were visible.  Their producer then issues the weight loads of
     // its first tile's first stages (the weights are inputs no kernel of the
     // layer writes) before it waits, so the HBM stream starts while the
     // previous kernel finishes.
