@@ -518,3 +518,24 @@ def test_skewed_full_shape(mixtral_weights):
     _, counts = big_check("skewed", mixtral_weights, 256)
     share = counts / counts.sum()
     assert abs(share[0] - 0.35) < 0.005 and (np.diff(share) < 0).all()
+
+
+def test_many_tokens_small_widths():
+    """65536 tokens with the skewed router (hottest expert ~35 %: ~45 000
+    rows, 180 pair row blocks, several groups of the tile order) at small
+    widths: 2048 permutation chunks, 1024 router clusters, the combine's
+    arrival counters for every token; routing and permutation checked on
+    every token, outputs on a stratified sample."""
+    s = synth.MoEShape("many", 65536, 128, 256, 8, 2, "bf16", skew=True)
+    t = device_inputs(s, 41)
+    y = run_layer(t, s.k)
+    idx_g, w_g = moe.moe_router_topk(t["x"], t["Wg"], s.k)
+    off_g, perm_g, inv_g = moe.moe_permute(idx_g, s.E)
+    torch.cuda.synchronize()
+    h = host_copy(t)
+    idx_o, _, _ = check_routing(idx_g.cpu().numpy(), w_g.cpu().numpy(), f64(h["x"]), f64(h["Wg"]), s.k)
+    off, perm, _ = check_permutation(off_g.cpu().numpy(), perm_g.cpu().numpy(), inv_g.cpu().numpy(), idx_o, s.E)
+    assert np.diff(off).max() > 12 * 256 * 2  # the hottest expert spans several groups of row blocks
+    toks = stratified_tokens(off, perm, s.k, 512)
+    y_ref, _, _ = oracle_rows(h, s.k, toks)
+    assert_close(to64(y)[toks], y_ref, "bf16")
