@@ -102,7 +102,7 @@ Workspace carve_workspace(void* base, int T, int d, int f, int E, int k, bool bf
     w.tile_counters = reinterpret_cast<int32_t*>(take(kTileCounters * 4));
     w.arrivals_bytes = align256((size_t)T * ((d + kCombineCols - 1) / kCombineCols) * 4);
     w.arrivals = reinterpret_cast<unsigned int*>(take(w.arrivals_bytes));
-    w.chunk_base = reinterpret_cast<int32_t*>(take((size_t)E * ((n + kChunkA - 1) / kChunkA) * 4));
+    w.chunk_counts = reinterpret_cast<int32_t*>(take((size_t)E * ((n + kChunkA - 1) / kChunkA) * 4));
     w.bytes = off;
     return w;
 }
@@ -427,29 +427,31 @@ int moe_layer_forward_ex(const void* x, const void* Wg, const void* W1, const vo
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     moe::Workspace w = moe::carve_workspace(workspace, T, d, f, E, k, bf16);
     cudaError_t e;
-    // chunked permutation: counts and scan ("permute" stage), then the
-    // stable scatter with the x row copies ("gather_rows" stage); a layer
-    // whose tokens fit one router cluster has the router permute as well
+    // The permutation: from 2048 assignments the router writes the
+    // per-(expert, chunk) counts and the scatter ("gather_rows" stage) derives
+    // the rows, writes perm / inv and copies the x rows; a layer whose tokens
+    // fit one router cluster has the router permute outright; otherwise the
+    // one-block permutation ("permute" stage) and the row gather run.
     const bool chunked = moe::chunked_permute_fits(T * k, E);
     const bool router_permutes = !chunked && moe::router_can_permute(T, k);
     {
         StageTimer tm(kRouter, s);
-        moe::PermuteOut po;
-        if (router_permutes) po = moe::PermuteOut{w.offsets, w.perm, w.inv};
-        e = moe::launch_router_topk(x, Wg, T, d, E, k, bf16, w.topk_idx, w.topk_w, s, po);
+        moe::RouterOut ro;
+        if (router_permutes) ro = moe::RouterOut{w.offsets, w.perm, w.inv, nullptr};
+        if (chunked) ro = moe::RouterOut{nullptr, nullptr, nullptr, w.chunk_counts};
+        e = moe::launch_router_topk(x, Wg, T, d, E, k, bf16, w.topk_idx, w.topk_w, s, ro);
         tm.done(s);
     }
     if (e != cudaSuccess) return cuda_fail(e, "router_topk");
-    if (!router_permutes) {
+    if (!router_permutes && !chunked) {
         StageTimer tm(kPermute, s);
-        e = chunked ? moe::launch_chunk_count_scan(w.topk_idx, T * k, E, w.chunk_base, w.offsets, s)
-                    : moe::launch_permute(w.topk_idx, T * k, E, w.offsets, w.perm, w.inv, s);
+        e = moe::launch_permute(w.topk_idx, T * k, E, w.offsets, w.perm, w.inv, s);
         tm.done(s);
+        if (e != cudaSuccess) return cuda_fail(e, "permute");
     }
-    if (e != cudaSuccess) return cuda_fail(e, "permute");
     if (chunked) {
         StageTimer tm(kGather, s);
-        e = moe::launch_chunk_scatter(w.topk_idx, T * k, E, k, w.chunk_base, w.perm, w.inv,
+        e = moe::launch_chunk_scatter(w.topk_idx, T * k, E, k, w.chunk_counts, w.offsets, w.perm, w.inv,
                                       bf16 ? static_cast<const __nv_bfloat16*>(x) : nullptr, d,
                                       bf16 ? static_cast<__nv_bfloat16*>(w.x_perm) : nullptr, zero_args(w), s);
         tm.done(s);

@@ -70,39 +70,43 @@ struct Workspace {
     unsigned int* arrivals;  // [T, ceil(d / kCombineCols)] slot arrivals of the fused combine, zeroed
                              // with the tile counters
     size_t arrivals_bytes;   // bytes of the arrivals region (a multiple of 256)
-    int32_t* chunk_base;     // [E * ceil(T*k / kChunkA)] first row of each (expert, chunk)
+    int32_t* chunk_counts;   // [E * ceil(T*k / kChunkA)] assignments of each (expert, chunk)
     size_t bytes;
 };
 
 Workspace carve_workspace(void* base, int T, int d, int f, int E, int k, bool bf16);
 
 // ---- launchers (return cudaError_t of the launch) ------------------------
-// The router of a layer whose tokens fit one router cluster (up to 64
-// tokens and 256 assignments: router_can_permute) also writes the expert
-// permutation (offsets, perm, inv; the same bits as launch_permute) when
-// `po` names its buffers, which saves the permutation's launch.
-struct PermuteOut {
+// What the layer's router writes besides the indices and weights:
+// - a layer whose tokens fit one router cluster (up to 64 tokens and 256
+//   assignments: router_can_permute) gets the whole expert permutation
+//   (offsets, perm, inv; the same bits as launch_permute), which saves the
+//   permutation's launch;
+// - a chunked layer (chunked_permute_fits) gets chunk_counts[e * nch + c],
+//   the assignments of 64-assignment chunk c to expert e (a router cluster
+//   covers exactly k chunks), for launch_chunk_scatter.
+struct RouterOut {
     int32_t* offsets = nullptr;
     int32_t* perm = nullptr;
     int32_t* inv = nullptr;
+    int32_t* chunk_counts = nullptr;
 };
 bool router_can_permute(int T, int k);
 cudaError_t launch_router_topk(const void* x, const void* Wg, int T, int d, int E, int k,
                                bool bf16, int32_t* idx, float* w, cudaStream_t s,
-                               const PermuteOut& po = PermuteOut{});
+                               const RouterOut& ro = RouterOut{});
 cudaError_t launch_permute(const int32_t* idx, int n, int E, int32_t* offsets, int32_t* perm,
                            int32_t* inv, cudaStream_t s);
-// The layer's permutation in two launches: count_scan (one block: per-chunk
-// expert counts, their scan into chunk_base and offsets), then scatter (one
-// block per chunk: ranks, writes perm / inv and, if x_perm is not null,
-// copies the x rows).  Same results as launch_permute followed by
-// launch_gather_rows_bf16, whose work it replaces, including the clearing
-// of `z`.  Only when chunked_permute_fits(n, E).
+// The layer's permutation from 2048 assignments (chunked_permute_fits):
+// the router writes the per-(expert, 64-assignment chunk) counts
+// (RouterOut::chunk_counts), then the scatter (one block per chunk) derives
+// each chunk's first rows and the offsets, ranks the chunk stably, writes
+// perm / inv and, if x_perm is not null, copies the x rows.  Same results as
+// launch_permute followed by launch_gather_rows_bf16, whose work it
+// replaces, including the clearing of `z`.
 bool chunked_permute_fits(int n, int E);
-cudaError_t launch_chunk_count_scan(const int32_t* idx, int n, int E, int32_t* chunk_base, int32_t* offsets,
-                                    cudaStream_t s);
-cudaError_t launch_chunk_scatter(const int32_t* idx, int n, int E, int k, const int32_t* chunk_base,
-                                 int32_t* perm, int32_t* inv, const __nv_bfloat16* x, int d,
+cudaError_t launch_chunk_scatter(const int32_t* idx, int n, int E, int k, const int32_t* chunk_counts,
+                                 int32_t* offsets, int32_t* perm, int32_t* inv, const __nv_bfloat16* x, int d,
                                  __nv_bfloat16* x_perm, const ZeroArgs& z, cudaStream_t s);
 // Also clears the memory of `z` for the GEMMs that follow on the same stream
 // and writes the y rows of unrouted tokens (`u`).

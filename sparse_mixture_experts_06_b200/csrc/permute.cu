@@ -4,10 +4,11 @@
 //
 //  permute_kernel   histogram -> exclusive scan -> stable scatter, one block
 //                   (moe_permute, and the layer when E x chunks is large)
-//  chunk_count_scan + chunk_scatter   the layer's permutation: per-chunk
-//                   expert counts and their scan in one block, then one block
-//                   per 64-assignment chunk ranks it stably, writes perm / inv
-//                   and copies the x rows to their permuted places
+//  chunk_scatter    the layer's permutation from 2048 assignments: the
+//                   router writes each (expert, 64-assignment chunk) count;
+//                   one block per chunk derives the chunk's first rows from
+//                   the counts, ranks it stably, writes perm / inv and
+//                   copies the x rows to their permuted places
 //  gather_rows      x_perm[r] = x[perm[r] / k]            (bf16 path)
 //  combine_f32      y[t] = (residual[t] +) sum_j obuf[inv[t*k + j]]   (fp32
 //                   path; the bf16 down-projection GEMM does it in its epilogue)
@@ -113,112 +114,71 @@ __device__ __forceinline__ void clear_for_gemms(const ZeroArgs& z) {
 }
 
 // ---- chunked permutation ---------------------------------------------------
-// Assignments q = 0 .. n-1 are cut into chunks of kChunkA.  base[e * nch + c]
-// = the first permuted row of chunk c's assignments to expert e = the
-// exclusive prefix sum, in expert-major order, of the per-(expert, chunk)
-// counts; so offsets[e] = base[e * nch], and inside a chunk the rank of an
-// assignment among the chunk's earlier assignments to the same expert
-// completes its row.  The order is the stable one of permute_kernel
-// (increasing q inside each expert's block), so both give identical bits.
+// Assignments q = 0 .. n-1 are cut into chunks of kChunkA.  The first
+// permuted row of chunk c's assignments to expert e is the exclusive prefix
+// sum, in expert-major order, of the per-(expert, chunk) counts; offsets[e]
+// is that of chunk 0; inside a chunk the rank of an assignment among the
+// chunk's earlier assignments to the same expert completes its row.  The
+// order is the stable one of permute_kernel (increasing q inside each
+// expert's block), so both give identical bits.
 
-constexpr int kScanThreads = 1024;
 constexpr int kScatThreads = 256;
 
-__global__ void __launch_bounds__(kScanThreads)
-chunk_count_scan_kernel(const int32_t* __restrict__ idx, int n, int E, int nch, int32_t* __restrict__ base,
-                        int32_t* __restrict__ offsets) {
-    extern __shared__ int s_cnt[];  // [E * nch], expert-major
-    __shared__ int s_wsum[32];
-    __shared__ int s_carry;
-    pdl_wait();
-    pdl_trigger();
-    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int m = E * nch;
-    for (int i = tid; i < m; i += kScanThreads) s_cnt[i] = 0;
-    if (tid == 0) s_carry = 0;
-    __syncthreads();
-    // counts: one warp per chunk, so each (expert, chunk) cell has one
-    // writer; a warp loads the ids of 4 of its chunks before counting them
-    constexpr int kRounds = kChunkA / 32;
-    constexpr int kBatch = 4;
-    constexpr int kStride = kScanThreads / 32;
-    for (int c0 = warp; c0 < nch; c0 += kBatch * kStride) {
-        int ev[kBatch][kRounds];
-#pragma unroll
-        for (int b = 0; b < kBatch; ++b)
-#pragma unroll
-            for (int r = 0; r < kRounds; ++r) {
-                const int q = (c0 + b * kStride) * kChunkA + r * 32 + lane;
-                ev[b][r] = (c0 + b * kStride < nch && q < n) ? __ldg(idx + q) : -2;  // -2: no assignment
-            }
-#pragma unroll
-        for (int b = 0; b < kBatch; ++b) {
-            const int c = c0 + b * kStride;
-            if (c >= nch) break;  // warp-uniform
-#pragma unroll
-            for (int r = 0; r < kRounds; ++r) {
-                const int e = ev[b][r];
-                const bool valid = (unsigned)e < (unsigned)E;
-                if (e != -2 && !valid) atomicOr(&g_dev_err, 2u);
-                const unsigned peers = __match_any_sync(0xffffffffu, valid ? e : -1);
-                if (valid && (peers & ((1u << lane) - 1u)) == 0) s_cnt[e * nch + c] += __popc(peers);
-            }
-        }
-    }
-    __syncthreads();
-    // exclusive scan of s_cnt in place, kScanThreads cells per pass
-    for (int b0 = 0; b0 < m; b0 += kScanThreads) {
-        const int i = b0 + tid;
-        const int v = i < m ? s_cnt[i] : 0;
-        int x = v;
-#pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-            const int y = __shfl_up_sync(0xffffffffu, x, o);
-            if (lane >= o) x += y;
-        }
-        if (lane == 31) s_wsum[warp] = x;
-        __syncthreads();
-        if (warp == 0) {
-            int w = s_wsum[lane];
-#pragma unroll
-            for (int o = 1; o < 32; o <<= 1) {
-                const int y = __shfl_up_sync(0xffffffffu, w, o);
-                if (lane >= o) w += y;
-            }
-            s_wsum[lane] = w;  // inclusive over warps
-        }
-        __syncthreads();
-        const int excl = s_carry + (warp ? s_wsum[warp - 1] : 0) + x - v;
-        if (i < m) {
-            s_cnt[i] = excl;
-            base[i] = excl;
-        }
-        __syncthreads();
-        if (tid == 0) s_carry += s_wsum[31];
-        __syncthreads();
-    }
-    if (tid < E) offsets[tid] = s_cnt[tid * nch];
-    if (tid == 0) offsets[E] = s_carry;
-}
-
-// Block (chunk c, part): ranks the chunk's assignments; part 0 writes perm
-// and inv; every part copies the x rows of its share of the chunk (bf16
-// path; xp may be null).  The blocks also clear the memory of z.
+// Block (chunk c, part): the chunk's first permuted row per expert from
+// the per-(expert, chunk) counts cnt[e * nch + c] (the router writes them):
+// base(e, c) = (assignments to experts < e) + (assignments to e in chunks
+// < c), sums of integers in a fixed order; block 0 writes the offsets.
+// Then it ranks the chunk's assignments; part 0 writes perm and inv; every
+// part copies the x rows of its share of the chunk (bf16 path; xp may be
+// null).  The blocks also clear the memory of z.
 __global__ void __launch_bounds__(kScatThreads)
 chunk_scatter_kernel(const int32_t* __restrict__ idx, int n, int E, int nch, int k, int parts,
-                     const int32_t* __restrict__ base, int32_t* __restrict__ perm, int32_t* __restrict__ inv,
-                     const __nv_bfloat16* __restrict__ x, int d, __nv_bfloat16* __restrict__ xp,
-                     const ZeroArgs z) {
+                     const int32_t* __restrict__ cnt, int32_t* __restrict__ offsets, int32_t* __restrict__ perm,
+                     int32_t* __restrict__ inv, const __nv_bfloat16* __restrict__ x, int d,
+                     __nv_bfloat16* __restrict__ xp, const ZeroArgs z) {
     constexpr int kRankWarps = kChunkA / 32;
+    constexpr int kWarpsAll = kScatThreads / 32;
     __shared__ int s_wcnt[kRankWarps][kMaxExperts];
     __shared__ int s_pos[kChunkA];
     __shared__ int s_tok[kChunkA];
+    __shared__ int s_before[kMaxExperts];
+    __shared__ int s_total[kMaxExperts];
+    __shared__ int s_base[kMaxExperts];
     const int c = blockIdx.x / parts, part = blockIdx.x - c * parts;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     pdl_wait();
     pdl_trigger();
     clear_for_gemms(z);
     for (int i = tid; i < kRankWarps * kMaxExperts; i += kScatThreads) (&s_wcnt[0][0])[i] = 0;
+    // warp w: experts w, w + 8, ...; its lanes add the expert's counts of the
+    // chunks before c, and of all chunks
+    for (int e = warp; e < E; e += kWarpsAll) {
+        int before = 0, total = 0;
+        for (int cc = lane; cc < nch; cc += 32) {
+            const int v = __ldg(cnt + (size_t)e * nch + cc);
+            total += v;
+            before += cc < c ? v : 0;
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) {
+            before += __shfl_xor_sync(0xffffffffu, before, o);
+            total += __shfl_xor_sync(0xffffffffu, total, o);
+        }
+        if (lane == 0) {
+            s_before[e] = before;
+            s_total[e] = total;
+        }
+    }
+    __syncthreads();
+    if (tid == 0) {
+        int run = 0;
+        for (int e = 0; e < E; ++e) {
+            s_base[e] = run + s_before[e];
+            if (blockIdx.x == 0) offsets[e] = run;
+            run += s_total[e];
+        }
+        if (blockIdx.x == 0) offsets[E] = run;
+    }
     __syncthreads();
     const int q = c * kChunkA + tid;
     int e = -1, rank = 0;
@@ -236,7 +196,7 @@ chunk_scatter_kernel(const int32_t* __restrict__ idx, int n, int E, int nch, int
         if (valid) {
             int before = 0;
             for (int w = 0; w < warp; ++w) before += s_wcnt[w][e];
-            pos = __ldg(base + e * nch + c) + before + rank;
+            pos = s_base[e] + before + rank;
         }
         s_pos[tid] = pos;
         s_tok[tid] = q / k;
@@ -428,31 +388,15 @@ cudaError_t launch_permute(const int32_t* idx, int n, int E, int32_t* offsets, i
 
 // Below 2048 assignments the one-block permutation and the row gather are
 // faster (decode, 64 assignments: 6.6 + 6.6 us vs 6.5 + 8.5 us); above
-// kChunkScanMaxCells (expert, chunk) cells the counts do not fit in shared
-// memory.
+// kChunkScanMaxCells (expert, chunk) cells every scatter block would read
+// that many counts, and the one-block kernel runs instead.
 bool chunked_permute_fits(int n, int E) {
     const long long nch = ((long long)n + kChunkA - 1) / kChunkA;
     return n >= 2048 && (long long)E * nch <= kChunkScanMaxCells;
 }
 
-cudaError_t launch_chunk_count_scan(const int32_t* idx, int n, int E, int32_t* chunk_base, int32_t* offsets,
-                                    cudaStream_t s) {
-    static bool attr_done[64] = {false};
-    int dev = 0;
-    cudaGetDevice(&dev);
-    if (dev < 64 && !attr_done[dev]) {
-        cudaError_t e = cudaFuncSetAttribute(chunk_count_scan_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             (int)(kChunkScanMaxCells * sizeof(int)));
-        if (e != cudaSuccess) return e;
-        attr_done[dev] = true;
-    }
-    const int nch = (n + kChunkA - 1) / kChunkA;
-    return launch_pdl(chunk_count_scan_kernel, 1, kScanThreads, (size_t)E * nch * sizeof(int), s, idx, n, E, nch,
-                      chunk_base, offsets);
-}
-
-cudaError_t launch_chunk_scatter(const int32_t* idx, int n, int E, int k, const int32_t* chunk_base,
-                                 int32_t* perm, int32_t* inv, const __nv_bfloat16* x, int d,
+cudaError_t launch_chunk_scatter(const int32_t* idx, int n, int E, int k, const int32_t* chunk_counts,
+                                 int32_t* offsets, int32_t* perm, int32_t* inv, const __nv_bfloat16* x, int d,
                                  __nv_bfloat16* x_perm, const ZeroArgs& z, cudaStream_t s) {
     const int nch = (n + kChunkA - 1) / kChunkA;
     // about two blocks per SM: split each chunk's row copies over `parts` blocks
@@ -460,8 +404,8 @@ cudaError_t launch_chunk_scatter(const int32_t* idx, int n, int E, int k, const 
     int parts = (want + nch - 1) / nch;
     parts = parts < 1 ? 1 : (parts > 8 ? 8 : parts);
     if (!x_perm) parts = 1;
-    return launch_pdl(chunk_scatter_kernel, nch * parts, kScatThreads, 0, s, idx, n, E, nch, k, parts, chunk_base,
-                      perm, inv, x, d, x_perm, z);
+    return launch_pdl(chunk_scatter_kernel, nch * parts, kScatThreads, 0, s, idx, n, E, nch, k, parts, chunk_counts,
+                      offsets, perm, inv, x, d, x_perm, z);
 }
 
 cudaError_t launch_gather_rows_bf16(const __nv_bfloat16* x, const int32_t* perm, int rows, int d,

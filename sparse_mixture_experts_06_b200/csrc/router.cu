@@ -143,14 +143,42 @@ __device__ __forceinline__ void permute_in_cta(const int32_t* idx, int n, int E,
     }
 }
 
+// The expert counts of the 64-assignment chunks of this cluster's tokens
+// (tokens tok0 .. tok0+63, i.e. assignments tok0*k .. (tok0+64)*k: exactly k
+// chunks, the last one cut at n), done by CTA 0 after every CTA's indices
+// are visible: cnt[e * nch + c] for each of those chunks c and every expert
+// e (zeros included), so every cell has one writer and nothing needs
+// clearing.  smem is the CTA's scratch: [k][E] counters.
+__device__ __forceinline__ void count_chunks_in_cta(const int32_t* idx, int tok0, int T, int E, int k, int nch,
+                                                    int32_t* cnt, int* smem) {
+    const int q0 = tok0 * k, q1 = min(T, tok0 + kTokBlock) * k;
+    const int c0 = q0 / kChunkA, c1 = (q1 + kChunkA - 1) / kChunkA;  // q0 is a multiple of kChunkA
+    const int cells = (c1 - c0) * E;
+    for (int i = threadIdx.x; i < cells; i += kWarps * 32) smem[i] = 0;
+    __syncthreads();
+    for (int q = q0 + (int)threadIdx.x; q < q1; q += kWarps * 32) {
+        const int e = __ldcg(idx + q);  // written by other CTAs of the cluster
+        atomicAdd(&smem[((q - q0) / kChunkA) * E + e], 1);
+    }
+    __syncthreads();
+    for (int i = threadIdx.x; i < cells; i += kWarps * 32) {
+        const int c = i / E, e = i - c * E;
+        cnt[(size_t)e * nch + c0 + c] = smem[i];
+    }
+}
+
 template <bool BF16>
 __global__ void __launch_bounds__(kWarps * 32, BF16 ? 4 : 2)  // bf16: 64 registers, 4 CTAs per SM
 router_topk_kernel(const void* __restrict__ x, const void* __restrict__ Wg, int T, int d, int E, int k,
                    int32_t* __restrict__ idx_out, float* __restrict__ w_out, int32_t* __restrict__ offsets,
-                   int32_t* __restrict__ perm, int32_t* __restrict__ inv) {
+                   int32_t* __restrict__ perm, int32_t* __restrict__ inv, int32_t* __restrict__ chunk_counts,
+                   int nch) {
     extern __shared__ __align__(16) unsigned char smem_raw[];
     pdl_wait();     // x may be the previous kernel's output (a layer stack)
-    pdl_trigger();
+    // The next kernel may start early, except the chunked permutation's
+    // scatter (one block per chunk): its waiting blocks would take the
+    // registers of this one-wave grid's CTAs; it starts as these CTAs exit.
+    if (chunk_counts == nullptr) pdl_trigger();
     double* wfrag = reinterpret_cast<double*>(smem_raw);  // [kChunks][8][32]
     double* part = wfrag + kFragDoubles;                  // [kTokBlock][E]
     cg::cluster_group cluster = cg::this_cluster();
@@ -297,12 +325,15 @@ router_topk_kernel(const void* __restrict__ x, const void* __restrict__ Wg, int 
     if (perm != nullptr) {  // one cluster holds every token: the permutation here too
         cluster.sync();     // every CTA's indices are written and visible in the cluster
         if (rank == 0) permute_in_cta(idx_out, T * k, E, offsets, perm, inv, reinterpret_cast<int*>(wfrag));
+    } else if (chunk_counts != nullptr) {  // a chunked permutation follows: this cluster's chunk counts
+        cluster.sync();
+        if (rank == 0) count_chunks_in_cta(idx_out, tok0, T, E, k, nch, chunk_counts, reinterpret_cast<int*>(wfrag));
     }
 }
 
 template <bool BF16>
 cudaError_t launch_impl(const void* x, const void* Wg, int T, int d, int E, int k, int32_t* idx, float* w,
-                        const PermuteOut& po, cudaStream_t s) {
+                        const RouterOut& ro, cudaStream_t s) {
     static bool attr_done[64] = {false};
     int dev = 0;
     cudaGetDevice(&dev);
@@ -326,9 +357,11 @@ cudaError_t launch_impl(const void* x, const void* Wg, int T, int d, int E, int 
     cfg.stream = s;
     cfg.attrs = attr;
     cfg.numAttrs = 2;
-    const bool fuse = po.perm != nullptr && router_can_permute(T, k);
+    const bool fuse = ro.perm != nullptr && router_can_permute(T, k);
+    const int nch = (int)(((long long)T * k + kChunkA - 1) / kChunkA);
     return cudaLaunchKernelEx(&cfg, router_topk_kernel<BF16>, x, Wg, T, d, E, k, idx, w,
-                              fuse ? po.offsets : nullptr, fuse ? po.perm : nullptr, fuse ? po.inv : nullptr);
+                              fuse ? ro.offsets : nullptr, fuse ? ro.perm : nullptr, fuse ? ro.inv : nullptr,
+                              fuse ? nullptr : ro.chunk_counts, nch);
 }
 
 }  // namespace
@@ -336,9 +369,9 @@ cudaError_t launch_impl(const void* x, const void* Wg, int T, int d, int E, int 
 bool router_can_permute(int T, int k) { return T >= 1 && T <= kTokBlock && (long long)T * k <= kFusedPermute; }
 
 cudaError_t launch_router_topk(const void* x, const void* Wg, int T, int d, int E, int k,
-                               bool bf16, int32_t* idx, float* w, cudaStream_t s, const PermuteOut& po) {
-    return bf16 ? launch_impl<true>(x, Wg, T, d, E, k, idx, w, po, s)
-                : launch_impl<false>(x, Wg, T, d, E, k, idx, w, po, s);
+                               bool bf16, int32_t* idx, float* w, cudaStream_t s, const RouterOut& ro) {
+    return bf16 ? launch_impl<true>(x, Wg, T, d, E, k, idx, w, ro, s)
+                : launch_impl<false>(x, Wg, T, d, E, k, idx, w, ro, s);
 }
 
 }  // namespace moe

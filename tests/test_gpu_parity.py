@@ -186,9 +186,9 @@ def workspace_routing_views(ws, T, E, k):
 ], ids=lambda s: s.name)
 def test_layer_permutation_matches_the_stable_sort(shape):
     """The permutation the layer builds for itself (in the router's cluster
-    up to 64 tokens and 256 assignments, else chunked count/scan + scatter,
-    or the one-block kernel for few assignments or when E x chunks is too
-    large) equals
+    up to 64 tokens and 256 assignments; from 2048 assignments from the
+    router's per-chunk counts in the scatter; else, or when E x chunks is
+    too large, the one-block kernel) equals
     the oracle's stable counting sort of the router's choices, bit for bit,
     and the layer's output on sampled tokens matches the oracle."""
     t = device_inputs(shape, 31)
@@ -397,14 +397,14 @@ def test_entry_points_agree_and_are_deterministic():
     moe.moe_release_workspace()
 
 
-@pytest.mark.parametrize("T,kernels", [(32, 4), (100, 5), (2304, 5)],
+@pytest.mark.parametrize("T,kernels", [(32, 4), (100, 5), (2304, 4)],
                          ids=["router-permutes", "one-block-permutation", "chunked-permutation"])
 def test_bf16_layer_kernels(T, kernels):
-    """The bf16 layer is router, permutation (count/scan or one block), row
-    scatter or gather, up-projection GEMM and down-projection GEMM: the
-    combine runs in the down GEMM's epilogue, with no kernel of its own.  Up
-    to 64 tokens (one router cluster) the router writes the permutation too:
-    four kernels."""
+    """The bf16 layer is router, one-block permutation and row gather, up-
+    projection GEMM and down-projection GEMM: the combine runs in the down
+    GEMM's epilogue, with no kernel of its own.  Up to 64 tokens (one router
+    cluster) the router writes the permutation, and from 2048 assignments
+    the per-chunk counts for the row scatter: four kernels."""
     s = synth.MoEShape("launches", T, 256, 512, 8, 2, "bf16")
     t = device_inputs(s, 3)
     ws = torch.empty(moe.moe_workspace_size(T, s.d, s.f, s.E, s.k, 0), dtype=torch.uint8, device="cuda")
@@ -419,7 +419,7 @@ def test_bf16_layer_kernels(T, kernels):
     n = {name: cnt for name, (_, cnt) in prof.items()}
     assert n["combine"] == 0 and n["down_combine_gemm"] == 1 and n["up_swiglu_gemm"] == 1
     assert sum(n.values()) == kernels, n
-    assert n["permute"] == (0 if kernels == 4 else 1)
+    assert n["permute"] == (0 if kernels == 4 else 1) and n["gather_rows"] == 1
     h = host_copy(t)
     y_ref, _, _ = oracle_rows(h, 2, np.arange(T))
     assert_close(to64(y), y_ref, "bf16")
