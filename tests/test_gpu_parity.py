@@ -222,6 +222,8 @@ BF16_SHAPES = [
     synth.MoEShape("bf16-many-tiles", 2500, 256, 768, 8, 2, "bf16"),  # 625 rows/expert, 2-3 pair tiles
     synth.MoEShape("bf16-k-eq-E", 150, 128, 256, 8, 8, "bf16"),       # K = E: dense softmax mixture
     synth.MoEShape("bf16-E16k12", 120, 128, 256, 16, 12, "bf16"),
+    synth.MoEShape("bf16-wide-d", 200, 8192, 512, 8, 2, "bf16"),      # up K = 8192, down 16+ column tiles
+    synth.MoEShape("bf16-deep-f", 200, 128, 28672, 8, 2, "bf16"),     # down K = 28672 (448 k blocks)
 ]
 
 
