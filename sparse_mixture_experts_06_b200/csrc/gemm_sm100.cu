@@ -4,8 +4,10 @@
 //         SwiGLU expert):  for every permuted row r of expert e,
 //         a = W1_e x_r, b = W3_e x_r (fp32 in tensor memory),
 //         h_r = SiLU(a) * b rounded to bf16.
-//   down (second half and the gate weighting of §2.1 display 3):
-//         obuf_r = topk_w[perm[r]] * (W2_e h_r), fp32.
+//   down (second half, the gate weighting and the scatter-back of §2.1
+//         display 3): obuf_r = topk_w[perm[r]] * (W2_e h_r), fp32, parked;
+//         the last of a token's slot rows to arrive (per 128 output
+//         columns) adds the parked rows in slot order into y[t] (bf16).
 //
 // Both are one persistent, warp-specialised kernel (320 threads per CTA):
 //   warp 0      TMA producer: 2-D tiled bulk copies (128-byte swizzle) of the
@@ -47,11 +49,14 @@
 // A rows and B columns least (G x A-tile + P / G x B-tile, with the A and B
 // tiles' bytes in proportion to their rows); an expert of at most G row
 // blocks is one group (every expert at T = 4096 on Mixtral shapes; at
-// T = 16384 with skewed routing the hottest expert has 45).  Tiles are handed out
-// dynamically: the producer (the even CTA's, for pairs) takes the next tile
-// number from a global counter and passes it to the other roles (and to the
-// odd CTA) through a small shared-memory ring, so short and full tiles
-// balance across the persistent CTAs.  Ragged row blocks read the
+// T = 16384 with skewed routing the hottest expert has 45).  The down
+// projection numbers its short pair tiles after all others.  Tiles are
+// handed out dynamically: the producer (the even CTA's, for pairs) takes
+// the next tile number from a global counter and passes it to the other
+// roles (and to the odd CTA) through a small shared-memory ring, so short
+// and full tiles balance across the persistent CTAs.  Weight-streaming
+// launches (32-row tiles) run in even waves and start their first weight
+// loads before the dependency wait (see below).  Ragged row blocks read the
 // next expert's rows (or the zero fill past the end) and simply do not
 // store them; ragged column blocks are masked the same way.
 //
