@@ -253,8 +253,10 @@ def test_layer_parity_every_token_bf16(shape, variant):
 
 # Expert block sizes around every tile edge: pair tiles are 256 rows, or 128
 # (an M = 128 pair MMA, 64 rows per CTA) when an expert's last block holds at
-# most 128 rows; single-CTA tiles are 128 rows.
-BLOCK_SIZES = [1, 64, 65, 128, 129, 200, 384, 385]
+# most 128 rows; in the up projection's 256 x 512 pair tiles such a tail after
+# a whole block is merged with it (257, 320, 321, 384, 640: tails of 1, 64,
+# 65 and 128 rows); single-CTA tiles are 128 rows.
+BLOCK_SIZES = [1, 64, 65, 128, 129, 200, 257, 320, 321, 384, 385, 640]
 
 
 @pytest.mark.parametrize("cta_group,wide", [("1", "0"), ("2", "0"), ("2", "1"), ("h", "0")])
