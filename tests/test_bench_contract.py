@@ -83,3 +83,16 @@ def test_clock_sampler_reads_the_benchmarked_gpu_through_nvml(monkeypatch):
     assert c["samples"] >= 2 and c["sm_mhz"] == 1500.0 and c["sm_max_mhz"] == 1965.0
     assert c["reasons"] == ["sw_power_cap"] and c["power_w_max"] == 998.0
     assert "NVML" in c["source"]
+
+
+def test_roofline_peak_follows_the_sampled_clock_regime():
+    """The up GEMM's roofline is held to the sustained bf16 figure when the
+    clock sampled during the timed steps was held well below its maximum (the
+    power cap over a long run), to the burst figure at full clock or when no
+    clock was sampled."""
+    import bench
+    assert bench.clock_regime(None) == "burst"
+    assert bench.clock_regime({"sm_mhz": 1965.0, "sm_max_mhz": 1965.0, "reasons": []}) == "burst"
+    assert bench.clock_regime({"sm_mhz": 1850.0, "sm_max_mhz": 1965.0, "reasons": ["sw_power_cap"]}) == "burst"
+    assert bench.clock_regime({"sm_mhz": 1455.0, "sm_max_mhz": 1965.0, "reasons": ["sw_power_cap"]}) == "sustained"
+    assert bench.clock_regime({"sm_mhz": None, "sm_max_mhz": 1965.0}) == "burst"
