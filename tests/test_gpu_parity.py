@@ -503,8 +503,10 @@ def test_decode_full_shape_every_token(mixtral_weights):
     big_check("decode", mixtral_weights, None)
 
 
-def test_prefill_full_shape(mixtral_weights):
-    big_check("prefill", mixtral_weights, 256)
+def test_prefill_full_shape_every_token(mixtral_weights):
+    """The headline workload (T = 4096, Mixtral dimensions, the default
+    256 x 512 pair tiles) against the oracle on all 4096 tokens."""
+    big_check("prefill", mixtral_weights, None)
 
 
 @pytest.mark.parametrize("name,cta_group,bn,rb,wide", [
@@ -513,13 +515,16 @@ def test_prefill_full_shape(mixtral_weights):
     ("prefill", "1", "128", "128", "0"), ("prefill", "2", "256", "128", "0"), ("prefill", "2", "256", "128", "1"),
     ("prefill", "1", "256", "128", "0"), ("prefill", "1", "256", "32", "0")])
 def test_full_shapes_other_gemm_variant(name, cta_group, bn, rb, wide, mixtral_weights):
-    """Variants the size heuristics do not pick, at the full shapes."""
+    """Variants the size heuristics do not pick, at the full shapes, on
+    every token."""
     force_variant(cta_group, bn, rb, wide)
-    big_check(name, mixtral_weights, None if name == "decode" else 256)
+    big_check(name, mixtral_weights, None)
 
 
-def test_skewed_full_shape(mixtral_weights):
-    _, counts = big_check("skewed", mixtral_weights, 256)
+def test_skewed_full_shape_every_token(mixtral_weights):
+    """T = 16384 with the skewed router (hottest expert 35 %, 45 pair row
+    blocks, several groups of the tile order) on every token."""
+    _, counts = big_check("skewed", mixtral_weights, None)
     share = counts / counts.sum()
     assert abs(share[0] - 0.35) < 0.005 and (np.diff(share) < 0).all()
 
