@@ -503,6 +503,13 @@ def test_decode_full_shape_every_token(mixtral_weights):
     big_check("decode", mixtral_weights, None)
 
 
+def test_decode_full_shape_f32_every_token():
+    """The fp32 layer (router, permutation, fp32 expert kernels, combine) at
+    Mixtral dimensions (T = 32, d = 4096, f = 14336: 5.6 GB of fp32 expert
+    weights), every token within the fp32 bound."""
+    full_check(synth.MoEShape("decode-f32", 32, 4096, 14336, 8, 2, "f32"), 3)
+
+
 def test_prefill_full_shape_every_token(mixtral_weights):
     """The headline workload (T = 4096, Mixtral dimensions, the default
     256 x 512 pair tiles) against the oracle on all 4096 tokens."""
