@@ -528,6 +528,26 @@ def test_full_shapes_other_gemm_variant(name, cta_group, bn, rb, wide, mixtral_w
     big_check(name, mixtral_weights, None)
 
 
+def test_top4_at_mixtral_dimensions_every_token(mixtral_weights):
+    """k = 4 of E = 8 at d = 4096, f = 14336 (the Mixtral expert weights),
+    T = 1024: 4096 assignments, so the chunked permutation and CTA-pair tiles
+    run, and the combine adds slots 2 and 3 through inv; routing, permutation
+    and outputs against the oracle on every token."""
+    s = synth.MoEShape("top4", 1024, 4096, 14336, 8, 4, "bf16")
+    tw, hw = mixtral_weights
+    t = device_inputs(synth.MoEShape(s.name, s.T, s.d, 8, s.E, s.k, s.dtype), 5)
+    t = {"x": t["x"], "Wg": t["Wg"], "W1": tw["W1"], "W3": tw["W3"], "W2": tw["W2"]}
+    y = run_layer(t, s.k)
+    idx_g, w_g = moe.moe_router_topk(t["x"], t["Wg"], s.k)
+    off_g, perm_g, inv_g = moe.moe_permute(idx_g, s.E)
+    torch.cuda.synchronize()
+    h = dict(hw, x=to_bits(t["x"]), Wg=to_bits(t["Wg"]))
+    idx_o, _, _ = check_routing(idx_g.cpu().numpy(), w_g.cpu().numpy(), f64(h["x"]), f64(h["Wg"]), s.k)
+    check_permutation(off_g.cpu().numpy(), perm_g.cpu().numpy(), inv_g.cpu().numpy(), idx_o, s.E)
+    y_ref, _, _ = oracle_rows(h, s.k, np.arange(s.T))
+    assert_close(to64(y), y_ref, "bf16")
+
+
 def test_skewed_full_shape_every_token(mixtral_weights):
     """T = 16384 with the skewed router (hottest expert 35 %, 45 pair row
     blocks, several groups of the tile order) on every token."""
