@@ -115,12 +115,18 @@ def test_host_layer_chained_through_host_memory():
     assert torch.equal(out.view(torch.int16), y2.cpu().view(torch.int16))
 
 
-def test_host_layer_prefill_shape_two_chunks():
+@pytest.mark.parametrize("chunks", [1, 2])
+def test_host_layer_prefill_shape(chunks):
+    """The serving entry at the bench's end-to-end size (T = 4096, Mixtral
+    dimensions, pinned host buffers; the bench uses one piece): the bits of
+    the device entry point on the same split, which the full-shape tests
+    check against the oracle."""
     s = synth.CONFIGS["prefill"]
     t = device_inputs(s, 0)
     x_h = t["x"].cpu().pin_memory()
-    y_h = moe.moe_layer_forward_host(x_h, t["Wg"], t["W1"], t["W3"], t["W2"], s.k, chunks=2)
+    y_h = moe.moe_layer_forward_host(x_h, t["Wg"], t["W1"], t["W3"], t["W2"], s.k, chunks=chunks)
     torch.cuda.current_stream().synchronize()
-    ref = piecewise_device(t, s.k, 2).cpu()
+    ref = piecewise_device(t, s.k, chunks).cpu()
     assert torch.equal(y_h.view(torch.int16), ref.view(torch.int16))
     moe.moe_release_workspace()
+
