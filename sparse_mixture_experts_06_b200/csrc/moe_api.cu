@@ -1,7 +1,10 @@
 // C ABI of the sparse MoE layer (declared in include/moe.h): argument
 // validation, workspace layout, and the launch sequence
-//   bf16: router_topk -> permute -> [gather] -> up GEMM -> down GEMM (+ combine)
-//   fp32: router_topk -> permute -> fp32 expert kernels -> combine
+//   bf16: router_topk (with the permutation up to 64 tokens, or the
+//         per-chunk expert counts from 2048 assignments) -> [permute] ->
+//         row gather (or the chunked scatter) -> up GEMM -> down GEMM with
+//         the combine in its epilogue
+//   fp32: router_topk -> [permute] -> fp32 expert kernels -> combine
 // on the caller's stream.  Nothing here waits on the device.
 
 #include <cstdarg>
