@@ -4,7 +4,8 @@
 //         per-chunk expert counts from 2048 assignments) -> [permute] ->
 //         row gather (or the chunked scatter) -> up GEMM -> down GEMM with
 //         the combine in its epilogue
-//   fp32: router_topk -> [permute] -> fp32 expert kernels -> combine
+//   fp32: router_topk -> [permute or the chunked scatter] -> fp32 expert
+//         kernels -> combine
 // on the caller's stream.  Nothing here waits on the device.
 
 #include <cstdarg>
