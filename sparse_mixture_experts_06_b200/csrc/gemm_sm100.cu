@@ -1368,10 +1368,10 @@ cudaError_t launch_gemm(const GroupedGemmArgs& a, const CUtensorMap& mA, const C
     KParams p = p0;
     p.wait_limit_ns = g_wait_limit_ns.load(std::memory_order_relaxed);
     p.stall_test = g_stall_test.load(std::memory_order_relaxed);
-    static int units_cache[64] = {0};
+    static std::atomic<int> units_cache[64];  // per device and variant; any thread may fill it (same value)
     int dev = 0;
     cudaGetDevice(&dev);
-    int units = (dev < 64) ? units_cache[dev] : 0;
+    int units = (dev < 64) ? units_cache[dev].load(std::memory_order_relaxed) : 0;
     cudaLaunchConfig_t cfg = {};
     cudaLaunchAttribute attr[2];
     cfg.blockDim = dim3(NUM_THREADS);
@@ -1399,7 +1399,7 @@ cudaError_t launch_gemm(const GroupedGemmArgs& a, const CUtensorMap& mA, const C
                 units = clusters;
             cudaGetLastError();  // an unsupported query is not an error for the launch
         }
-        if (dev < 64) units_cache[dev] = units;
+        if (dev < 64) units_cache[dev].store(units, std::memory_order_relaxed);
     }
     const long long ub = (long long)p.n_tiles * ((a.rows + C::kTileRows - 1) / C::kTileRows + a.E);
     const int grid_units = (int)(ub < units ? ub : units);

@@ -8,6 +8,7 @@
 //         kernels -> combine
 // on the caller's stream.  Nothing here waits on the device.
 
+#include <atomic>
 #include <cstdarg>
 #include <cstdio>
 #include <mutex>
@@ -40,14 +41,17 @@ bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) ==
 size_t align256(size_t v) { return (v + 255) & ~size_t(255); }
 
 int num_sms_current() {
-    static int cache[64] = {0};
+    static std::atomic<int> cache[64];  // per device; any thread may fill it (same value)
     int dev = 0;
     cudaGetDevice(&dev);
-    if (dev < 64 && cache[dev]) return cache[dev];
+    if (dev < 64) {
+        const int c = cache[dev].load(std::memory_order_relaxed);
+        if (c) return c;
+    }
     int sms = 0;
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
     if (sms <= 0) sms = 148;
-    if (dev < 64) cache[dev] = sms;
+    if (dev < 64) cache[dev].store(sms, std::memory_order_relaxed);
     return sms;
 }
 

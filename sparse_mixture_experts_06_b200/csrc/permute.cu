@@ -22,6 +22,8 @@
 // the number of lower lanes in its group; a per-tile exclusive scan over the
 // 32 warps gives each warp's base inside the expert's block.
 
+#include <atomic>
+
 #include "moe_internal.cuh"
 
 namespace moe {
@@ -347,14 +349,14 @@ cudaError_t launch_pdl(void (*kernel)(KArgs...), int grid, int block, size_t sme
 // Grid for a row kernel over `items` rows: one block per row, capped at 8
 // resident blocks per SM (the kernels loop with a grid stride).
 int flat_grid(long long items) {
-    static int sms_cache[64] = {0};
+    static std::atomic<int> sms_cache[64];  // per device; any thread may fill it (same value)
     int dev = 0;
     cudaGetDevice(&dev);
-    int sms = (dev < 64) ? sms_cache[dev] : 0;
+    int sms = (dev < 64) ? sms_cache[dev].load(std::memory_order_relaxed) : 0;
     if (!sms) {
         cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
         if (sms <= 0) sms = 148;
-        if (dev < 64) sms_cache[dev] = sms;
+        if (dev < 64) sms_cache[dev].store(sms, std::memory_order_relaxed);
     }
     const long long need = items;
     const long long cap = (long long)sms * 8;

@@ -33,6 +33,8 @@
 // logits.  The split changes the summation order but not the rule:
 // logits are fp64 sums of exact products.
 
+#include <atomic>
+
 #include <cooperative_groups.h>
 
 #include "moe_internal.cuh"
@@ -334,14 +336,14 @@ router_topk_kernel(const void* __restrict__ x, const void* __restrict__ Wg, int 
 template <bool BF16>
 cudaError_t launch_impl(const void* x, const void* Wg, int T, int d, int E, int k, int32_t* idx, float* w,
                         const RouterOut& ro, cudaStream_t s) {
-    static bool attr_done[64] = {false};
+    static std::atomic<bool> attr_done[64];  // per device; setting the attribute twice is harmless
     int dev = 0;
     cudaGetDevice(&dev);
-    if (dev < 64 && !attr_done[dev]) {
+    if (dev >= 64 || !attr_done[dev].load(std::memory_order_relaxed)) {
         cudaError_t e = cudaFuncSetAttribute(router_topk_kernel<BF16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                              (int)router_smem_bytes(kMaxExperts));
         if (e != cudaSuccess) return e;
-        attr_done[dev] = true;
+        if (dev < 64) attr_done[dev].store(true, std::memory_order_relaxed);
     }
     const int blocks = (T + kTokBlock - 1) / kTokBlock;
     cudaLaunchConfig_t cfg = {};
