@@ -366,13 +366,16 @@ int flat_grid(long long items) {
 }  // namespace
 
 unsigned int* device_error_word() {
-    static unsigned int* cache[64] = {nullptr};
+    static std::atomic<unsigned int*> cache[64];  // per device; any thread may fill it (same value)
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) return nullptr;
-    if (dev < 64 && cache[dev]) return cache[dev];
+    if (dev < 64) {
+        unsigned int* c = cache[dev].load(std::memory_order_relaxed);
+        if (c) return c;
+    }
     void* p = nullptr;
     if (cudaGetSymbolAddress(&p, g_dev_err) != cudaSuccess) return nullptr;
-    if (dev < 64) cache[dev] = static_cast<unsigned int*>(p);
+    if (dev < 64) cache[dev].store(static_cast<unsigned int*>(p), std::memory_order_relaxed);
     return static_cast<unsigned int*>(p);
 }
 
